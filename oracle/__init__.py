@@ -1,0 +1,253 @@
+"""fp64 CPU oracle for the exact attention forward pass.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package.  It shares no code
+with the CUDA library and never imports it.
+
+Contents
+--------
+``attention``            the definition (three steps, two-pass softmax) in plain C,
+                         fp64, threaded over rows (``attn_oracle.c``).
+``attention_online``     a numpy fp64 re-statement of the tiled algorithm with a
+                         running max ``m`` and running sum ``l`` rescaled per key
+                         block, used only to cross-check ``attention``.
+``probabilities``        the materialised probability matrix P (numpy fp64), for
+                         the row-sum invariant.
+``attention_loops``      pure-Python loops for tiny inputs (brute force).
+
+Sources: "FlashAttention technical analysis" (jsqmd.com/news/722897) section 2.1
+(the three steps), section 2.2 (tiling plus online softmax with running max and
+sum), section 3.3 (only the O(N) statistics are kept) and section 6.2 (two-pass
+safe softmax); "Flash Attention in a production Stable-Diffusion service"
+(xxmr.cn/news/81028) section 2.3 (order: QK^T, scale, add mask, softmax, PV).
+
+Readings where the pages are silent: see the header of ``attn_oracle.c``; the
+numpy variants below follow the same readings.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "attn_oracle.c")
+_LIB_DIR = os.path.join(_HERE, "_build")
+_LIB = os.path.join(_LIB_DIR, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``attn_oracle.c`` into ``_build/liboracle.so`` with gcc (no fast-math)."""
+    os.makedirs(_LIB_DIR, exist_ok=True)
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math",
+             "-ffp-contract=off", "-o", tmp, _SRC, "-lm", "-lpthread"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _bind(path):
+    lib = ctypes.CDLL(path)
+    dp = ctypes.POINTER(ctypes.c_double)
+    ip = ctypes.POINTER(ctypes.c_int32)
+    lib.oracle_attention_fwd.restype = ctypes.c_int
+    lib.oracle_attention_fwd.argtypes = [
+        dp, dp, dp, dp, dp,
+        ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+        ctypes.c_double, ctypes.c_int,
+        ip, dp, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+        ip, ctypes.c_int, ctypes.c_int]
+    lib.oracle_default_threads.restype = ctypes.c_int
+    return lib
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            _lib = _bind(build())
+    return _lib
+
+
+def compile_variant(src_text: str, out_path: str):
+    """Compile a modified copy of the oracle source to ``out_path`` and return a
+    loaded handle for ``attention(..., lib=handle)``.  Used only by the tests that
+    plant a mistake in the oracle to show that the pins catch it."""
+    c_path = out_path + ".c"
+    with open(c_path, "w") as f:
+        f.write(src_text)
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math",
+                           "-ffp-contract=off", "-o", out_path, c_path, "-lm", "-lpthread"])
+    return _bind(out_path)
+
+
+def source_text() -> str:
+    with open(_SRC) as f:
+        return f.read()
+
+
+def default_threads() -> int:
+    return int(_load().oracle_default_threads())
+
+
+def _f64(x) -> np.ndarray:
+    """Exact conversion of a CPU tensor / array to a contiguous fp64 numpy array."""
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            x = x.detach().to("cpu", torch.float64).numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a, ctype=ctypes.c_double):
+    return a.ctypes.data_as(ctypes.POINTER(ctype)) if a is not None else None
+
+
+def _mask_view(mask, B, Hq, Nq, Nk):
+    """Return (fp64 array, sb, sh, sq) for a mask broadcastable to [B, Hq, Nq, Nk]."""
+    m = np.asarray(mask, dtype=np.float64)
+    while m.ndim < 4:
+        m = m[None]
+    m = np.broadcast_to(m, (B, Hq, Nq, Nk))
+    base = np.ascontiguousarray(m[:, :, :, :])  # materialise (tests only; sizes are small)
+    return base, Hq * Nq * Nk, Nq * Nk, Nk
+
+
+def attention(q, k, v, *, scale: float | None = None, is_causal: bool = False,
+              key_lens=None, mask=None, rows=None, n_threads: int = 0, lib=None):
+    """The definition, in fp64.
+
+    q: [B, Hq, Nq, d]; k, v: [B, Hkv, Nk, d]; key_lens: [B] ints or None;
+    mask: additive mask broadcastable to [B, Hq, Nq, Nk] or None;
+    rows: optional list of query indices computed in every head (others are NaN).
+    Returns (O [B, Hq, Nq, d] fp64, LSE [B, Hq, Nq] fp64).
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Hq, Nq, d = q.shape
+    _, Hkv, Nk, _ = k.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    out = np.full((B, Hq, Nq, d), np.nan)
+    lse = np.full((B, Hq, Nq), np.nan)
+    kl = None if key_lens is None else np.ascontiguousarray(np.asarray(key_lens, dtype=np.int32))
+    rw = None if rows is None else np.ascontiguousarray(np.asarray(rows, dtype=np.int32))
+    mk, sb, sh, sq = (None, 0, 0, 0) if mask is None else _mask_view(_f64(mask), B, Hq, Nq, Nk)
+    rc = (lib or _load()).oracle_attention_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+        B, Hq, Hkv, Nq, Nk, d, float(scale), int(bool(is_causal)),
+        _ptr(kl, ctypes.c_int32), _ptr(mk), sb, sh, sq,
+        _ptr(rw, ctypes.c_int32), 0 if rw is None else len(rw), int(n_threads))
+    if rc != 0:
+        raise ValueError(f"oracle_attention_fwd rejected its arguments (status {rc})")
+    return out, lse
+
+
+def _masked_scores(q, k, scale, is_causal, key_lens, mask):
+    """Scaled scores with masked positions at -inf, [B, Hq, Nq, Nk] fp64 (numpy)."""
+    B, Hq, Nq, d = q.shape
+    _, Hkv, Nk, _ = k.shape
+    group = Hq // Hkv
+    kk = np.repeat(k, group, axis=1)  # query head h reads K/V head h // group
+    s = scale * np.einsum("bhid,bhjd->bhij", q, kk)
+    if mask is not None:
+        s = s + np.broadcast_to(np.asarray(mask, dtype=np.float64), s.shape)
+    j = np.arange(Nk)
+    if key_lens is not None:
+        kl = np.asarray(key_lens).reshape(B, 1, 1, 1)
+        s = np.where(j[None, None, None, :] >= kl, -np.inf, s)
+    if is_causal:
+        i = np.arange(Nq)
+        s = np.where(j[None, :] > i[:, None], -np.inf, s)
+    return s
+
+
+def probabilities(q, k, *, scale=None, is_causal=False, key_lens=None, mask=None):
+    """Materialised softmax matrix P [B, Hq, Nq, Nk] (fp64); fully masked rows are 0."""
+    q, k = _f64(q), _f64(k)
+    if scale is None:
+        scale = 1.0 / math.sqrt(q.shape[-1])
+    s = _masked_scores(q, k, scale, is_causal, key_lens, mask)
+    m = s.max(axis=-1, keepdims=True)
+    safe_m = np.where(np.isneginf(m), 0.0, m)
+    p = np.exp(s - safe_m)
+    l = p.sum(axis=-1, keepdims=True)
+    return np.where(l > 0, p / np.where(l > 0, l, 1.0), 0.0)
+
+
+def attention_online(q, k, v, *, block: int, scale=None, is_causal=False, key_lens=None, mask=None):
+    """Tiled re-statement: loop over key blocks of size ``block`` keeping, per row,
+    a running max m, a running sum l and an unnormalised accumulator acc; when a
+    block raises the max, rescale l and acc by exp(m_old - m_new); divide once at
+    the end (jsqmd.com/news/722897 section 2.2 and the deferred rescaling of
+    section 4.1).  fp64, numpy, tiny inputs only.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Hq, Nq, d = q.shape
+    _, Hkv, Nk, _ = k.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    group = Hq // Hkv
+    vv = np.repeat(v, group, axis=1)
+    s_all = _masked_scores(q, k, scale, is_causal, key_lens, mask)
+    m = np.full((B, Hq, Nq), -np.inf)
+    l = np.zeros((B, Hq, Nq))
+    acc = np.zeros((B, Hq, Nq, d))
+    for j0 in range(0, Nk, block):
+        s = s_all[..., j0:j0 + block]
+        m_new = np.maximum(m, s.max(axis=-1))
+        # rows that have seen no unmasked key keep m = -inf; use 0 as the shift there
+        shift = np.where(np.isneginf(m_new), 0.0, m_new)
+        alpha = np.where(np.isneginf(m), 0.0, np.exp(m - shift))
+        p = np.exp(s - shift[..., None])
+        l = alpha * l + p.sum(axis=-1)
+        acc = alpha[..., None] * acc + np.einsum("bhij,bhjd->bhid", p, vv[:, :, j0:j0 + block])
+        m = m_new
+    out = np.where(l[..., None] > 0, acc / np.where(l > 0, l, 1.0)[..., None], 0.0)
+    lse = np.where(l > 0, m + np.log(np.where(l > 0, l, 1.0)), -np.inf)
+    return out, lse
+
+
+def attention_loops(q, k, v, *, scale=None, is_causal=False, key_lens=None, mask=None):
+    """Brute force with pure-Python loops and the math module; tiny inputs only."""
+    q, k, v = _f64(q).tolist(), _f64(k).tolist(), _f64(v).tolist()
+    B, Hq, Nq, d = len(q), len(q[0]), len(q[0][0]), len(q[0][0][0])
+    Hkv, Nk = len(k[0]), len(k[0][0])
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    mk = None if mask is None else np.broadcast_to(_f64(mask), (B, Hq, Nq, Nk)).tolist()
+    out = [[[[0.0] * d for _ in range(Nq)] for _ in range(Hq)] for _ in range(B)]
+    lse = [[[0.0] * Nq for _ in range(Hq)] for _ in range(B)]
+    for b in range(B):
+        n_valid = Nk if key_lens is None else int(key_lens[b])
+        for h in range(Hq):
+            hk = h // (Hq // Hkv)
+            for i in range(Nq):
+                keys = [j for j in range(Nk) if j < n_valid and not (is_causal and j > i)]
+                scores = {}
+                for j in keys:
+                    dot = 0.0
+                    for t in range(d):
+                        dot += q[b][h][i][t] * k[b][hk][j][t]
+                    sc = scale * dot + (mk[b][h][i][j] if mk is not None else 0.0)
+                    if sc != -math.inf:
+                        scores[j] = sc
+                if not scores:
+                    lse[b][h][i] = -math.inf
+                    continue
+                top = max(scores.values())
+                w = {j: math.exp(sc - top) for j, sc in scores.items()}
+                total = sum(w.values())
+                for t in range(d):
+                    out[b][h][i][t] = sum(w[j] * v[b][hk][j][t] for j in w) / total
+                lse[b][h][i] = top + math.log(total)
+    return np.array(out, dtype=np.float64), np.array(lse, dtype=np.float64)

@@ -1,0 +1,106 @@
+"""Seeded synthetic attention workloads shared by the tests, the smoke check and
+the benchmark.
+
+This module holds no attention arithmetic: it only names the shapes and draws
+the random inputs, so that the CUDA path and the fp64 oracle see the same bf16
+bits.  Q, K and V are drawn i.i.d. N(0, 1) in fp32 from a seeded torch
+generator and rounded to bf16 (round to nearest even); per-sample key lengths
+are drawn uniformly from [8, 77].
+
+The shapes stand in for the pages' workloads (no model weights or datasets are
+used):
+  tiny         B1  H2  N128          d64   -- small enough for full brute force
+  vit          B128 H16 N196         d64   -- 14x14-patch ViT self-attention
+                                               (atyun.com/61003.html, toy ViT)
+  long         B8  H32 N4096         d128  -- the B8 H32 N4096 d128 benchmark shape
+  long_causal  same, is_causal             (aiknowledge.cn FlashAttention benchmark page)
+  unet_self    B4  H8  N4096         d64   -- 64x64-latent UNet self-attention
+  unet_cross   B4  H8  Nq4096 Nk77   d64   -- UNet text cross-attention, padded keys
+                                               (xxmr.cn/news/81028, sections 2.1-2.2)
+  prefill_gqa  B1  Hq32 Hkv2 N16384  d128, causal -- grouped-head LLM prefill
+                                               (jsqmd.com/news/348824, causal=True)
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import torch
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    Nq: int
+    Nk: int
+    d: int
+    is_causal: bool = False
+    key_lens: tuple | None = None  # (low, high) inclusive range of per-sample key lengths
+    seed: int = 0
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    def flops(self) -> float:
+        """Forward FLOPs as the metric counts them: 4*B*Hq*Nq*Nk*d, halved when causal.
+
+        The count 4*N^2*d for one head is the one "FlashAttention technical analysis"
+        (jsqmd.com/news/722897) section 3.1 uses (8.6 GFLOP at N=4096, d=128).
+        """
+        f = 4.0 * self.B * self.Hq * self.Nq * self.Nk * self.d
+        return f / 2.0 if self.is_causal else f
+
+    def qkvo_bytes(self) -> int:
+        """Compulsory HBM bytes: read Q, K, V once, write O once (bf16)."""
+        return 2 * self.d * (2 * self.B * self.Hq * self.Nq + 2 * self.B * self.Hkv * self.Nk)
+
+    def lse_bytes(self) -> int:
+        return 4 * self.B * self.Hq * self.Nq
+
+
+WORKLOADS = {
+    w.name: w for w in [
+        Workload("tiny", 1, 2, 2, 128, 128, 64, seed=1000),
+        Workload("vit", 128, 16, 16, 196, 196, 64, seed=1001),
+        Workload("long", 8, 32, 32, 4096, 4096, 128, seed=1002),
+        Workload("long_causal", 8, 32, 32, 4096, 4096, 128, is_causal=True, seed=1012),
+        Workload("unet_self", 4, 8, 8, 4096, 4096, 64, seed=1003),
+        Workload("unet_cross", 4, 8, 8, 4096, 77, 64, key_lens=(8, 77), seed=1013),
+        Workload("prefill_gqa", 1, 32, 2, 16384, 16384, 128, is_causal=True, seed=1004),
+    ]
+}
+
+
+def make_qkv(B, Hq, Hkv, Nq, Nk, d, seed, device="cpu"):
+    """bf16 Q [B,Hq,Nq,d], K/V [B,Hkv,Nk,d], i.i.d. N(0,1) rounded to bf16."""
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+
+    def draw(shape):
+        return torch.randn(shape, generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+
+    q = draw((B, Hq, Nq, d))
+    k = draw((B, Hkv, Nk, d))
+    v = draw((B, Hkv, Nk, d))
+    return q, k, v
+
+
+def make_key_lens(B, low, high, seed):
+    """int32 [B] drawn uniformly from [low, high] inclusive (CPU generator)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed) + 7919)
+    return torch.randint(int(low), int(high) + 1, (B,), generator=g, dtype=torch.int64).to(torch.int32)
+
+
+def make_inputs(w: Workload, device="cpu", seed=None):
+    """Returns (q, k, v, key_lens or None) for a workload."""
+    s = w.seed if seed is None else seed
+    q, k, v = make_qkv(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, s, device)
+    kl = None
+    if w.key_lens is not None:
+        kl = make_key_lens(w.B, w.key_lens[0], w.key_lens[1], s).to(device)
+    return q, k, v, kl
