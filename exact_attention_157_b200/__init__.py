@@ -1,0 +1,191 @@
+"""Python binding of the sm_100a exact attention library (include/attn.h).
+
+Argument marshalling only: every step of the forward pass runs in the CUDA
+kernels of ``libattn_sm100.so``.  There is no fallback: if the library or a
+B200 is missing, calls raise.
+
+    from exact_attention_157_b200 import attention
+    out, lse = attention(q, k, v, is_causal=True)        # torch bf16 CUDA tensors
+
+Lower level, with the C names and raw pointers:
+
+    attn_fwd(q_ptr, k_ptr, v_ptr, out_ptr, lse_ptr, B, Hq, Hkv, Nq, Nk, d,
+             scale, is_causal, key_lens_ptr, mask_ptr, mask_strides, stream)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libattn_sm100.so")
+
+ATTN_OK = 0
+ATTN_ERR_INVALID_ARG = 1
+ATTN_ERR_UNSUPPORTED = 2
+ATTN_ERR_ALIGNMENT = 3
+ATTN_ERR_CUDA = 4
+ATTN_ERR_TIMEOUT = 5
+ATTN_ERR_DEVICE = 6
+
+# Every symbol include/attn.h declares.
+EXPORTED = ("attn_fwd", "attn_check_device_status", "attn_set_wait_timeout_ns",
+            "attn_selftest_timeout", "attn_status_string", "attn_last_cuda_error", "attn_version")
+
+_lock = threading.Lock()
+_lib = None
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = status_string(status)
+        if status == ATTN_ERR_CUDA:
+            msg += f" (cudaError {last_cuda_error()})"
+        super().__init__(f"{where}: {msg}")
+
+
+def lib() -> ctypes.CDLL:
+    """Load ``libattn_sm100.so`` (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise ImportError(f"{LIB_PATH} is missing; build it with "
+                                  "`python -m exact_attention_157_b200.build`")
+            L = ctypes.CDLL(LIB_PATH)
+            vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+            L.attn_fwd.restype = i
+            L.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, vp, vp, vp]
+            L.attn_check_device_status.restype = i
+            L.attn_check_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
+            L.attn_set_wait_timeout_ns.restype = i
+            L.attn_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
+            L.attn_selftest_timeout.restype = i
+            L.attn_selftest_timeout.argtypes = [vp]
+            L.attn_status_string.restype = ctypes.c_char_p
+            L.attn_status_string.argtypes = [i]
+            L.attn_last_cuda_error.restype = i
+            L.attn_last_cuda_error.argtypes = []
+            L.attn_version.restype = i
+            L.attn_version.argtypes = []
+            _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().attn_status_string(int(status)).decode()
+
+
+def last_cuda_error() -> int:
+    return int(lib().attn_last_cuda_error())
+
+
+def version() -> int:
+    return int(lib().attn_version())
+
+
+# ------------------------------------------------------------- C-named calls
+def attn_fwd(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, is_causal,
+             key_lens=None, additive_mask=None, mask_strides=None, stream=None) -> int:
+    """The C entry point with raw device pointers (ints); returns the status code."""
+    ms = None
+    if mask_strides is not None:
+        arr = (ctypes.c_int64 * 3)(*[int(x) for x in mask_strides])
+        ms = ctypes.cast(arr, ctypes.c_void_p)
+    return int(lib().attn_fwd(q, k, v, out, lse, int(B), int(Hq), int(Hkv), int(Nq), int(Nk), int(d),
+                              float(scale), int(bool(is_causal)), key_lens, additive_mask, ms, stream))
+
+
+def attn_check_device_status(stream=None):
+    """Synchronises ``stream``; returns (status, raw error word)."""
+    info = ctypes.c_uint32(0)
+    st = int(lib().attn_check_device_status(stream, ctypes.byref(info)))
+    return st, int(info.value)
+
+
+def attn_set_wait_timeout_ns(ns: int) -> int:
+    return int(lib().attn_set_wait_timeout_ns(int(ns)))
+
+
+def attn_selftest_timeout(stream=None) -> int:
+    return int(lib().attn_selftest_timeout(stream))
+
+
+# ------------------------------------------------------- torch marshalling
+def _stream_handle(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check_bf16_cuda(name, t, ndim):
+    import torch
+    if not isinstance(t, torch.Tensor) or t.device.type != "cuda":
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != torch.bfloat16:
+        raise TypeError(f"{name} must be bfloat16")
+    if t.dim() != ndim or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {ndim}-D tensor")
+
+
+def attention(q, k, v, *, scale: float | None = None, is_causal: bool = False, key_lens=None,
+              attn_mask=None, out=None, lse=None, return_lse: bool = True, stream=None):
+    """O = softmax(scale * Q K^T + mask) V on bf16 CUDA tensors.
+
+    q [B, Hq, Nq, d], k/v [B, Hkv, Nk, d] (contiguous bf16); key_lens int32 [B]
+    (CUDA) or None; attn_mask fp32 CUDA tensor broadcastable to [B, Hq, Nq, Nk]
+    with a contiguous last dimension, or None.  Returns (out, lse or None).
+    """
+    import torch
+    _check_bf16_cuda("q", q, 4)
+    _check_bf16_cuda("k", k, 4)
+    _check_bf16_cuda("v", v, 4)
+    B, Hq, Nq, d = q.shape
+    Bk, Hkv, Nk, dk = k.shape
+    if Bk != B or dk != d or tuple(v.shape) != tuple(k.shape):
+        raise ValueError("q, k, v shapes disagree")
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _check_bf16_cuda("out", out, 4)
+        if tuple(out.shape) != tuple(q.shape):
+            raise ValueError("out has the wrong shape")
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    if lse is not None and (lse.dtype != torch.float32 or not lse.is_contiguous()
+                            or tuple(lse.shape) != (B, Hq, Nq)):
+        raise ValueError("lse must be a contiguous fp32 [B, Hq, Nq] tensor")
+    kl_ptr = None
+    if key_lens is not None:
+        if key_lens.dtype != torch.int32 or key_lens.device != q.device or key_lens.numel() != B:
+            raise ValueError("key_lens must be an int32 CUDA tensor with B entries")
+        key_lens = key_lens.contiguous()
+        kl_ptr = key_lens.data_ptr()
+    m_ptr, m_strides = None, None
+    if attn_mask is not None:
+        if attn_mask.dtype != torch.float32 or attn_mask.device != q.device:
+            raise ValueError("attn_mask must be a float32 CUDA tensor")
+        m = attn_mask
+        while m.dim() < 4:
+            m = m.unsqueeze(0)
+        m = m.expand(B, Hq, Nq, Nk)
+        if m.stride(3) != 1:
+            m = m.contiguous()
+        m_ptr, m_strides = m.data_ptr(), (m.stride(0), m.stride(1), m.stride(2))
+    st = attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                  None if lse is None else lse.data_ptr(), B, Hq, Hkv, Nq, Nk, d,
+                  0.0 if scale is None else float(scale), is_causal, kl_ptr, m_ptr, m_strides,
+                  _stream_handle(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd")
+    return out, lse
+
+
+def check_device_status(stream=None):
+    """Raises AttnError if a kernel recorded a device-side failure."""
+    st, info = attn_check_device_status(_stream_handle(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, f"device status (word 0x{info:08x})")

@@ -1,0 +1,241 @@
+// attn_api.cu -- host side of the C ABI declared in include/attn.h: argument
+// validation, TMA tensor-map encoding, kernel selection and launch on the
+// caller's stream.  No device memory is allocated here.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "attn.h"
+#include "fwd_kernel.cuh"
+
+using namespace attn_sm100;
+
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;
+
+std::atomic<int> g_last_cuda_error{0};
+std::atomic<unsigned long long> g_timeout_ns{kDefaultTimeoutNs};
+std::atomic<unsigned int> g_epoch{0};
+
+// Launch id for the launch-wide abort flag; never 0 (the flag's initial value).
+unsigned int next_epoch() {
+    unsigned int e = g_epoch.fetch_add(1u) + 1u;
+    return e == 0u ? next_epoch() : e;
+}
+
+struct DeviceState {
+    bool ready = false;
+    attn_status_t status = ATTN_OK;
+    int sm_count = 0;
+};
+constexpr int kMaxDevices = 64;
+DeviceState g_dev[kMaxDevices];
+std::mutex g_mutex;
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+attn_status_t cuda_fail(cudaError_t e) {
+    g_last_cuda_error.store(static_cast<int>(e));
+    return ATTN_ERR_CUDA;
+}
+
+template <int D, int NS, bool M>
+cudaError_t set_kernel_attrs() {
+    return cudaFuncSetAttribute(attn_fwd_kernel<D, NS, M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                Smem<D, NS>::kAlloc);
+}
+
+constexpr int kStages128 = 3;
+constexpr int kStages64 = 4;
+
+// One-time per-device set-up: architecture check, SM count, kernel attributes,
+// and the driver's tensor-map encoder.
+attn_status_t device_setup(int* dev_out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_UNSUPPORTED;
+    *dev_out = dev;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    DeviceState& st = g_dev[dev];
+    if (st.ready) return st.status;
+    int major = 0, minor = 0;
+    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess) return cuda_fail(e);
+    if ((e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess) return cuda_fail(e);
+    if ((e = cudaDeviceGetAttribute(&st.sm_count, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return cuda_fail(e);
+    if (major != 10 || minor != 0) {
+        st.ready = true;
+        st.status = ATTN_ERR_UNSUPPORTED;
+        return st.status;
+    }
+    if (g_encode == nullptr) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+        if (e != cudaSuccess) return cuda_fail(e);
+        if (q != cudaDriverEntryPointSuccess || fn == nullptr) return ATTN_ERR_UNSUPPORTED;
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    if ((e = set_kernel_attrs<128, kStages128, false>()) != cudaSuccess) return cuda_fail(e);
+    if ((e = set_kernel_attrs<128, kStages128, true>()) != cudaSuccess) return cuda_fail(e);
+    if ((e = set_kernel_attrs<64, kStages64, false>()) != cudaSuccess) return cuda_fail(e);
+    if ((e = set_kernel_attrs<64, kStages64, true>()) != cudaSuccess) return cuda_fail(e);
+    st.ready = true;
+    st.status = ATTN_OK;
+    return ATTN_OK;
+}
+
+// 3-D map over a [heads, rows, d] bf16 tensor, box = 64 columns x 128 rows x 1,
+// 128-byte swizzle (the layout the UMMA shared-memory descriptors expect).
+attn_status_t encode_map(CUtensorMap* map, const void* base, int d, int rows, long long heads) {
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(heads)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2u, static_cast<cuuint64_t>(rows) * d * 2u};
+    cuuint32_t box[3] = {64u, 128u, 1u};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        g_last_cuda_error.store(static_cast<int>(r));
+        return ATTN_ERR_CUDA;
+    }
+    return ATTN_OK;
+}
+
+template <int D, int NS, bool M>
+cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
+                   const FwdParams& p, unsigned grid, cudaStream_t stream) {
+    attn_fwd_kernel<D, NS, M><<<grid, kThreads, Smem<D, NS>::kAlloc, stream>>>(tq, tk, tv, to, p);
+    return cudaGetLastError();
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
+                       int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                       float scale, int is_causal,
+                       const int32_t* key_lens,
+                       const float* additive_mask, const int64_t* mask_strides,
+                       void* stream) {
+    // ---- host-side validation (no CUDA call before this passes)
+    if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return ATTN_ERR_INVALID_ARG;
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nk <= 0 || d <= 0) return ATTN_ERR_INVALID_ARG;
+    if (Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+    if (key_lens != nullptr && additive_mask != nullptr) return ATTN_ERR_INVALID_ARG;
+    if (!(std::isfinite(scale)) || scale < 0.0f) return ATTN_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return ATTN_ERR_ALIGNMENT;
+    if ((lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) ||
+        (key_lens != nullptr && (reinterpret_cast<uintptr_t>(key_lens) & 3u)) ||
+        (additive_mask != nullptr && (reinterpret_cast<uintptr_t>(additive_mask) & 3u)))
+        return ATTN_ERR_ALIGNMENT;
+    const long long n_qtiles = (static_cast<long long>(Nq) + kBM - 1) / kBM;
+    const long long grid = static_cast<long long>(B) * Hq * n_qtiles;
+    if (grid > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+    long long msb = 0, msh = 0, msq = 0;
+    if (additive_mask != nullptr) {
+        if (mask_strides != nullptr) {
+            msb = mask_strides[0];
+            msh = mask_strides[1];
+            msq = mask_strides[2];
+            if (msb < 0 || msh < 0 || msq < 0) return ATTN_ERR_INVALID_ARG;
+        } else {
+            msq = Nk;
+            msh = static_cast<long long>(Nq) * Nk;
+            msb = msh * Hq;
+        }
+    }
+
+    int dev = 0;
+    attn_status_t st = device_setup(&dev);
+    if (st != ATTN_OK) return st;
+
+    float scale_eff = scale == 0.0f ? static_cast<float>(1.0 / std::sqrt(static_cast<double>(d))) : scale;
+    FwdParams p;
+    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Nq = Nq; p.Nk = Nk;
+    p.group = Hq / Hkv;
+    p.n_qtiles = static_cast<int>(n_qtiles);
+    p.scale_log2 = static_cast<float>(static_cast<double>(scale_eff) * 1.4426950408889634);
+    p.is_causal = is_causal ? 1 : 0;
+    p.key_lens = key_lens;
+    p.mask = additive_mask;
+    p.msb = msb; p.msh = msh; p.msq = msq;
+    p.lse = lse;
+    p.timeout_ns = g_timeout_ns.load();
+    p.epoch = next_epoch();
+
+    CUtensorMap tq, tk, tv, to;
+    if ((st = encode_map(&tq, q, d, Nq, static_cast<long long>(B) * Hq)) != ATTN_OK) return st;
+    if ((st = encode_map(&tk, k, d, Nk, static_cast<long long>(B) * Hkv)) != ATTN_OK) return st;
+    if ((st = encode_map(&tv, v, d, Nk, static_cast<long long>(B) * Hkv)) != ATTN_OK) return st;
+    if ((st = encode_map(&to, out, d, Nq, static_cast<long long>(B) * Hq)) != ATTN_OK) return st;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const unsigned g = static_cast<unsigned>(grid);
+    const bool has_mask = additive_mask != nullptr;
+    cudaError_t e;
+    if (d == 128)
+        e = has_mask ? launch<128, kStages128, true>(tq, tk, tv, to, p, g, s)
+                     : launch<128, kStages128, false>(tq, tk, tv, to, p, g, s);
+    else
+        e = has_mask ? launch<64, kStages64, true>(tq, tk, tv, to, p, g, s)
+                     : launch<64, kStages64, false>(tq, tk, tv, to, p, g, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return ATTN_OK;
+}
+
+attn_status_t attn_check_device_status(void* stream, uint32_t* info) {
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e);
+    unsigned int word = 0;
+    if ((e = cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word))) != cudaSuccess) return cuda_fail(e);
+    if (info != nullptr) *info = word;
+    if (word == 0u) return ATTN_OK;
+    const unsigned int zero = 0u;
+    if ((e = cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero))) != cudaSuccess) return cuda_fail(e);
+    return (word & 0xffu) == kErrTimeout ? ATTN_ERR_TIMEOUT : ATTN_ERR_DEVICE;
+}
+
+attn_status_t attn_set_wait_timeout_ns(uint64_t ns) {
+    g_timeout_ns.store(ns == 0 ? kDefaultTimeoutNs : static_cast<unsigned long long>(ns));
+    return ATTN_OK;
+}
+
+attn_status_t attn_selftest_timeout(void* stream) {
+    int dev = 0;
+    attn_status_t st = device_setup(&dev);
+    if (st != ATTN_OK) return st;
+    attn_selftest_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(g_timeout_ns.load(), next_epoch());
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e);
+    return ATTN_OK;
+}
+
+const char* attn_status_string(int status) {
+    switch (status) {
+        case ATTN_OK: return "ok";
+        case ATTN_ERR_INVALID_ARG: return "invalid argument";
+        case ATTN_ERR_UNSUPPORTED: return "unsupported head dimension or device (needs d in {64,128} on sm_100)";
+        case ATTN_ERR_ALIGNMENT: return "tensor base pointer not 16-byte aligned";
+        case ATTN_ERR_CUDA: return "CUDA runtime or driver error (see attn_last_cuda_error)";
+        case ATTN_ERR_TIMEOUT: return "a bounded wait inside a kernel expired";
+        case ATTN_ERR_DEVICE: return "device-side consistency check failed";
+        default: return "unknown status";
+    }
+}
+
+int attn_last_cuda_error(void) { return g_last_cuda_error.load(); }
+
+int attn_version(void) { return kVersion; }
+
+}  // extern "C"

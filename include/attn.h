@@ -1,0 +1,124 @@
+/*
+ * attn.h -- C ABI of the B200 (sm_100a) exact attention forward library.
+ *
+ * The operation is exact scaled-dot-product attention, forward only:
+ *
+ *     O = softmax(scale * Q K^T + mask) V,     LSE = logsumexp(scale * Q K^T + mask)
+ *
+ * as stated in "Flash Attention in a production Stable-Diffusion service"
+ * (xxmr.cn/news/81028), section 2.3 (QK^T, divide by sqrt(d_k), add attn_mask,
+ * softmax over the last axis, multiply by V; dropout is zero at inference) and
+ * computed tile by tile with an online softmax as in "FlashAttention technical
+ * analysis" (jsqmd.com/news/722897), section 2.2.  The N x N score matrix never
+ * reaches device memory; the only extra output is the per-row log-sum-exp that
+ * a recomputing backward pass needs (same page, section 3.3).
+ *
+ * Conventions shared by every entry point:
+ *   - Pointers named "device" must point to device memory of the current CUDA
+ *     device; the library neither allocates, frees nor retains them.  Calls are
+ *     asynchronous on the given stream: buffers must stay alive until the
+ *     stream has passed the call.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *   - Every function returns an attn_status_t and never prints, exits or traps.
+ *     Host-side argument errors are reported synchronously; faults detected
+ *     inside a kernel (an expired bounded wait) are recorded on the device and
+ *     reported by attn_check_device_status().
+ */
+#ifndef ATTN_H_
+#define ATTN_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum attn_status_t {
+    ATTN_OK = 0,
+    ATTN_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, Hq % Hkv != 0, bad scale ... */
+    ATTN_ERR_UNSUPPORTED = 2,  /* head dim other than 64 / 128, or no sm_100 device */
+    ATTN_ERR_ALIGNMENT = 3,    /* a tensor base is not 16-byte aligned */
+    ATTN_ERR_CUDA = 4,         /* a CUDA runtime / driver call failed; see attn_last_cuda_error() */
+    ATTN_ERR_TIMEOUT = 5,      /* a bounded wait inside a kernel expired (asynchronous) */
+    ATTN_ERR_DEVICE = 6        /* another device-side consistency check failed (asynchronous) */
+} attn_status_t;
+
+/*
+ * attn_fwd -- exact attention forward pass.
+ *
+ * Layout ([batch, heads, seq, head_dim], the layout the Stable-Diffusion page,
+ * section 3.1, passes to scaled_dot_product_attention), all contiguous:
+ *   q    device bf16 [B, Hq,  Nq, d]
+ *   k    device bf16 [B, Hkv, Nk, d]
+ *   v    device bf16 [B, Hkv, Nk, d]
+ *   out  device bf16 [B, Hq,  Nq, d]    (written; rounded to nearest even)
+ *   lse  device fp32 [B, Hq,  Nq] or NULL (written: natural-log log-sum-exp of
+ *        the scaled, masked scores of each query row; -inf for a row that has
+ *        no unmasked key, whose output row is then 0)
+ * Sizes: B, Hq, Hkv, Nq, Nk >= 1; Hq % Hkv == 0 (query head h reads K/V head
+ * h / (Hq / Hkv)); d in {64, 128}.  Every base pointer 16-byte aligned.
+ * scale: multiplies Q K^T; 0 selects 1/sqrt(d) (flash_attn_func's
+ * softmax_scale=None on the ChatGLM2 page, jsqmd.com/news/348824); negative,
+ * infinite or NaN scales are rejected.
+ * is_causal: non-zero masks key j for query i when j > i (top-left alignment,
+ * the convention of scaled_dot_product_attention's is_causal).
+ * key_lens: device int32 [B] or NULL.  Keys j >= key_lens[b] of batch b are
+ *   masked (padding); 0 <= key_lens[b] <= Nk is the caller's contract.
+ * additive_mask: device fp32 or NULL, added to the scaled scores
+ *   (s = scale * q.k + mask, the order of section 2.3 of the Stable-Diffusion
+ *   page); -inf entries mask a key.  Element (b, h, i, j) is read at
+ *   additive_mask[b*mask_strides[0] + h*mask_strides[1] + i*mask_strides[2] + j];
+ *   a stride of 0 broadcasts that axis; mask_strides (host, 3 x int64) NULL
+ *   means dense [B, Hq, Nq, Nk].  key_lens and additive_mask may not both be
+ *   given.  Mask values must not be +inf or NaN.
+ * Masked keys get probability exactly 0.  Q, K and V must be finite everywhere,
+ * padding included (0 * inf is NaN inside the matrix units).
+ * Errors: ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_ALIGNMENT,
+ * ATTN_ERR_CUDA (launch failure); kernel-side faults via attn_check_device_status.
+ */
+attn_status_t attn_fwd(const void *q, const void *k, const void *v, void *out, float *lse,
+                       int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                       float scale, int is_causal,
+                       const int32_t *key_lens,
+                       const float *additive_mask, const int64_t *mask_strides,
+                       void *stream);
+
+/*
+ * attn_check_device_status -- synchronise `stream`, then read and clear the
+ * device-side error word of the current device.  Returns ATTN_OK,
+ * ATTN_ERR_TIMEOUT, ATTN_ERR_DEVICE, or ATTN_ERR_CUDA if the synchronisation
+ * itself failed.  `info` (host, may be NULL) receives the raw error word
+ * (bits 0-7: code, bits 8-15: kernel role, bits 16-31: wait site).
+ */
+attn_status_t attn_check_device_status(void *stream, uint32_t *info);
+
+/*
+ * attn_set_wait_timeout_ns -- upper bound (nanoseconds, wall clock on the
+ * device) of every wait inside the library's kernels; default 2e9.  After it
+ * expires the waiting role records ATTN_ERR_TIMEOUT, stops its work, and the
+ * block releases its tensor memory and returns.  0 restores the default.
+ */
+attn_status_t attn_set_wait_timeout_ns(uint64_t ns);
+
+/*
+ * attn_selftest_timeout -- launches a one-warp kernel that waits, with the
+ * current bound, on a barrier nothing ever arrives at, so that the bounded
+ * wait must expire and record ATTN_ERR_TIMEOUT.  Used by the failure tests;
+ * it touches no caller memory.  Asynchronous on `stream`.
+ */
+attn_status_t attn_selftest_timeout(void *stream);
+
+/* Text for a status code (static storage). */
+const char *attn_status_string(int status);
+
+/* The cudaError_t kept from the last call that returned ATTN_ERR_CUDA (0 if none). */
+int attn_last_cuda_error(void);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_H_ */
