@@ -1,0 +1,407 @@
+#!/usr/bin/env python
+"""Forward-attention throughput on B200: TFLOP/s and fraction of roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload long] [--impl ours|reference]
+
+One step = one exact-attention forward pass (every step of the hot path, one
+kernel launch) over the whole workload, inputs resident in HBM.  The default
+workload is B8 H32 N4096 d128 bf16, non-causal (the shape of the pages' B8 H32
+N4096 d128 benchmark).  FLOPs per step = 4 B Hq Nq Nk d (halved when causal).
+
+Multi-GPU (torchrun, one process per GPU): every rank runs an independent
+batch of the same shape (weak scaling, no collective on the data path);
+``value`` is the FLOPs of all ranks divided by the slowest rank's time.
+
+``--impl reference`` times the fp64 CPU oracle on the host cores instead, on a
+bounded sample of the same workload per step (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "fwd attention TFLOP/s (B8 H32 N4096 d128 bf16) and % of B200 BF16 peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["exact_attention_157_b200/csrc/fwd_kernel.cuh", "exact_attention_157_b200/csrc/sm100_ptx.cuh",
+                  "exact_attention_157_b200/csrc/attn_api.cu"]
+
+
+# --------------------------------------------------------------- helpers
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS, source="fallback")
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu summary of this kernel and
+    workload, if it was taken on the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", f"attn_fwd_{workload}.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m_b = re.search(r"^traffic_bytes_per_launch:\s*([0-9.eE+]+)", text, re.M)
+    m_h = re.search(r"^kernel_source_sha:\s*([0-9a-f]+)", text, re.M)
+    if not m_b or not m_h or m_h.group(1) != kernel_source_hash():
+        return None
+    return float(m_b.group(1))
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+
+    REASONS = {  # NVML clocks-event reason bits
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.idx, self.period = device_index, period_s
+        self.samples, self.reason_bits = [], 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.handle = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+        except Exception:  # noqa: BLE001 - NVML missing: clocks are reported as unknown
+            self.nvml = None
+
+    def _run(self):
+        n = self.nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(n.nvmlDeviceGetClockInfo(self.handle, n.NVML_CLOCK_SM))
+                self.reason_bits |= int(n.nvmlDeviceGetCurrentClocksEventReasons(self.handle))
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self):
+        reasons = [name for bit, name in self.REASONS.items() if self.reason_bits & bit and bit != 0x1]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "samples": len(self.samples), "reasons": reasons}
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Slowest rank's time (all ranks call this in the same order)."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ---------------------------------------------------------- CPU baseline
+def oracle_sample(w, q, k, v, kl, target_s: float, max_rows=None):
+    """Runs the fp64 oracle on a bounded sample of the workload: whole query
+    rows of the first (batch, head) pairs, as many as fit in ~target_s.
+    Returns (flops, seconds, description, threads)."""
+    import numpy as np
+    import oracle
+    threads = oracle.default_threads()
+    kl_list = None if kl is None else kl.cpu().tolist()
+    group = w.Hq // w.Hkv
+
+    def head_inputs(b, h):
+        hk = h // group
+        return (q[b:b + 1, h:h + 1].cpu().double().numpy(), k[b:b + 1, hk:hk + 1].cpu().double().numpy(),
+                v[b:b + 1, hk:hk + 1].cpu().double().numpy(), None if kl_list is None else [kl_list[b]])
+
+    def flops_of(b, rows):
+        nk = w.Nk if kl_list is None else kl_list[b]
+        total = 0.0
+        for i in rows:
+            keys = min(nk, i + 1) if w.is_causal else nk
+            total += 4.0 * keys * w.d
+        return total
+
+    # calibrate on a slice of the first head
+    qh, kh, vh, klh = head_inputs(0, 0)
+    cal_rows = list(range(0, w.Nq, max(1, w.Nq // max(1, min(w.Nq, 4 * threads)))))[: 4 * threads]
+    t0 = time.perf_counter()
+    oracle.attention(qh, kh, vh, is_causal=w.is_causal, key_lens=klh, rows=cal_rows)
+    t_cal = max(time.perf_counter() - t0, 1e-6)
+    per_flop = t_cal / max(flops_of(0, cal_rows), 1.0)
+    budget = target_s / per_flop  # flops we can afford
+    # choose rows: whole heads while they fit, then a prefix of rows of the next head
+    plan, used = [], 0.0
+    for bh in range(w.B * w.Hq):
+        b, h = divmod(bh, w.Hq)
+        rows = list(range(w.Nq))
+        f = flops_of(b, rows)
+        if used + f <= budget:
+            plan.append((b, h, rows))
+            used += f
+            continue
+        # partial head: as many rows as fit (at least one row overall)
+        n = max(1 if not plan else 0, int(w.Nq * (budget - used) / max(f, 1.0)))
+        if max_rows is not None:
+            n = min(n, max_rows)
+        if n > 0:
+            plan.append((b, h, rows[:n]))
+            used += flops_of(b, rows[:n])
+        break
+    t0 = time.perf_counter()
+    total = 0.0
+    for b, h, rows in plan:
+        qh, kh, vh, klh = head_inputs(b, h)
+        oracle.attention(qh, kh, vh, is_causal=w.is_causal, key_lens=klh,
+                         rows=None if len(rows) == w.Nq else rows)
+        total += flops_of(b, rows)
+    dt = time.perf_counter() - t0
+    n_rows = sum(len(r) for _, _, r in plan)
+    desc = (f"{n_rows} query rows over {len(plan)} (batch, head) pairs of the {w.name} workload "
+            f"({n_rows / (w.B * w.Hq * w.Nq):.2e} of it), fp64, all keys of each row")
+    return total, dt, desc, threads
+
+
+# -------------------------------------------------------------- our arm
+def run_ours(args, w):
+    import torch
+    import exact_attention_157_b200 as ea
+    from workloads import make_inputs
+
+    world, rank, local = dist_env()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    q, k, v, kl = make_inputs(w, device=dev, seed=w.seed + 7 * rank)
+    out = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flops = w.flops()
+    in_bytes = q.numel() * 2 + k.numel() * 2 + v.numel() * 2 + (0 if kl is None else kl.numel() * 4)
+    out_bytes = out.numel() * 2 + lse.numel() * 4
+    l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = None
+    if in_bytes + out_bytes < 2 * l2_bytes:  # small working set: flush L2 between steps
+        flush = torch.empty(2 * l2_bytes // 4, dtype=torch.float32, device=dev)
+
+    def step():
+        if flush is not None:
+            flush.fill_(1.0)
+        ea.attention(q, k, v, is_causal=w.is_causal, key_lens=kl, out=out, lse=lse, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    ea.check_device_status(stream)
+
+    # --- device-timed region: K steps, events on the launching stream
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * args.steps)] if flush is not None else None
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world, dev)
+    torch.cuda.synchronize(dev)
+    launches = 0
+    with ClockSampler(dev.index) as clocks:
+        start.record(stream)
+        for i in range(args.steps):
+            if flush is not None:
+                flush.fill_(1.0)
+                ev[2 * i].record(stream)
+                ea.attention(q, k, v, is_causal=w.is_causal, key_lens=kl, out=out, lse=lse, stream=stream)
+                ev[2 * i + 1].record(stream)
+            else:
+                ea.attention(q, k, v, is_causal=w.is_causal, key_lens=kl, out=out, lse=lse, stream=stream)
+            launches += 1
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    ea.check_device_status(stream)
+    total_ms = start.elapsed_time(end)
+    if flush is not None:  # kernel time only, the L2 flush between steps excluded
+        kernel_ms = sum(ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(args.steps))
+    else:
+        kernel_ms = total_ms
+    kernel_ms = max_over_ranks(kernel_ms, world, dev)
+    ms_per_step = kernel_ms / args.steps
+    value = flops * world / (ms_per_step * 1e-3) / 1e12
+
+    # --- end to end through the public API with pinned host buffers
+    qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
+    klh = None if kl is None else kl.cpu().pin_memory()
+    outh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    lseh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    runner = ea.HostAttention(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, device=dev, with_key_lens=kl is not None)
+    e2e_steps = max(1, min(args.steps, 20))
+    for _ in range(min(args.warmup, 3)):
+        runner(qh, kh, vh, outh, lseh, klh, is_causal=w.is_causal, stream=stream)
+    barrier(world, dev)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        runner(qh, kh, vh, outh, lseh, klh, is_causal=w.is_causal, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / e2e_steps
+    ea.check_device_status(stream)
+    e2e_value = flops * world / (e2e_ms * 1e-3) / 1e12
+
+    peaks = load_peaks()
+    per_launch_flops = flops
+    per_launch_bytes = w.qkvo_bytes() + w.lse_bytes()
+    t_launch = ms_per_step * 1e-3
+    compute_floor = per_launch_flops / (peaks["bf16_tflops"] * 1e12)
+    hbm_floor = per_launch_bytes / (peaks["hbm_gbs"] * 1e9)
+    if compute_floor >= hbm_floor:
+        roof = {"bound": "tensor", "achieved": per_launch_flops / t_launch / 1e12, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s"}
+    else:
+        roof = {"bound": "hbm", "achieved": per_launch_bytes / t_launch / 1e9, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = recorded_traffic(w.name)
+    roof["peak_source"] = peaks["source"] + " (burst)"
+    roof["frac_of_roofline_time"] = max(compute_floor, hbm_floor) / t_launch
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        f, dt, desc, threads = oracle_sample(w, q, k, v, kl, target_s=args.cpu_seconds)
+        cpu = {"value": f / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc,
+               "seconds": dt}
+
+    result = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{w.name}: B{w.B} Hq{w.Hq} Hkv{w.Hkv} Nq{w.Nq} Nk{w.Nk} d{w.d}"
+                               f"{' causal' if w.is_causal else ''}",
+                   "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Nq": w.Nq, "Nk": w.Nk, "d": w.d,
+                   "is_causal": w.is_causal, "key_lens": w.key_lens,
+                   "flops_per_step": flops, "parallelism": f"independent batch per GPU x{world}",
+                   "l2": ("L2 flushed between steps (kernel time only)" if flush is not None
+                          else f"inputs larger than L2 ({in_bytes / 1e6:.0f} MB > {l2_bytes / 1e6:.0f} MB)")},
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": in_bytes,
+                "d2h_bytes_per_step": out_bytes, "ms_per_step": e2e_ms},
+        "gpu_launches": launches,
+        "clocks": clocks.summary(),
+        "kernel_source_sha": kernel_source_hash(),
+    }
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+# -------------------------------------------------------- reference arm
+def run_reference(args, w):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return  # rank 0 alone runs the CPU oracle
+    import torch
+    from workloads import make_inputs
+    q, k, v, kl = make_inputs(w, device="cpu")
+    steps, warmup = max(1, args.steps), max(0, args.warmup)
+    per_step = max(0.2, min(10.0, args.reference_seconds / (steps + warmup)))
+    times, flops_total, desc, threads = [], 0.0, "", 1
+    for i in range(warmup + steps):
+        f, dt, desc, threads = oracle_sample(w, q, k, v, kl, target_s=per_step)
+        if i >= warmup:
+            times.append(dt)
+            flops_total += f
+    t = sum(times)
+    value = flops_total / t / 1e12
+    result = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": steps, "warmup": warmup,
+        "ms_per_step": 1e3 * t / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": f"{w.name}: B{w.B} Hq{w.Hq} Hkv{w.Hkv} Nq{w.Nq} Nk{w.Nk} d{w.d}"
+                               f"{' causal' if w.is_causal else ''}",
+                   "sample_per_step": desc},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(result), flush=True)
+
+
+def main(argv=None):
+    from workloads import WORKLOADS
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="long", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-baseline sample budget")
+    ap.add_argument("--reference-seconds", type=float, default=120.0, help="total budget of --impl reference")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_ours(args, w)
+
+
+if __name__ == "__main__":
+    main()

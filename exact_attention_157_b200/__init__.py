@@ -189,3 +189,43 @@ def check_device_status(stream=None):
     st, info = attn_check_device_status(_stream_handle(stream))
     if st != ATTN_OK:
         raise AttnError(st, f"device status (word 0x{info:08x})")
+
+
+class HostAttention:
+    """End-to-end call for inputs that live in (pinned) host memory.
+
+    Each call copies Q, K, V (and key lengths) host -> device on ``stream``,
+    runs ``attn_fwd`` and copies O and LSE back into the host tensors it was
+    given; the device staging buffers are allocated once, here, and reused.
+    """
+
+    def __init__(self, B, Hq, Hkv, Nq, Nk, d, device="cuda:0", with_lse=True, with_key_lens=False):
+        import torch
+        dev = torch.device(device)
+        bf = torch.bfloat16
+        self.shape = (B, Hq, Hkv, Nq, Nk, d)
+        self.q = torch.empty((B, Hq, Nq, d), dtype=bf, device=dev)
+        self.k = torch.empty((B, Hkv, Nk, d), dtype=bf, device=dev)
+        self.v = torch.empty((B, Hkv, Nk, d), dtype=bf, device=dev)
+        self.out = torch.empty((B, Hq, Nq, d), dtype=bf, device=dev)
+        self.lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=dev) if with_lse else None
+        self.key_lens = torch.empty((B,), dtype=torch.int32, device=dev) if with_key_lens else None
+
+    def __call__(self, q_h, k_h, v_h, out_h, lse_h=None, key_lens_h=None, *, scale=None,
+                 is_causal=False, stream=None):
+        import torch
+        s = torch.cuda.current_stream() if stream is None else stream
+        with torch.cuda.stream(s):
+            self.q.copy_(q_h, non_blocking=True)
+            self.k.copy_(k_h, non_blocking=True)
+            self.v.copy_(v_h, non_blocking=True)
+            kl = None
+            if key_lens_h is not None:
+                self.key_lens.copy_(key_lens_h, non_blocking=True)
+                kl = self.key_lens
+            attention(self.q, self.k, self.v, scale=scale, is_causal=is_causal, key_lens=kl,
+                      out=self.out, lse=self.lse, return_lse=self.lse is not None, stream=s)
+            out_h.copy_(self.out, non_blocking=True)
+            if lse_h is not None and self.lse is not None:
+                lse_h.copy_(self.lse, non_blocking=True)
+        return out_h, lse_h

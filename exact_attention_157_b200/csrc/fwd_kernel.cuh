@@ -73,9 +73,10 @@ struct Smem {
     static constexpr int VEMPTY = 1 + 3 * NS;
     static constexpr int SFULL = 1 + 4 * NS;   // 2
     static constexpr int PFULL = 3 + 4 * NS;   // 2
-    static constexpr int ODONE = 5 + 4 * NS;
-    static constexpr int MMAFIN = 6 + 4 * NS;
-    static constexpr int kNumBars = 7 + 4 * NS;
+    static constexpr int ODONE = 5 + 4 * NS;   // one phase per PV (used only while PV_{j-2} is known done)
+    static constexpr int OFINAL = 6 + 4 * NS;  // the last PV only: the epilogue's wait
+    static constexpr int MMAFIN = 7 + 4 * NS;
+    static constexpr int kNumBars = 8 + 4 * NS;
     static constexpr int kMisc = kBars + 8 * kNumBars;
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
@@ -137,6 +138,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             mbar_init(bar(L::PFULL + i), 128);
         }
         mbar_init(bar(L::ODONE), 1);
+        mbar_init(bar(L::OFINAL), 1);
         mbar_init(bar(L::MMAFIN), 1);
         // A CTA that starts after another CTA of this launch timed out does no work.
         *abort_flag = launch_aborted(p.epoch) ? 1 : 0;
@@ -242,7 +244,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 mma_commit(bar(L::SFULL + (j & 1)));
                 if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
             }
-            if (ok) issue_pv(n_blocks - 1);
+            if (ok && issue_pv(n_blocks - 1)) mma_commit(bar(L::OFINAL));
             // Wait until every MMA this thread issued has completed before teardown.
             mma_commit(bar(L::MMAFIN));
             mbar_drain(bar(L::MMAFIN), 0, kRoleMma, 24);
@@ -302,11 +304,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * c_log2;
             }
 
-            // Lazy correction: only when the max grew by more than tau somewhere in the warp.
+            // Lazy correction: a row moves its reference max only when the block max
+            // exceeds it by more than tau.  The TMEM load/store of O is warp-collective,
+            // but each row applies its own decision (alpha = 1 exactly otherwise), so a
+            // row's result never depends on the other rows of its warp.
             const bool need = mx > m_used + kLazyTau;
             if (__any_sync(0xffffffffu, need)) {
-                const float m_new = fmaxf(m_used, mx);
-                const float alpha = (m_used == -INFINITY) ? 0.0f : ex2_approx(m_used - m_new);
+                const float m_new = need ? mx : m_used;
+                const float alpha = !need ? 1.0f : (m_used == -INFINITY) ? 0.0f : ex2_approx(m_used - m_new);
                 l_sum *= alpha;
                 if (j > 0) {
                     // O holds sum_{i<j} P_i V_i once PV_{j-1} has completed.
@@ -352,7 +357,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
         // ---------------------------------------------------------- epilogue
         if (ok && n_blocks > 0) {
-            bool got = mbar_wait(bar(L::ODONE), (n_blocks - 1) & 1, limit, abort_flag, p.epoch, kRoleSoftmax, 32);
+            // A dedicated barrier: ODONE may still be a phase behind here (PV_{n-2}
+            // need not have completed), and a parity test cannot tell.
+            bool got = mbar_wait(bar(L::OFINAL), 0, limit, abort_flag, p.epoch, kRoleSoftmax, 32);
             ok = __all_sync(0xffffffffu, got);
             tc_fence_after();
         }

@@ -1,9 +1,11 @@
 """GPU parity: the sm_100a kernels (through the C ABI) against the fp64 oracle
 on the same seeded bf16 inputs.
 
-Tolerances (bf16 inputs, fp32 accumulation): max |O - O_ref| <= 1e-2 and
-max |LSE - LSE_ref| <= 1e-3; mask structure bit-exact (a masked key changes
-nothing, a row with no key gives O = 0 and LSE = -inf).
+Tolerances (bf16 inputs, fp32 accumulation): |O - O_ref| <= 1e-2 beyond the
+half-ulp of the bf16 output format (the stored output is bf16, and no bf16
+value lies within 1e-2 of, say, 4.03: the grid spacing there is 2^-5), and
+max |LSE - LSE_ref| <= 1e-3 (LSE is fp32); mask structure bit-exact (a masked
+key changes nothing, a row with no key gives O = 0 and LSE = -inf).
 """
 import math
 
@@ -31,14 +33,23 @@ def run_gpu(q, k, v, **kw):
     return out, lse
 
 
+def bf16_half_ulp(x):
+    """Half the spacing of the bf16 grid at |x| (8 significant bits)."""
+    ax = np.abs(x)
+    e = np.floor(np.log2(np.where(ax > 0, ax, 1.0)))
+    return np.where(ax > 0, 2.0 ** (e - 8), 0.0)
+
+
 def assert_close(o, lse, ro, rl, rows=None):
     o = o.double().cpu().numpy() if torch.is_tensor(o) else o
     lse = lse.double().cpu().numpy() if torch.is_tensor(lse) else lse
     if rows is not None:
         o, lse, ro, rl = o[..., rows, :], lse[..., rows], ro[..., rows, :], rl[..., rows]
     assert np.isfinite(o).all(), "non-finite output"
-    err_o = np.abs(o - ro).max()
-    assert err_o <= O_TOL, f"max|dO| = {err_o}"
+    err_o = np.abs(o - ro) - bf16_half_ulp(ro)
+    worst = np.unravel_index(np.argmax(err_o), err_o.shape)
+    assert err_o.max() <= O_TOL, (f"|dO| - half_ulp = {err_o.max()} at {worst}: "
+                                  f"O={o[worst]} O_ref={ro[worst]}")
     np.testing.assert_array_equal(np.isneginf(lse), np.isneginf(rl))
     fin = np.isfinite(rl)
     if fin.any():
@@ -48,7 +59,8 @@ def assert_close(o, lse, ro, rl, rows=None):
     assert (o[np.isneginf(rl)] == 0).all()
 
 
-SHAPES = [(1, 1), (2, 2), (127, 127), (128, 128), (129, 129), (255, 300), (300, 255), (1, 513), (513, 1), (77, 640)]
+SHAPES = [(1, 1), (2, 2), (127, 127), (128, 128), (129, 129), (200, 260), (255, 300), (300, 255), (1, 513),
+          (513, 1), (77, 640)]
 
 
 @pytest.mark.parametrize("Nq,Nk", SHAPES)
@@ -152,7 +164,7 @@ def test_no_lse_requested():
     ea.check_device_status()
     assert lse is None
     ro, rl = oracle.attention(q, k, v)
-    assert np.abs(out.double().cpu().numpy() - ro).max() <= O_TOL
+    assert (np.abs(out.double().cpu().numpy() - ro) - bf16_half_ulp(ro)).max() <= O_TOL
 
 
 # ---------------------------------------------------------- full workloads
