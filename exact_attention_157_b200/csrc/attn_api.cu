@@ -12,6 +12,7 @@
 
 #include "attn.h"
 #include "fwd_kernel.cuh"
+#include "fwd_kernel_pp.cuh"
 
 using namespace attn_sm100;
 
@@ -53,6 +54,14 @@ cudaError_t set_kernel_attrs() {
 
 constexpr int kStages128 = 3;
 constexpr int kStages64 = 4;
+constexpr int kSlots128 = 5;  // two-tile kernel: Q_A + Q_B + 5 K/V slots = 224 KB
+constexpr int kSlots64 = 8;
+
+template <int D, int NSLOT, bool M>
+cudaError_t set_pp_attrs() {
+    return cudaFuncSetAttribute(attn_fwd_pp_kernel<D, NSLOT, M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                SmemPP<D, NSLOT>::kAlloc);
+}
 
 // One-time per-device set-up: architecture check, SM count, kernel attributes,
 // and the driver's tensor-map encoder.
@@ -86,6 +95,10 @@ attn_status_t device_setup(int* dev_out) {
     if ((e = set_kernel_attrs<128, kStages128, true>()) != cudaSuccess) return cuda_fail(e);
     if ((e = set_kernel_attrs<64, kStages64, false>()) != cudaSuccess) return cuda_fail(e);
     if ((e = set_kernel_attrs<64, kStages64, true>()) != cudaSuccess) return cuda_fail(e);
+    if ((e = set_pp_attrs<128, kSlots128, false>()) != cudaSuccess) return cuda_fail(e);
+    if ((e = set_pp_attrs<128, kSlots128, true>()) != cudaSuccess) return cuda_fail(e);
+    if ((e = set_pp_attrs<64, kSlots64, false>()) != cudaSuccess) return cuda_fail(e);
+    if ((e = set_pp_attrs<64, kSlots64, true>()) != cudaSuccess) return cuda_fail(e);
     st.ready = true;
     st.status = ATTN_OK;
     return ATTN_OK;
@@ -112,6 +125,13 @@ template <int D, int NS, bool M>
 cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
                    const FwdParams& p, unsigned grid, cudaStream_t stream) {
     attn_fwd_kernel<D, NS, M><<<grid, kThreads, Smem<D, NS>::kAlloc, stream>>>(tq, tk, tv, to, p);
+    return cudaGetLastError();
+}
+
+template <int D, int NSLOT, bool M>
+cudaError_t launch_pp(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
+                      const FwdParams& p, unsigned grid, cudaStream_t stream) {
+    attn_fwd_pp_kernel<D, NSLOT, M><<<grid, kPPThreads, SmemPP<D, NSLOT>::kAlloc, stream>>>(tq, tk, tv, to, p);
     return cudaGetLastError();
 }
 
@@ -181,15 +201,17 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* out, f
     if ((st = encode_map(&to, out, d, Nq, static_cast<long long>(B) * Hq)) != ATTN_OK) return st;
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const unsigned g = static_cast<unsigned>(grid);
     const bool has_mask = additive_mask != nullptr;
     cudaError_t e;
+    // Two query tiles (256 rows) per CTA share each K/V block.
+    p.n_qtiles = static_cast<int>((static_cast<long long>(Nq) + 2 * kBM - 1) / (2 * kBM));
+    const unsigned g = static_cast<unsigned>(static_cast<long long>(B) * Hq * p.n_qtiles);
     if (d == 128)
-        e = has_mask ? launch<128, kStages128, true>(tq, tk, tv, to, p, g, s)
-                     : launch<128, kStages128, false>(tq, tk, tv, to, p, g, s);
+        e = has_mask ? launch_pp<128, kSlots128, true>(tq, tk, tv, to, p, g, s)
+                     : launch_pp<128, kSlots128, false>(tq, tk, tv, to, p, g, s);
     else
-        e = has_mask ? launch<64, kStages64, true>(tq, tk, tv, to, p, g, s)
-                     : launch<64, kStages64, false>(tq, tk, tv, to, p, g, s);
+        e = has_mask ? launch_pp<64, kSlots64, true>(tq, tk, tv, to, p, g, s)
+                     : launch_pp<64, kSlots64, false>(tq, tk, tv, to, p, g, s);
     if (e != cudaSuccess) return cuda_fail(e);
     return ATTN_OK;
 }
