@@ -54,13 +54,17 @@ cudaError_t set_kernel_attrs() {
 
 constexpr int kStages128 = 3;
 constexpr int kStages64 = 4;
-constexpr int kSlots128 = 5;  // two-tile kernel: Q_A + Q_B + 5 K/V slots = 224 KB
-constexpr int kSlots64 = 8;
+// Persistent two-tile kernel: d=128 keeps one Q buffer (64 KB) and 5 K/V slots
+// (160 KB) for deep K/V prefetch on long sequences; d=64 double-buffers Q
+// (2 x 32 KB) so that the next unit's Q loads behind the current one, with
+// 8 K/V slots (128 KB).
+constexpr int kSlots128 = 5, kQStages128 = 1;
+constexpr int kSlots64 = 8, kQStages64 = 2;
 
-template <int D, int NSLOT, bool M>
+template <int D, int NSLOT, int QS, bool M>
 cudaError_t set_pp_attrs() {
-    return cudaFuncSetAttribute(attn_fwd_pp_kernel<D, NSLOT, M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                SmemPP<D, NSLOT>::kAlloc);
+    return cudaFuncSetAttribute(attn_fwd_pp_kernel<D, NSLOT, QS, M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                SmemPP<D, NSLOT, QS>::kAlloc);
 }
 
 // One-time per-device set-up: architecture check, SM count, kernel attributes,
@@ -95,10 +99,10 @@ attn_status_t device_setup(int* dev_out) {
     if ((e = set_kernel_attrs<128, kStages128, true>()) != cudaSuccess) return cuda_fail(e);
     if ((e = set_kernel_attrs<64, kStages64, false>()) != cudaSuccess) return cuda_fail(e);
     if ((e = set_kernel_attrs<64, kStages64, true>()) != cudaSuccess) return cuda_fail(e);
-    if ((e = set_pp_attrs<128, kSlots128, false>()) != cudaSuccess) return cuda_fail(e);
-    if ((e = set_pp_attrs<128, kSlots128, true>()) != cudaSuccess) return cuda_fail(e);
-    if ((e = set_pp_attrs<64, kSlots64, false>()) != cudaSuccess) return cuda_fail(e);
-    if ((e = set_pp_attrs<64, kSlots64, true>()) != cudaSuccess) return cuda_fail(e);
+    if ((e = set_pp_attrs<128, kSlots128, kQStages128, false>()) != cudaSuccess) return cuda_fail(e);
+    if ((e = set_pp_attrs<128, kSlots128, kQStages128, true>()) != cudaSuccess) return cuda_fail(e);
+    if ((e = set_pp_attrs<64, kSlots64, kQStages64, false>()) != cudaSuccess) return cuda_fail(e);
+    if ((e = set_pp_attrs<64, kSlots64, kQStages64, true>()) != cudaSuccess) return cuda_fail(e);
     st.ready = true;
     st.status = ATTN_OK;
     return ATTN_OK;
@@ -128,10 +132,10 @@ cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
     return cudaGetLastError();
 }
 
-template <int D, int NSLOT, bool M>
+template <int D, int NSLOT, int QS, bool M>
 cudaError_t launch_pp(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
                       const FwdParams& p, unsigned grid, cudaStream_t stream) {
-    attn_fwd_pp_kernel<D, NSLOT, M><<<grid, kPPThreads, SmemPP<D, NSLOT>::kAlloc, stream>>>(tq, tk, tv, to, p);
+    attn_fwd_pp_kernel<D, NSLOT, QS, M><<<grid, kPPThreads, SmemPP<D, NSLOT, QS>::kAlloc, stream>>>(tq, tk, tv, to, p);
     return cudaGetLastError();
 }
 
@@ -191,6 +195,8 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* out, f
     p.mask = additive_mask;
     p.msb = msb; p.msh = msh; p.msq = msq;
     p.lse = lse;
+    p.out = out;
+    p.unit_run = 1;
     p.timeout_ns = g_timeout_ns.load();
     p.epoch = next_epoch();
 
@@ -203,15 +209,23 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* out, f
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const bool has_mask = additive_mask != nullptr;
     cudaError_t e;
-    // Two query tiles (256 rows) per CTA share each K/V block.
+    // Work units of 256 query rows (two tiles sharing each K/V block); one
+    // persistent CTA per SM loops over them.
     p.n_qtiles = static_cast<int>((static_cast<long long>(Nq) + 2 * kBM - 1) / (2 * kBM));
-    const unsigned g = static_cast<unsigned>(static_cast<long long>(B) * Hq * p.n_qtiles);
+    const long long n_units = static_cast<long long>(B) * Hq * p.n_qtiles;
+    if (n_units > (1LL << 30)) return ATTN_ERR_INVALID_ARG;  // unit sequence positions stay in int range
+    const int sms = g_dev[dev].sm_count > 0 ? g_dev[dev].sm_count : 1;
+    // Causal units differ in cost: with at least two units per SM, each CTA
+    // takes heavy/light pairs of one head (equal cost per pair).
+    p.unit_run = (is_causal && n_units >= 2LL * sms) ? 2 : 1;
+    const long long want = (n_units + p.unit_run - 1) / p.unit_run;
+    const unsigned g = static_cast<unsigned>(want < sms ? want : sms);
     if (d == 128)
-        e = has_mask ? launch_pp<128, kSlots128, true>(tq, tk, tv, to, p, g, s)
-                     : launch_pp<128, kSlots128, false>(tq, tk, tv, to, p, g, s);
+        e = has_mask ? launch_pp<128, kSlots128, kQStages128, true>(tq, tk, tv, to, p, g, s)
+                     : launch_pp<128, kSlots128, kQStages128, false>(tq, tk, tv, to, p, g, s);
     else
-        e = has_mask ? launch_pp<64, kSlots64, true>(tq, tk, tv, to, p, g, s)
-                     : launch_pp<64, kSlots64, false>(tq, tk, tv, to, p, g, s);
+        e = has_mask ? launch_pp<64, kSlots64, kQStages64, true>(tq, tk, tv, to, p, g, s)
+                     : launch_pp<64, kSlots64, kQStages64, false>(tq, tk, tv, to, p, g, s);
     if (e != cudaSuccess) return cuda_fail(e);
     return ATTN_OK;
 }

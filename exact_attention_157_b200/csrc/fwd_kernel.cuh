@@ -52,6 +52,8 @@ struct FwdParams {
     const float* mask;
     long long msb, msh, msq;
     float* lse;
+    void* out;     // O base (bf16), for rows written without the TMA store
+    int unit_run;  // persistent kernel: consecutive units per CTA turn (1 or 2)
     unsigned long long timeout_ns;
     unsigned int epoch;  // launch id for the launch-wide abort (never 0)
 };
@@ -282,21 +284,23 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if constexpr (HAS_MASK) {
                 // t = scale*log2e*qk + log2e*mask; masked keys -> -inf
                 #pragma unroll
+                // keys c >= lim are masked (past the end of K, or past the diagonal)
+                int lim = mask_row != nullptr ? kv_len - j0 : 0;
+                if (p.is_causal && q_idx - j0 + 1 < lim) lim = q_idx - j0 + 1;
+                #pragma unroll
                 for (int c = 0; c < kBN; ++c) {
-                    const int key = j0 + c;
-                    const bool valid = mask_row != nullptr && key < kv_len && !(p.is_causal && key > q_idx);
-                    const float mv = valid ? __ldg(mask_row + key) : 0.0f;
+                    const bool valid = c < lim;
+                    const float mv = valid ? __ldg(mask_row + j0 + c) : 0.0f;
                     s[c] = valid ? fmaf(s[c], c_log2, mv * kLog2e) : -INFINITY;
                     mx = fmaxf(mx, s[c]);
                 }
             } else {
                 const bool boundary = (j0 + kBN > kv_len) || (p.is_causal && j0 + kBN - 1 > q0);
                 if (boundary) {
+                    int lim = kv_len - j0;
+                    if (p.is_causal && q_idx - j0 + 1 < lim) lim = q_idx - j0 + 1;
                     #pragma unroll
-                    for (int c = 0; c < kBN; ++c) {
-                        const int key = j0 + c;
-                        if (key >= kv_len || (p.is_causal && key > q_idx)) s[c] = -INFINITY;
-                    }
+                    for (int c = 0; c < kBN; ++c) s[c] = (c < lim) ? s[c] : -INFINITY;
                 }
                 float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
                 #pragma unroll

@@ -1,20 +1,28 @@
-// fwd_kernel_pp.cuh -- exact attention forward pass for sm_100a, two query tiles
-// per CTA ("ping-pong").
+// fwd_kernel_pp.cuh -- exact attention forward pass for sm_100a: persistent
+// CTAs, two query tiles per work unit ("ping-pong").
 //
-// A CTA owns 256 query rows of one (batch, query head): tile A = rows q0..q0+127,
-// tile B = rows q0+128..q0+255.  Both tiles share every K/V block, so K/V are
-// read from shared memory once per 256 rows.
+// Work unit = 256 query rows of one (batch, query head): tile A = rows
+// q0..q0+127, tile B = rows q0+128..q0+255.  Both tiles share every K/V block,
+// so K/V are read from shared memory once per 256 rows.  One CTA per SM loops
+// over units.  Units are numbered head-major (the units of one head run at
+// about the same time, so its K/V stay in L2); within a head, causal units
+// alternate heavy and light (query tiles n-1, 0, n-2, 1, ...), and, when there
+// are at least two units per CTA, every CTA takes consecutive pairs (CTA c:
+// sequence positions 2(c + kG), 2(c + kG) + 1), so each CTA's causal work is a
+// sum of equal-cost pairs; otherwise CTA c takes c, c + G, ...  Set-up (barriers,
+// TMEM) is paid once per CTA, and the loads and MMAs of the next unit overlap
+// the epilogue of the current one.
 //
-//   warps 0-3   softmax of tile A (thread = row = TMEM lane)
-//   warps 4-7   softmax of tile B
-//   warp 8      TMA producer: Q_A, Q_B once, then K_0, V_0, K_1, V_1, ... into
-//               one ring of NSLOT shared-memory slots (128-byte swizzle, no
-//               multicast), in the order the MMAs consume them
-//   warps 10-11 idle (they complete the third warpgroup that setmaxnreg needs)
-//   warp 9      TMEM owner and MMA issuer (one thread), order
-//                 S_A(0) S_B(0) | PV_A(0) S_A(1) PV_B(0) S_B(1) | PV_A(1) S_A(2) ...
+//   warps 0-3   softmax + epilogue of tile A (thread = row = TMEM lane)
+//   warps 4-7   softmax + epilogue of tile B
+//   warp 8      TMA producer: Q_A, Q_B of each unit into one of QS Q buffers,
+//               K_0, V_0, K_1, V_1, ... of every unit into one ring of NSLOT
+//               slots (128-byte swizzle, no multicast), in consumption order
+//   warp 9      TMEM owner and MMA issuer (one thread), per unit
+//                 S_A(0) S_B(0) | PV_A(0) S_A(1) PV_B(0) S_B(1) | PV_A(1) ...
 //               so that while the softmax of one tile runs, the tensor cores
 //               work on the other tile (two MMAs of cover each way)
+//   warps 10-11 idle (they complete the third warpgroup that setmaxnreg needs)
 //
 // TMEM: S_A cols [0,128), S_B [128,256), O_A [256,256+D), O_B [256+D,256+2D).
 // P_t (bf16 pairs, 64 cols) overwrites the first half of S_t once the softmax
@@ -22,11 +30,17 @@
 // tcgen05.mma operations of one thread execute in issue order.  Because S_t(j)
 // is issued after PV_t(j-1), S_t(j) complete implies O_t = sum_{i<j} P_i V_i,
 // so the softmax may rescale O_t right away, without another barrier.
+// Across units, PV_t(0) of the next unit waits until the epilogue has read O_t
+// out of TMEM (OEMPTY), and the epilogue stages O_t through the unit's own
+// (dead) Q_t buffer, which the producer refills only after the TMA store has
+// read it (QEMPTY).
 //
 // Online softmax in base 2 with the scale folded into the FMA and lazy
 // rescaling ("FlashAttention technical analysis", jsqmd.com/news/722897,
 // sections 2.2 and 4.1); one final normalisation; LSE = (m + log2 l) ln 2.
 #pragma once
+
+#include <type_traits>
 
 #include "sm100_ptx.cuh"
 
@@ -34,29 +48,32 @@ namespace attn_sm100 {
 
 constexpr int kPPThreads = 384;  // 12 warps = 3 warpgroups
 // Register split (setmaxnreg): launched at 168 per thread (384 x 168 = 64512);
-// the TMA/MMA warpgroup gives back to 72 and the two softmax warpgroups take
-// 216: 2 x 128 x 216 + 128 x 72 = 64512, exactly the launch total.
-constexpr int kRegsSoftmax = 216;
-constexpr int kRegsControl = 72;
+// the TMA/MMA warpgroup gives back to 88 and the two softmax warpgroups take
+// 208: 2 x 128 x 208 + 128 x 88 = 64512, exactly the launch total.
+constexpr int kRegsSoftmax = 200;
+constexpr int kRegsControl = 104;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl <= kPPThreads * 168, "register split");
 
-template <int D, int NSLOT>
+template <int D, int NSLOT, int QS>
 struct SmemPP {
     static constexpr int kChunks = D / 64;
     static constexpr int kChunkBytes = 128 * 128;
     static constexpr int kTileBytes = kChunks * kChunkBytes;  // 128 rows x D bf16
-    static constexpr int kQ = 0;                              // Q_A, then Q_B
-    static constexpr int kRing = 2 * kTileBytes;
+    static constexpr int kQBuf = 2 * kTileBytes;              // Q_A then Q_B of one unit
+    static constexpr int kQ = 0;                              // QS buffers
+    static constexpr int kRing = QS * kQBuf;
     static constexpr int kBars = kRing + NSLOT * kTileBytes;
     // barrier indices
-    static constexpr int QFULL = 0;
-    static constexpr int FULL = 1;                 // NSLOT
-    static constexpr int EMPTY = 1 + NSLOT;        // NSLOT
-    static constexpr int SFULL = 1 + 2 * NSLOT;    // 2 (per tile)
-    static constexpr int PFULL = 3 + 2 * NSLOT;    // 2
-    static constexpr int OFINAL = 5 + 2 * NSLOT;   // 2
-    static constexpr int MMAFIN = 7 + 2 * NSLOT;
-    static constexpr int kNumBars = 8 + 2 * NSLOT;
+    static constexpr int QFULL = 0;                   // QS: Q buffer loaded
+    static constexpr int QEMPTY = QS;                 // QS: Q buffer free (2 arrivals: both tiles' stores)
+    static constexpr int FULL = 2 * QS;               // NSLOT: K/V slot loaded
+    static constexpr int EMPTY = 2 * QS + NSLOT;      // NSLOT: K/V slot released
+    static constexpr int SFULL = 2 * QS + 2 * NSLOT;  // 2: S_t(j) complete
+    static constexpr int PFULL = SFULL + 2;           // 2: P_t(j) stored (128 arrivals)
+    static constexpr int OFINAL = SFULL + 4;          // 2: last PV_t of a unit complete
+    static constexpr int OEMPTY = SFULL + 6;          // 2: O_t read out by the epilogue (128 arrivals)
+    static constexpr int MMAFIN = SFULL + 8;
+    static constexpr int kNumBars = MMAFIN + 1;
     static constexpr int kMisc = kBars + 8 * kNumBars;
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;
@@ -91,12 +108,97 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
 __device__ __forceinline__ float lo_f32(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v)); }
 __device__ __forceinline__ float hi_f32(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
 
-template <int D, int NSLOT, bool HAS_MASK>
+// Part of the exponentials can run on the FMA pipe instead of the MUFU unit:
+// one pair in every kExp2EmuEvery (0 disables; measured neutral to negative
+// on B200 at d = 128, where the softmax is latency- rather than MUFU-bound).
+// Used only on blocks without a masked key, so masked probabilities stay
+// exactly 0 (ex2(-inf)).
+#ifndef ATTN_EXP2_EMU_EVERY
+#define ATTN_EXP2_EMU_EVERY 0
+#endif
+constexpr int kExp2EmuEvery = ATTN_EXP2_EMU_EVERY;
+
+constexpr uint64_t splat2(uint32_t bits) { return (static_cast<uint64_t>(bits) << 32) | bits; }
+
+// 2^x for a pair, x <= ~9: Cody-Waite reduction x = n + f, n = round(x) (the
+// 1.5 * 2^23 rounding constant leaves n in the low mantissa bits), then a
+// degree-3 minimax polynomial for 2^f on [-1/2, 1/2] (max relative error
+// 7.5e-5; coefficients fitted by csrc/fit_exp2_poly.py) and n added to the
+// exponent field.  x is clamped at -120, where the result (~1e-36) is zero for
+// every practical purpose next to the row maximum (>= 1).
+__device__ __forceinline__ void exp2_poly_pair(uint64_t x, float& e0, float& e1) {
+    constexpr uint64_t kMagic = splat2(0x4B400000u);     //  12582912.0f
+    constexpr uint64_t kNegMagic = splat2(0xCB400000u);  // -12582912.0f
+    constexpr uint64_t kNegOne = splat2(0xBF800000u);    // -1.0f
+    constexpr uint64_t kC0 = splat2(0x3F7FFB49u);        // 0.99992806
+    constexpr uint64_t kC1 = splat2(0x3F31798Du);        // 0.69326097
+    constexpr uint64_t kC2 = splat2(0x3E786F0Du);        // 0.24261113
+    constexpr uint64_t kC3 = splat2(0x3D61FBB0u);        // 0.05517167
+    const uint64_t xx = pack_f32x2(fmaxf(lo_f32(x), -120.0f), fmaxf(hi_f32(x), -120.0f));
+    const uint64_t t = fadd2(xx, kMagic);
+    const uint64_t f = ffma2(fadd2(t, kNegMagic), kNegOne, xx);  // x - n, in [-1/2, 1/2]
+    uint64_t p = ffma2(f, kC3, kC2);
+    p = ffma2(p, f, kC1);
+    p = ffma2(p, f, kC0);
+    e0 = __uint_as_float(static_cast<uint32_t>(p) + (static_cast<uint32_t>(t) << 23));
+    e1 = __uint_as_float(static_cast<uint32_t>(p >> 32) + (static_cast<uint32_t>(t >> 32) << 23));
+}
+
+// Everything about one work unit that every role derives identically.
+struct Unit {
+    int bh, b, h, bhk, q0, kv_len;
+    int n_t[2];  // key blocks of tile A / B (0: nothing to compute)
+    bool tile_b_valid;
+    __device__ __forceinline__ int n_max() const { return n_t[0] > n_t[1] ? n_t[0] : n_t[1]; }
+};
+
+// Sequence position of the k-th unit of CTA c among G CTAs: runs of P
+// consecutive units (P = 2 pairs heavy with light causal units, P = 1 is plain
+// round-robin).
+__device__ __forceinline__ int unit_seq(int c, int k, int G, int P) {
+    return P == 2 ? 2 * (c + (k >> 1) * G) + (k & 1) : c + k * G;
+}
+
+// The key length of the batch entry of the unit at sequence position s (a
+// global load, issued one unit ahead by every role so that its latency is off
+// the critical path).
+__device__ __forceinline__ int unit_key_len(const FwdParams& p, int s, int n_units) {
+    if (p.key_lens == nullptr || s >= n_units) return p.Nk;
+    return __ldg(p.key_lens + (s / p.n_qtiles) / p.Hq);
+}
+
+__device__ __forceinline__ Unit decode_unit(const FwdParams& p, int s, int kv_len, bool report) {
+    Unit x;
+    x.bh = s / p.n_qtiles;
+    const int pos = s - x.bh * p.n_qtiles;
+    // causal: heavy and light query tiles alternate (n-1, 0, n-2, 1, ...)
+    const int qt = !p.is_causal ? pos : (pos & 1) ? (pos >> 1) : p.n_qtiles - 1 - (pos >> 1);
+    x.b = x.bh / p.Hq;
+    x.h = x.bh - x.b * p.Hq;
+    x.bhk = x.b * p.Hkv + x.h / p.group;
+    x.q0 = qt * 2 * kBM;
+    x.tile_b_valid = x.q0 + kBM < p.Nq;
+    if (kv_len < 0 || kv_len > p.Nk) {
+        if (report) record_error(kErrDevice, kRoleSoftmax, 1);
+        kv_len = kv_len < 0 ? 0 : p.Nk;
+    }
+    x.kv_len = kv_len;
+    #pragma unroll
+    for (int t = 0; t < 2; ++t) {
+        int end = x.kv_len;
+        if (p.is_causal && x.q0 + (t + 1) * kBM < end) end = x.q0 + (t + 1) * kBM;
+        x.n_t[t] = (end + kBN - 1) / kBN;
+    }
+    if (!x.tile_b_valid) x.n_t[1] = 0;
+    return x;
+}
+
+template <int D, int NSLOT, int QS, bool HAS_MASK>
 __global__ void __launch_bounds__(kPPThreads, 1)
 attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                    const FwdParams p) {
-    using L = SmemPP<D, NSLOT>;
+    using L = SmemPP<D, NSLOT, QS>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw_base = smem_u32(smem_raw);
     const uint32_t sbase = (raw_base + 1023u) & ~1023u;
@@ -104,40 +206,17 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-
-    // ---- CTA coordinates: p.n_qtiles counts 256-row CTA tiles here
-    const int bh = blockIdx.x / p.n_qtiles;
-    int qt = blockIdx.x % p.n_qtiles;
-    if (p.is_causal) qt = p.n_qtiles - 1 - qt;  // heavier causal tiles of a head first
-    const int b = bh / p.Hq;
-    const int h = bh - b * p.Hq;
-    const int bhk = b * p.Hkv + h / p.group;
-    const int q0 = qt * 2 * kBM;
-    const bool tile_b_valid = q0 + kBM < p.Nq;
-    int kv_len = p.Nk;
-    if (p.key_lens != nullptr) {
-        kv_len = p.key_lens[b];
-        if (kv_len < 0 || kv_len > p.Nk) {
-            if (threadIdx.x == 0) record_error(kErrDevice, kRoleSoftmax, 1);
-            kv_len = kv_len < 0 ? 0 : p.Nk;
-        }
-    }
-    // key blocks per tile: causal tiles stop at their diagonal block
-    int n_t[2];
-    #pragma unroll
-    for (int t = 0; t < 2; ++t) {
-        int end = kv_len;
-        if (p.is_causal && q0 + (t + 1) * kBM < end) end = q0 + (t + 1) * kBM;
-        n_t[t] = (end + kBN - 1) / kBN;
-    }
-    if (!tile_b_valid) n_t[1] = 0;
+    const int n_units = p.B * p.Hq * p.n_qtiles;  // p.n_qtiles counts 256-row units per head
 
     auto bar = [&](int i) -> uint32_t { return sbase + L::kBars + 8u * i; };
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
 
     if (threadIdx.x == 0) {
-        mbar_init(bar(L::QFULL), 1);
+        for (int q = 0; q < QS; ++q) {
+            mbar_init(bar(L::QFULL + q), 1);
+            mbar_init(bar(L::QEMPTY + q), 2);
+        }
         for (int s = 0; s < NSLOT; ++s) {
             mbar_init(bar(L::FULL + s), 1);
             mbar_init(bar(L::EMPTY + s), 1);
@@ -146,6 +225,7 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             mbar_init(bar(L::SFULL + t), 1);
             mbar_init(bar(L::PFULL + t), 128);
             mbar_init(bar(L::OFINAL + t), 1);
+            mbar_init(bar(L::OEMPTY + t), 128);
         }
         mbar_init(bar(L::MMAFIN), 1);
         *abort_flag = launch_aborted(p.epoch) ? 1 : 0;
@@ -166,10 +246,9 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint64_t limit = p.timeout_ns;
-    if (*abort_flag) { n_t[0] = 0; n_t[1] = 0; }
-    n_t[0] = __shfl_sync(0xffffffffu, n_t[0], 0);
-    n_t[1] = __shfl_sync(0xffffffffu, n_t[1], 0);
-    const int n_max = n_t[0] > n_t[1] ? n_t[0] : n_t[1];
+    // A CTA that starts after another CTA of this launch timed out does no work.
+    const int cta = __shfl_sync(0xffffffffu, *abort_flag ? n_units : static_cast<int>(blockIdx.x), 0);
+    const int G = static_cast<int>(gridDim.x);
 
     if (warp >= 8) {
       asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" :: "n"(kRegsControl));
@@ -177,270 +256,389 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         // idle warps
       } else if (warp == 8) {
         // ============================== TMA producer ==============================
-        if (lane == 0 && n_max > 0) {
+        if (lane == 0) {
             int uses[NSLOT];
             #pragma unroll
             for (int s = 0; s < NSLOT; ++s) uses[s] = 0;
-            const int n_q_tiles = tile_b_valid ? 2 : 1;
-            mbar_arrive_expect_tx(bar(L::QFULL), n_q_tiles * L::kTileBytes);
-            for (int t = 0; t < n_q_tiles; ++t) {
-                #pragma unroll
-                for (int c = 0; c < L::kChunks; ++c)
-                    tma_load_3d(sbase + L::kQ + t * L::kTileBytes + c * L::kChunkBytes, &tm_q, bar(L::QFULL),
-                                c * 64, q0 + t * kBM, bh);
+            int q_loads[QS];
+            #pragma unroll
+            for (int q = 0; q < QS; ++q) q_loads[q] = 0;
+            int i_glob = 0;  // K/V loads issued so far (ring position)
+            bool ok = true;
+            int it = 0;
+            int kv_next = unit_key_len(p, unit_seq(cta, 0, G, p.unit_run), n_units);
+            for (int u = unit_seq(cta, 0, G, p.unit_run); ok && u < n_units; ++it, u = unit_seq(cta, it, G, p.unit_run)) {
+                const Unit x = decode_unit(p, u, kv_next, false);
+                kv_next = unit_key_len(p, unit_seq(cta, it + 1, G, p.unit_run), n_units);
+                const int qb = it % QS;
+                const int n_max = x.n_max();
+                if (n_max == 0) continue;  // nothing to load; its epilogue does not use a Q buffer
+                // the Q buffer is free once both tiles' stores of its previous unit have read it
+                if (q_loads[qb] > 0 &&
+                    !mbar_wait(bar(L::QEMPTY + qb), (q_loads[qb] - 1) & 1, limit, abort_flag, p.epoch, kRoleProducer, 9))
+                    { ok = false; break; }
+                const int n_q_tiles = x.tile_b_valid ? 2 : 1;
+                mbar_arrive_expect_tx(bar(L::QFULL + qb), n_q_tiles * L::kTileBytes);
+                for (int t = 0; t < n_q_tiles; ++t) {
+                    #pragma unroll
+                    for (int c = 0; c < L::kChunks; ++c)
+                        tma_load_3d(sbase + L::kQ + qb * L::kQBuf + t * L::kTileBytes + c * L::kChunkBytes, &tm_q,
+                                    bar(L::QFULL + qb), c * 64, x.q0 + t * kBM, x.bh);
+                }
+                ++q_loads[qb];
+                for (int i = 0; i < 2 * n_max; ++i, ++i_glob) {  // K_0, V_0, K_1, V_1, ...
+                    const int s = i_glob % NSLOT;
+                    const int use = i_glob / NSLOT;
+                    if (use > 0 &&
+                        !mbar_wait(bar(L::EMPTY + s), (use - 1) & 1, limit, abort_flag, p.epoch, kRoleProducer, 10))
+                        { ok = false; break; }
+                    const CUtensorMap* map = (i & 1) ? &tm_v : &tm_k;
+                    mbar_arrive_expect_tx(bar(L::FULL + s), L::kTileBytes);
+                    #pragma unroll
+                    for (int c = 0; c < L::kChunks; ++c)
+                        tma_load_3d(sbase + L::kRing + s * L::kTileBytes + c * L::kChunkBytes, map, bar(L::FULL + s),
+                                    c * 64, (i >> 1) * kBN, x.bhk);
+                    uses[s] = use + 1;
+                }
             }
-            const int n_loads = 2 * n_max;  // K_0, V_0, K_1, V_1, ...
-            for (int i = 0; i < n_loads; ++i) {
-                const int s = i % NSLOT;
-                const int use = i / NSLOT;
-                if (use > 0 &&
-                    !mbar_wait(bar(L::EMPTY + s), (use - 1) & 1, limit, abort_flag, p.epoch, kRoleProducer, 10))
-                    break;
-                const CUtensorMap* map = (i & 1) ? &tm_v : &tm_k;
-                mbar_arrive_expect_tx(bar(L::FULL + s), L::kTileBytes);
-                #pragma unroll
-                for (int c = 0; c < L::kChunks; ++c)
-                    tma_load_3d(sbase + L::kRing + s * L::kTileBytes + c * L::kChunkBytes, map, bar(L::FULL + s),
-                                c * 64, (i >> 1) * kBN, bhk);
-                uses[s] = use + 1;
-            }
-            mbar_drain(bar(L::QFULL), 0, kRoleProducer, 12);
+            // Drain: every load this thread issued has landed before the CTA may exit.
+            #pragma unroll
+            for (int q = 0; q < QS; ++q)
+                if (q_loads[q] > 0) mbar_drain(bar(L::QFULL + q), (q_loads[q] - 1) & 1, kRoleProducer, 12);
             #pragma unroll
             for (int s = 0; s < NSLOT; ++s)
                 if (uses[s] > 0) mbar_drain(bar(L::FULL + s), (uses[s] - 1) & 1, kRoleProducer, 13);
         }
-    } else if (warp == 9) {
+      } else {
         // =============================== MMA issuer ===============================
-        if (lane == 0 && n_max > 0) {
+        if (lane == 0) {
             constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kBN, false);
             constexpr uint32_t kIdescO = idesc_bf16_f32(kBM, D, true);
-            auto slot_of = [](int i) { return i % NSLOT; };
-            auto wait_full = [&](int i, unsigned site) -> bool {
-                return mbar_wait(bar(L::FULL + slot_of(i)), (i / NSLOT) & 1, limit, abort_flag, p.epoch, kRoleMma, site);
-            };
-            auto issue_s = [&](int t, int j) {
-                const uint32_t q_addr = sbase + L::kQ + t * L::kTileBytes;
-                const uint32_t k_addr = sbase + L::kRing + slot_of(2 * j) * L::kTileBytes;
-                #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
-                    mma_ss(tmem + t * 128, smem_desc_sw128(q_addr + off, 16, 1024),
-                           smem_desc_sw128(k_addr + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
-                }
-                mma_commit(bar(L::SFULL + t));
-            };
-            auto issue_pv = [&](int t, int j) {
-                const uint32_t v_addr = sbase + L::kRing + slot_of(2 * j + 1) * L::kTileBytes;
-                const uint32_t o_tmem = tmem + L::kColO + t * D;
-                const uint32_t p_tmem = tmem + t * 128;
-                #pragma unroll
-                for (int kk = 0; kk < kBN / 16; ++kk)
-                    mma_ts(o_tmem, p_tmem + kk * 8, smem_desc_sw128(v_addr + kk * 2048, L::kChunkBytes, 1024),
-                           kIdescO, (j > 0 || kk > 0) ? 1u : 0u);
-            };
-            bool ok = mbar_wait(bar(L::QFULL), 0, limit, abort_flag, p.epoch, kRoleMma, 20) && wait_full(0, 21);
-            if (ok) {
+            int q_loads[QS];
+            #pragma unroll
+            for (int q = 0; q < QS; ++q) q_loads[q] = 0;
+            int i_glob = 0;      // K/V loads consumed so far
+            int gp[2] = {0, 0};  // P_t blocks consumed so far (PFULL phase)
+            bool ok = true;
+            int it = 0;
+            int kv_next = unit_key_len(p, unit_seq(cta, 0, G, p.unit_run), n_units);
+            for (int u = unit_seq(cta, 0, G, p.unit_run); ok && u < n_units; ++it, u = unit_seq(cta, it, G, p.unit_run)) {
+                const Unit x = decode_unit(p, u, kv_next, false);
+                kv_next = unit_key_len(p, unit_seq(cta, it + 1, G, p.unit_run), n_units);
+                const int n_max = x.n_max();
+                if (n_max == 0) continue;
+                const int qb = it % QS;
+                const uint32_t qbuf = sbase + L::kQ + qb * L::kQBuf;
+                auto slot_of = [&](int i) { return (i_glob + i) % NSLOT; };
+                auto wait_full = [&](int i, unsigned site) -> bool {
+                    return mbar_wait(bar(L::FULL + slot_of(i)), ((i_glob + i) / NSLOT) & 1, limit, abort_flag,
+                                     p.epoch, kRoleMma, site);
+                };
+                auto issue_s = [&](int t, int j) {
+                    const uint32_t q_addr = qbuf + t * L::kTileBytes;
+                    const uint32_t k_addr = sbase + L::kRing + slot_of(2 * j) * L::kTileBytes;
+                    #pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
+                        mma_ss(tmem + t * 128, smem_desc_sw128(q_addr + off, 16, 1024),
+                               smem_desc_sw128(k_addr + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(bar(L::SFULL + t));
+                };
+                auto issue_pv = [&](int t, int j) {
+                    const uint32_t v_addr = sbase + L::kRing + slot_of(2 * j + 1) * L::kTileBytes;
+                    const uint32_t o_tmem = tmem + L::kColO + t * D;
+                    const uint32_t p_tmem = tmem + t * 128;
+                    #pragma unroll
+                    for (int kk = 0; kk < kBN / 16; ++kk)
+                        mma_ts(o_tmem, p_tmem + kk * 8, smem_desc_sw128(v_addr + kk * 2048, L::kChunkBytes, 1024),
+                               kIdescO, (j > 0 || kk > 0) ? 1u : 0u);
+                };
+                ok = mbar_wait(bar(L::QFULL + qb), q_loads[qb] & 1, limit, abort_flag, p.epoch, kRoleMma, 20) &&
+                     wait_full(0, 21);
+                ++q_loads[qb];
+                if (!ok) break;
                 tc_fence_after();
                 for (int t = 0; t < 2; ++t)
-                    if (n_t[t] > 0) issue_s(t, 0);
+                    if (x.n_t[t] > 0) issue_s(t, 0);
                 mma_commit(bar(L::EMPTY + slot_of(0)));  // K_0 released once both S(0) complete
-            }
-            for (int j = 0; ok && j < n_max; ++j) {
-                bool v_ready = false, k_next_ready = false;
-                for (int t = 0; t < 2 && ok; ++t) {
-                    if (j >= n_t[t]) continue;
-                    if (!mbar_wait(bar(L::PFULL + t), j & 1, limit, abort_flag, p.epoch, kRoleMma, 22)) { ok = false; break; }
-                    if (!v_ready) {
-                        if (!wait_full(2 * j + 1, 23)) { ok = false; break; }
-                        v_ready = true;
-                    }
-                    tc_fence_after();
-                    issue_pv(t, j);
-                    if (j + 1 < n_t[t]) {
-                        if (!k_next_ready) {
-                            if (!wait_full(2 * j + 2, 24)) { ok = false; break; }
-                            k_next_ready = true;
-                            tc_fence_after();
+                for (int j = 0; ok && j < n_max; ++j) {
+                    bool v_ready = false, k_next_ready = false;
+                    for (int t = 0; t < 2 && ok; ++t) {
+                        if (j >= x.n_t[t]) continue;
+                        if (!mbar_wait(bar(L::PFULL + t), gp[t] & 1, limit, abort_flag, p.epoch, kRoleMma, 22))
+                            { ok = false; break; }
+                        ++gp[t];
+                        // the previous unit's epilogue must have read O_t out of TMEM
+                        if (j == 0 && it > 0 &&
+                            !mbar_wait(bar(L::OEMPTY + t), (it - 1) & 1, limit, abort_flag, p.epoch, kRoleMma, 23))
+                            { ok = false; break; }
+                        if (!v_ready) {
+                            if (!wait_full(2 * j + 1, 24)) { ok = false; break; }
+                            v_ready = true;
                         }
-                        issue_s(t, j + 1);
-                    } else {
-                        mma_commit(bar(L::OFINAL + t));
+                        tc_fence_after();
+                        issue_pv(t, j);
+                        if (j + 1 < x.n_t[t]) {
+                            if (!k_next_ready) {
+                                if (!wait_full(2 * j + 2, 25)) { ok = false; break; }
+                                k_next_ready = true;
+                                tc_fence_after();
+                            }
+                            issue_s(t, j + 1);
+                        } else {
+                            mma_commit(bar(L::OFINAL + t));
+                        }
                     }
+                    if (!ok) break;
+                    mma_commit(bar(L::EMPTY + slot_of(2 * j + 1)));  // V_j: both PV(j) issued above
+                    // K_{j+1}: the tile with n_t = n_max uses every block, so k_next_ready
+                    // holds exactly when j + 1 < n_max (each load is released once).
+                    if (k_next_ready) mma_commit(bar(L::EMPTY + slot_of(2 * j + 2)));
                 }
-                if (!ok) break;
-                mma_commit(bar(L::EMPTY + slot_of(2 * j + 1)));      // V_j: both PV(j) issued above
-                // K_{j+1}: the tile with n_t = n_max uses every block, so k_next_ready
-                // holds exactly when j + 1 < n_max (each load is released once).
-                if (k_next_ready) mma_commit(bar(L::EMPTY + slot_of(2 * j + 2)));
+                i_glob += 2 * n_max;
             }
             mma_commit(bar(L::MMAFIN));
-            mbar_drain(bar(L::MMAFIN), 0, kRoleMma, 25);
+            mbar_drain(bar(L::MMAFIN), 0, kRoleMma, 26);
         }
       }
     } else {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" :: "n"(kRegsSoftmax));
-        // ======================= softmax warpgroups (tiles A, B) ===================
-        const int t = warp >> 2;             // tile
+        // =================== softmax + epilogue warpgroups (tiles A, B) ===================
+        const int t = warp >> 2;  // tile
         const int row = (warp & 3) * 32 + lane;
-        const int q_idx = q0 + t * kBM + row;
-        const int q0_t = q0 + t * kBM;
-        const int n_blocks = n_t[t];
         const uint32_t lane_tmem = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
         const uint32_t s_tmem = lane_tmem + t * 128;
         const uint32_t o_tmem = lane_tmem + L::kColO + t * D;
         const float c_log2 = p.scale_log2;
         const uint64_t c2 = pack_f32x2(c_log2, c_log2);
-        float m_used = -INFINITY;
-        float l_sum = 0.0f;
+        int gs = 0;       // S_t blocks consumed so far (SFULL phase)
+        int n_final = 0;  // units with a PV for this tile so far (OFINAL phase)
         bool ok = true;
-        const float* mask_row = nullptr;
-        if constexpr (HAS_MASK) {
-            if (q_idx < p.Nq)
-                mask_row = p.mask + static_cast<long long>(b) * p.msb + static_cast<long long>(h) * p.msh +
-                           static_cast<long long>(q_idx) * p.msq;
-        }
-
-        for (int j = 0; j < n_blocks; ++j) {
-            bool got = mbar_wait(bar(L::SFULL + t), j & 1, limit, abort_flag, p.epoch, kRoleSoftmax, 30);
-            if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-            tc_fence_after();
-            uint32_t sr[kBN];
-            #pragma unroll
-            for (int c = 0; c < kBN / 32; ++c)
-                tmem_ld32(s_tmem + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
-            tmem_wait_ld();
-            float* s = reinterpret_cast<float*>(sr);
-            const int j0 = j * kBN;
-
-            float mx;
+        int it = 0;
+        int kv_next = unit_key_len(p, unit_seq(cta, 0, G, p.unit_run), n_units);
+        for (int u = unit_seq(cta, 0, G, p.unit_run); u < n_units; ++it, u = unit_seq(cta, it, G, p.unit_run)) {
+            const Unit x = decode_unit(p, u, kv_next, threadIdx.x == 0);
+            kv_next = unit_key_len(p, unit_seq(cta, it + 1, G, p.unit_run), n_units);
+            const int q0_t = x.q0 + t * kBM;
+            const int q_idx = q0_t + row;
+            const int n_blocks = ok ? x.n_t[t] : 0;
+            const int kv_len = x.kv_len;
+            float m_used = -INFINITY;  // running max (base-2, scaled), possibly stale by < tau
+            float l_sum = 0.0f;        // running sum of exp2(t - m_used)
+            const float* mask_row = nullptr;
             if constexpr (HAS_MASK) {
-                mx = -INFINITY;
+                if (q_idx < p.Nq)
+                    mask_row = p.mask + static_cast<long long>(x.b) * p.msb + static_cast<long long>(x.h) * p.msh +
+                               static_cast<long long>(q_idx) * p.msq;
+            }
+
+            for (int j = 0; j < n_blocks; ++j) {
+                bool got = mbar_wait(bar(L::SFULL + t), gs & 1, limit, abort_flag, p.epoch, kRoleSoftmax, 30);
+                if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+                ++gs;
+                tc_fence_after();
+                uint32_t sr[kBN];
                 #pragma unroll
-                for (int c = 0; c < kBN; ++c) {
-                    const int key = j0 + c;
-                    const bool valid = mask_row != nullptr && key < kv_len && !(p.is_causal && key > q_idx);
-                    const float mv = valid ? __ldg(mask_row + key) : 0.0f;
-                    s[c] = valid ? fmaf(s[c], c_log2, mv * kLog2e) : -INFINITY;
-                    mx = fmaxf(mx, s[c]);
-                }
-            } else {
-                if ((j0 + kBN > kv_len) || (p.is_causal && j0 + kBN - 1 > q0_t)) {
+                for (int c = 0; c < kBN / 32; ++c)
+                    tmem_ld32(s_tmem + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+                tmem_wait_ld();
+                float* s = reinterpret_cast<float*>(sr);
+                const int j0 = j * kBN;
+                const bool boundary = (j0 + kBN > kv_len) || (p.is_causal && j0 + kBN - 1 > q0_t);
+
+                float mx;
+                if constexpr (HAS_MASK) {
+                    mx = -INFINITY;
+                    #pragma unroll
+                    // keys c >= lim are masked (past the end of K, or past the diagonal)
+                    int lim = mask_row != nullptr ? kv_len - j0 : 0;
+                    if (p.is_causal && q_idx - j0 + 1 < lim) lim = q_idx - j0 + 1;
                     #pragma unroll
                     for (int c = 0; c < kBN; ++c) {
-                        const int key = j0 + c;
-                        if (key >= kv_len || (p.is_causal && key > q_idx)) s[c] = -INFINITY;
+                        const bool valid = c < lim;
+                        const float mv = valid ? __ldg(mask_row + j0 + c) : 0.0f;
+                        s[c] = valid ? fmaf(s[c], c_log2, mv * kLog2e) : -INFINITY;
+                        mx = fmaxf(mx, s[c]);
+                    }
+                } else {
+                    if (boundary) {
+                        // keys c >= lim of this block are masked (padding / past the diagonal);
+                        // one compare and select per element, c a compile-time constant
+                        int lim = kv_len - j0;
+                        if (p.is_causal && q_idx - j0 + 1 < lim) lim = q_idx - j0 + 1;
+                        #pragma unroll
+                        for (int c = 0; c < kBN; ++c) s[c] = (c < lim) ? s[c] : -INFINITY;
+                    }
+                    float m0 = fmax3(s[0], s[1], s[2]), m1 = fmax3(s[3], s[4], s[5]);
+                    float m2 = fmax3(s[6], s[7], s[8]), m3 = fmax3(s[9], s[10], s[11]);
+                    #pragma unroll
+                    for (int c = 12; c + 7 < kBN; c += 8) {
+                        m0 = fmax3(m0, s[c], s[c + 1]);
+                        m1 = fmax3(m1, s[c + 2], s[c + 3]);
+                        m2 = fmax3(m2, s[c + 4], s[c + 5]);
+                        m3 = fmax3(m3, s[c + 6], s[c + 7]);
+                    }
+                    m0 = fmax3(m0, s[kBN - 4], s[kBN - 3]);
+                    m1 = fmax3(m1, s[kBN - 2], s[kBN - 1]);
+                    mx = fmax3(m0, m1, fmaxf(m2, m3)) * c_log2;
+                }
+
+                // Lazy correction, decided per row: a row moves its reference max only when
+                // the block max exceeds it by more than tau.  The TMEM load/store of O_t is
+                // warp-collective, but rows that keep their max use alpha = 1 exactly, so a
+                // row's result never depends on the other rows of its warp.  O_t holds
+                // sum_{i<j} P_i V_i here (S_t(j) was issued after PV_t(j-1)); the rescale
+                // of O_t itself is done after P_t is stored (fewer live registers) and
+                // before the PFULL arrive that lets PV_t(j) start.
+                const bool need = mx > m_used + kLazyTau;
+                const bool warp_rescale = __any_sync(0xffffffffu, need) && j > 0;
+                float alpha = 1.0f;
+                if (need) {
+                    alpha = (m_used == -INFINITY) ? 0.0f : ex2_approx(m_used - mx);
+                    l_sum *= alpha;
+                    m_used = mx;
+                }
+                const float shift = (m_used == -INFINITY) ? 0.0f : m_used;
+                const uint64_t nshift2 = pack_f32x2(-shift, -shift);
+
+                // Three stages over the whole row, so that no instruction waits on the one
+                // just before it: (1) exponent arguments, (2) exponentials, (3) row sum and
+                // bf16 packing.
+                uint64_t acc0 = 0, acc1 = 0, acc2 = 0, acc3 = 0;  // packed partial sums
+                uint32_t pk[kBN / 2];
+                auto exp_row = [&](auto emulate) {
+                    if constexpr (HAS_MASK) {
+                        #pragma unroll
+                        for (int c = 0; c < kBN; ++c) s[c] = s[c] - shift;
+                    } else {
+                        #pragma unroll
+                        for (int c = 0; c < kBN / 2; ++c) {
+                            const uint64_t xv = ffma2(pack_f32x2(s[2 * c], s[2 * c + 1]), c2, nshift2);
+                            s[2 * c] = lo_f32(xv);
+                            s[2 * c + 1] = hi_f32(xv);
+                        }
+                    }
+                    #pragma unroll
+                    for (int c = 0; c < kBN / 2; ++c) {
+                        if (decltype(emulate)::value &&
+                            (c % (kExp2EmuEvery > 0 ? kExp2EmuEvery : 1)) == kExp2EmuEvery - 1) {
+                            exp2_poly_pair(pack_f32x2(s[2 * c], s[2 * c + 1]), s[2 * c], s[2 * c + 1]);
+                        } else {
+                            s[2 * c] = ex2_approx(s[2 * c]);
+                            s[2 * c + 1] = ex2_approx(s[2 * c + 1]);
+                        }
+                    }
+                    #pragma unroll
+                    for (int c = 0; c < kBN / 2; ++c) {
+                        const uint64_t e = pack_f32x2(s[2 * c], s[2 * c + 1]);
+                        switch (c & 3) {
+                            case 0: acc0 = fadd2(acc0, e); break;
+                            case 1: acc1 = fadd2(acc1, e); break;
+                            case 2: acc2 = fadd2(acc2, e); break;
+                            default: acc3 = fadd2(acc3, e); break;
+                        }
+                        pk[c] = pack_bf16x2(s[2 * c], s[2 * c + 1]);
+                    }
+                };
+                if (kExp2EmuEvery > 0 && !HAS_MASK && !boundary)
+                    exp_row(std::integral_constant<bool, kExp2EmuEvery != 0>{});
+                else
+                    exp_row(std::false_type{});
+                const uint64_t acc = fadd2(fadd2(acc0, acc2), fadd2(acc1, acc3));
+                l_sum += lo_f32(acc) + hi_f32(acc);
+
+                tmem_st32(s_tmem, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+                tmem_st32(s_tmem + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+                if (warp_rescale) {
+                    #pragma unroll
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t o[32];
+                        tmem_ld32(o_tmem + c * 32, o);
+                        tmem_wait_ld();
+                        #pragma unroll
+                        for (int v = 0; v < 32; ++v) o[v] = __float_as_uint(__uint_as_float(o[v]) * alpha);
+                        tmem_st32(o_tmem + c * 32, o);
                     }
                 }
-                float ma = fmax3(s[0], s[1], s[2]);
-                float mb = fmax3(s[3], s[4], s[5]);
-                #pragma unroll
-                for (int c = 6; c + 3 < kBN; c += 4) {
-                    ma = fmax3(ma, s[c], s[c + 1]);
-                    mb = fmax3(mb, s[c + 2], s[c + 3]);
-                }
-                mx = fmax3(ma, mb, s[kBN - 2]);
-                mx = fmaxf(mx, s[kBN - 1]) * c_log2;
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar(L::PFULL + t));
             }
 
-            // Lazy correction, decided per row (see the single-tile kernel).  O_t holds
-            // sum_{i<j} P_i V_i here: S_t(j) was issued after PV_t(j-1).  The TMEM
-            // rescale of O_t itself is done after P_t is stored (fewer live registers);
-            // it only has to precede the PFULL arrive that lets PV_t(j) start.
-            const bool need = mx > m_used + kLazyTau;
-            const bool warp_rescale = __any_sync(0xffffffffu, need) && j > 0;
-            float alpha = 1.0f;
-            if (need) {
-                alpha = (m_used == -INFINITY) ? 0.0f : ex2_approx(m_used - mx);
-                l_sum *= alpha;
-                m_used = mx;
-            }
-            const float shift = (m_used == -INFINITY) ? 0.0f : m_used;
-            const uint64_t nshift2 = pack_f32x2(-shift, -shift);
-
-            uint64_t acc0 = 0, acc1 = 0;  // two packed partial sums
-            uint32_t pk[kBN / 2];
-            #pragma unroll
-            for (int c = 0; c < kBN / 2; ++c) {
-                float e0, e1;
-                if constexpr (HAS_MASK) {
-                    e0 = ex2_approx(s[2 * c] - shift);
-                    e1 = ex2_approx(s[2 * c + 1] - shift);
-                } else {
-                    const uint64_t x = ffma2(pack_f32x2(s[2 * c], s[2 * c + 1]), c2, nshift2);
-                    e0 = ex2_approx(lo_f32(x));
-                    e1 = ex2_approx(hi_f32(x));
-                }
-                if (c & 1) acc1 = fadd2(acc1, pack_f32x2(e0, e1));
-                else acc0 = fadd2(acc0, pack_f32x2(e0, e1));
-                pk[c] = pack_bf16x2(e0, e1);
-            }
-            const uint64_t acc = fadd2(acc0, acc1);
-            l_sum += lo_f32(acc) + hi_f32(acc);
-
-            tmem_st32(s_tmem, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-            tmem_st32(s_tmem + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
-            if (warp_rescale) {
-                #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t o[32];
-                    tmem_ld32(o_tmem + c * 32, o);
-                    tmem_wait_ld();
+            // ------------------------------------------------------------ epilogue
+            const int qb = it % QS;
+            if (x.n_max() == 0) {
+                // No unmasked key at all (key length 0): O = 0, LSE = -inf, written
+                // directly (this unit loaded nothing and owns no Q buffer).
+                tc_fence_before();
+                mbar_arrive(bar(L::OEMPTY + t));
+                if (q_idx < p.Nq && ok && !*abort_flag) {
+                    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) +
+                                                          (static_cast<long long>(x.bh) * p.Nq + q_idx) * D);
                     #pragma unroll
-                    for (int u = 0; u < 32; ++u) o[u] = __float_as_uint(__uint_as_float(o[u]) * alpha);
-                    tmem_st32(o_tmem + c * 32, o);
+                    for (int v = 0; v < D / 8; ++v) dst[v] = make_uint4(0u, 0u, 0u, 0u);
+                    if (p.lse != nullptr) p.lse[static_cast<long long>(x.bh) * p.Nq + q_idx] = -INFINITY;
                 }
+                continue;
             }
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(bar(L::PFULL + t));
-        }
-
-        // ---------------------------------------------------------- epilogue
-        if (ok && n_blocks > 0) {
-            bool got = mbar_wait(bar(L::OFINAL + t), 0, limit, abort_flag, p.epoch, kRoleSoftmax, 32);
-            ok = __all_sync(0xffffffffu, got);
-            tc_fence_after();
-        }
-        const bool do_epilogue = __all_sync(0xffffffffu, ok && !*abort_flag) && q0_t < p.Nq;
-        if (do_epilogue) {
+            if (ok && n_blocks > 0) {
+                bool got = mbar_wait(bar(L::OFINAL + t), n_final & 1, limit, abort_flag, p.epoch, kRoleSoftmax, 32);
+                ok = __all_sync(0xffffffffu, got);
+                ++n_final;
+                tc_fence_after();
+            }
+            const bool do_epilogue = __all_sync(0xffffffffu, ok && !*abort_flag) && q0_t < p.Nq;
+            uint8_t* stage = smem + L::kQ + qb * L::kQBuf + t * L::kTileBytes;  // Q_t is dead after OFINAL_t
             const float inv_l = l_sum > 0.0f ? 1.0f / l_sum : 0.0f;
-            uint8_t* stage = smem + L::kQ + t * L::kTileBytes;  // Q_t is dead after OFINAL_t
             #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t o[32];
-                if (n_blocks > 0) {
+                if (n_blocks > 0 && do_epilogue) {
                     tmem_ld32(o_tmem + c * 32, o);
                     tmem_wait_ld();
                 } else {
                     #pragma unroll
-                    for (int u = 0; u < 32; ++u) o[u] = 0u;
+                    for (int v = 0; v < 32; ++v) o[v] = 0u;
                 }
-                uint32_t w[16];
-                #pragma unroll
-                for (int u = 0; u < 16; ++u)
-                    w[u] = pack_bf16x2(__uint_as_float(o[2 * u]) * inv_l, __uint_as_float(o[2 * u + 1]) * inv_l);
-                const int chunk = (c * 32) / 64;
-                const int unit0 = ((c * 32) % 64) / 8;
-                #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int phys = (unit0 + u) ^ (row & 7);
-                    uint4* dst = reinterpret_cast<uint4*>(stage + chunk * L::kChunkBytes + row * 128 + phys * 16);
-                    *dst = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+                if (c == D / 32 - 1) {
+                    // O_t has been read out of TMEM: the next unit's PV_t(0) may overwrite it.
+                    tc_fence_before();
+                    mbar_arrive(bar(L::OEMPTY + t));
+                }
+                if (do_epilogue) {
+                    uint32_t w[16];
+                    #pragma unroll
+                    for (int v = 0; v < 16; ++v)
+                        w[v] = pack_bf16x2(__uint_as_float(o[2 * v]) * inv_l, __uint_as_float(o[2 * v + 1]) * inv_l);
+                    const int chunk = (c * 32) / 64;
+                    const int unit0 = ((c * 32) % 64) / 8;
+                    #pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        const int phys = (unit0 + v) ^ (row & 7);
+                        uint4* dst = reinterpret_cast<uint4*>(stage + chunk * L::kChunkBytes + row * 128 + phys * 16);
+                        *dst = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+                    }
                 }
             }
-            fence_proxy_async_smem();
-            if (p.lse != nullptr && q_idx < p.Nq) {
-                const float lse = l_sum > 0.0f ? (m_used + __log2f(l_sum)) * kLn2 : -INFINITY;
-                p.lse[static_cast<long long>(bh) * p.Nq + q_idx] = lse;
+            if (do_epilogue) {
+                fence_proxy_async_smem();
+                if (p.lse != nullptr && q_idx < p.Nq) {
+                    const float lse = l_sum > 0.0f ? (m_used + __log2f(l_sum)) * kLn2 : -INFINITY;
+                    p.lse[static_cast<long long>(x.bh) * p.Nq + q_idx] = lse;
+                }
             }
-        }
-        named_barrier_sync(1 + t, 128);
-        if ((threadIdx.x & 127) == 0 && do_epilogue && !*abort_flag) {
-            #pragma unroll
-            for (int c = 0; c < L::kChunks; ++c)
-                tma_store_3d(&tm_o, sbase + L::kQ + t * L::kTileBytes + c * L::kChunkBytes, c * 64, q0_t, bh);
-            bulk_commit_group();
-            bulk_wait_group_read0();
+            named_barrier_sync(1 + t, 128);
+            if ((threadIdx.x & 127) == 0) {
+                if (do_epilogue && !*abort_flag) {
+                    #pragma unroll
+                    for (int c = 0; c < L::kChunks; ++c)
+                        tma_store_3d(&tm_o, smem_u32(stage) + c * L::kChunkBytes, c * 64, q0_t, x.bh);
+                    bulk_commit_group();
+                    bulk_wait_group_read0();
+                }
+                mbar_arrive(bar(L::QEMPTY + qb));  // the producer may refill this Q buffer
+            }
         }
     }
 

@@ -80,20 +80,24 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_
                                           unsigned int role, unsigned int site) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
-    for (;;) {
-        #pragma unroll 1
-        for (int i = 0; i < 32; ++i)
-            if (mbar_try_wait(bar, parity)) return true;
-        if (*abort) return false;
-        if (launch_aborted(epoch)) {
-            *abort = 1;
-            return false;
-        }
-        if (globaltimer_ns() - t0 > limit_ns) {
-            record_error(kErrTimeout, role, site);
-            *abort = 1;
-            atomicExch(&g_abort_epoch, epoch);
-            return false;
+    for (uint32_t n = 1;; ++n) {
+        if (mbar_try_wait(bar, parity)) return true;
+        // The slow checks run rarely, so that a phase completing meanwhile is seen
+        // at once: this CTA's abort flag and the clock every 256 polls, the
+        // launch-wide abort word (a global-memory read) only after 1 ms of waiting.
+        if ((n & 255u) == 0u) {
+            if (*abort) return false;
+            const uint64_t waited = globaltimer_ns() - t0;
+            if (waited > 1000000ull && launch_aborted(epoch)) {
+                *abort = 1;
+                return false;
+            }
+            if (waited > limit_ns) {
+                record_error(kErrTimeout, role, site);
+                *abort = 1;
+                atomicExch(&g_abort_epoch, epoch);
+                return false;
+            }
         }
     }
 }
@@ -106,11 +110,9 @@ constexpr uint64_t kDrainLimitNs = 20000000ull;  // 20 ms
 __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity, unsigned int role, unsigned int site) {
     if (mbar_try_wait(bar, parity)) return;
     const uint64_t t0 = globaltimer_ns();
-    for (;;) {
-        #pragma unroll 1
-        for (int i = 0; i < 32; ++i)
-            if (mbar_try_wait(bar, parity)) return;
-        if (globaltimer_ns() - t0 > kDrainLimitNs) {
+    for (uint32_t n = 1;; ++n) {
+        if (mbar_try_wait(bar, parity)) return;
+        if ((n & 255u) == 0u && globaltimer_ns() - t0 > kDrainLimitNs) {
             record_error(kErrTimeout, role, site);
             return;
         }
