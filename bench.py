@@ -34,8 +34,8 @@ if ROOT not in sys.path:
 
 METRIC = "fwd attention TFLOP/s (B8 H32 N4096 d128 bf16) and % of B200 BF16 peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCES = ["exact_attention_157_b200/csrc/fwd_kernel.cuh", "exact_attention_157_b200/csrc/sm100_ptx.cuh",
-                  "exact_attention_157_b200/csrc/attn_api.cu"]
+KERNEL_SOURCES = ["exact_attention_157_b200/csrc/fwd_kernel_pp.cuh", "exact_attention_157_b200/csrc/fwd_common.cuh",
+                  "exact_attention_157_b200/csrc/sm100_ptx.cuh", "exact_attention_157_b200/csrc/attn_api.cu"]
 
 
 # --------------------------------------------------------------- helpers

@@ -11,7 +11,7 @@
 #include <mutex>
 
 #include "attn.h"
-#include "fwd_kernel.cuh"
+#include "fwd_common.cuh"
 #include "fwd_kernel_pp.cuh"
 
 using namespace attn_sm100;
@@ -46,14 +46,6 @@ attn_status_t cuda_fail(cudaError_t e) {
     return ATTN_ERR_CUDA;
 }
 
-template <int D, int NS, bool M>
-cudaError_t set_kernel_attrs() {
-    return cudaFuncSetAttribute(attn_fwd_kernel<D, NS, M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                Smem<D, NS>::kAlloc);
-}
-
-constexpr int kStages128 = 3;
-constexpr int kStages64 = 4;
 // Persistent two-tile kernel: d=128 keeps one Q buffer (64 KB) and 5 K/V slots
 // (160 KB) for deep K/V prefetch on long sequences; d=64 double-buffers Q
 // (2 x 32 KB) so that the next unit's Q loads behind the current one, with
@@ -95,10 +87,6 @@ attn_status_t device_setup(int* dev_out) {
         if (q != cudaDriverEntryPointSuccess || fn == nullptr) return ATTN_ERR_UNSUPPORTED;
         g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
     }
-    if ((e = set_kernel_attrs<128, kStages128, false>()) != cudaSuccess) return cuda_fail(e);
-    if ((e = set_kernel_attrs<128, kStages128, true>()) != cudaSuccess) return cuda_fail(e);
-    if ((e = set_kernel_attrs<64, kStages64, false>()) != cudaSuccess) return cuda_fail(e);
-    if ((e = set_kernel_attrs<64, kStages64, true>()) != cudaSuccess) return cuda_fail(e);
     if ((e = set_pp_attrs<128, kSlots128, kQStages128, false>()) != cudaSuccess) return cuda_fail(e);
     if ((e = set_pp_attrs<128, kSlots128, kQStages128, true>()) != cudaSuccess) return cuda_fail(e);
     if ((e = set_pp_attrs<64, kSlots64, kQStages64, false>()) != cudaSuccess) return cuda_fail(e);
@@ -123,13 +111,6 @@ attn_status_t encode_map(CUtensorMap* map, const void* base, int d, int rows, lo
         return ATTN_ERR_CUDA;
     }
     return ATTN_OK;
-}
-
-template <int D, int NS, bool M>
-cudaError_t launch(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
-                   const FwdParams& p, unsigned grid, cudaStream_t stream) {
-    attn_fwd_kernel<D, NS, M><<<grid, kThreads, Smem<D, NS>::kAlloc, stream>>>(tq, tk, tv, to, p);
-    return cudaGetLastError();
 }
 
 template <int D, int NSLOT, int QS, bool M>
@@ -163,9 +144,6 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* out, f
         (key_lens != nullptr && (reinterpret_cast<uintptr_t>(key_lens) & 3u)) ||
         (additive_mask != nullptr && (reinterpret_cast<uintptr_t>(additive_mask) & 3u)))
         return ATTN_ERR_ALIGNMENT;
-    const long long n_qtiles = (static_cast<long long>(Nq) + kBM - 1) / kBM;
-    const long long grid = static_cast<long long>(B) * Hq * n_qtiles;
-    if (grid > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
     long long msb = 0, msh = 0, msq = 0;
     if (additive_mask != nullptr) {
         if (mask_strides != nullptr) {
@@ -188,7 +166,6 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* out, f
     FwdParams p;
     p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Nq = Nq; p.Nk = Nk;
     p.group = Hq / Hkv;
-    p.n_qtiles = static_cast<int>(n_qtiles);
     p.scale_log2 = static_cast<float>(static_cast<double>(scale_eff) * 1.4426950408889634);
     p.is_causal = is_causal ? 1 : 0;
     p.key_lens = key_lens;

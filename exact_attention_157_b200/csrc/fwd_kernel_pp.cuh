@@ -42,7 +42,7 @@
 
 #include <type_traits>
 
-#include "sm100_ptx.cuh"
+#include "fwd_common.cuh"
 
 namespace attn_sm100 {
 
