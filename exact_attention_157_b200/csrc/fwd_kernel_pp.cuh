@@ -69,10 +69,11 @@ struct SmemPP {
     static constexpr int FULL = 2 * QS;               // NSLOT: K/V slot loaded
     static constexpr int EMPTY = 2 * QS + NSLOT;      // NSLOT: K/V slot released
     static constexpr int SFULL = 2 * QS + 2 * NSLOT;  // 2: S_t(j) complete
-    static constexpr int PFULL = SFULL + 2;           // 2: P_t(j) stored (128 arrivals)
-    static constexpr int OFINAL = SFULL + 4;          // 2: last PV_t of a unit complete
-    static constexpr int OEMPTY = SFULL + 6;          // 2: O_t read out by the epilogue (128 arrivals)
-    static constexpr int MMAFIN = SFULL + 8;
+    static constexpr int P0 = SFULL + 2;              // 2: P_t(j) keys 0..63 stored (128 arrivals)
+    static constexpr int P1 = SFULL + 4;              // 2: P_t(j) keys 64..127 stored (128 arrivals)
+    static constexpr int OFINAL = SFULL + 6;          // 2: last PV_t of a unit complete
+    static constexpr int OEMPTY = SFULL + 8;          // 2: O_t read out by the epilogue (128 arrivals)
+    static constexpr int MMAFIN = SFULL + 10;
     static constexpr int kNumBars = MMAFIN + 1;
     static constexpr int kMisc = kBars + 8 * kNumBars;
     static constexpr int kBytes = kMisc + 16;
@@ -223,7 +224,8 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         }
         for (int t = 0; t < 2; ++t) {
             mbar_init(bar(L::SFULL + t), 1);
-            mbar_init(bar(L::PFULL + t), 128);
+            mbar_init(bar(L::P0 + t), 128);
+            mbar_init(bar(L::P1 + t), 128);
             mbar_init(bar(L::OFINAL + t), 1);
             mbar_init(bar(L::OEMPTY + t), 128);
         }
@@ -318,7 +320,7 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             #pragma unroll
             for (int q = 0; q < QS; ++q) q_loads[q] = 0;
             int i_glob = 0;      // K/V loads consumed so far
-            int gp[2] = {0, 0};  // P_t blocks consumed so far (PFULL phase)
+            int gp[2] = {0, 0};  // P_t blocks consumed so far (P0 / P1 phase)
             bool ok = true;
             int it = 0;
             int kv_next = unit_key_len(p, unit_seq(cta, 0, G, p.unit_run), n_units);
@@ -345,14 +347,17 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     }
                     mma_commit(bar(L::SFULL + t));
                 };
-                auto issue_pv = [&](int t, int j) {
+                // O_t += P_t(j)[:, keys 64 half .. +63] V_j[those keys, :]
+                auto issue_pv = [&](int t, int j, int half) {
                     const uint32_t v_addr = sbase + L::kRing + slot_of(2 * j + 1) * L::kTileBytes;
                     const uint32_t o_tmem = tmem + L::kColO + t * D;
                     const uint32_t p_tmem = tmem + t * 128;
                     #pragma unroll
-                    for (int kk = 0; kk < kBN / 16; ++kk)
+                    for (int k4 = 0; k4 < kBN / 32; ++k4) {
+                        const int kk = half * (kBN / 32) + k4;
                         mma_ts(o_tmem, p_tmem + kk * 8, smem_desc_sw128(v_addr + kk * 2048, L::kChunkBytes, 1024),
                                kIdescO, (j > 0 || kk > 0) ? 1u : 0u);
+                    }
                 };
                 ok = mbar_wait(bar(L::QFULL + qb), q_loads[qb] & 1, limit, abort_flag, p.epoch, kRoleMma, 20) &&
                      wait_full(0, 21);
@@ -366,9 +371,9 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     bool v_ready = false, k_next_ready = false;
                     for (int t = 0; t < 2 && ok; ++t) {
                         if (j >= x.n_t[t]) continue;
-                        if (!mbar_wait(bar(L::PFULL + t), gp[t] & 1, limit, abort_flag, p.epoch, kRoleMma, 22))
+                        // first half of P_t(j): PV over keys 0..63 overlaps the rest of the softmax
+                        if (!mbar_wait(bar(L::P0 + t), gp[t] & 1, limit, abort_flag, p.epoch, kRoleMma, 22))
                             { ok = false; break; }
-                        ++gp[t];
                         // the previous unit's epilogue must have read O_t out of TMEM
                         if (j == 0 && it > 0 &&
                             !mbar_wait(bar(L::OEMPTY + t), (it - 1) & 1, limit, abort_flag, p.epoch, kRoleMma, 23))
@@ -378,7 +383,12 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                             v_ready = true;
                         }
                         tc_fence_after();
-                        issue_pv(t, j);
+                        issue_pv(t, j, 0);
+                        if (!mbar_wait(bar(L::P1 + t), gp[t] & 1, limit, abort_flag, p.epoch, kRoleMma, 27))
+                            { ok = false; break; }
+                        ++gp[t];
+                        tc_fence_after();
+                        issue_pv(t, j, 1);
                         if (j + 1 < x.n_t[t]) {
                             if (!k_next_ready) {
                                 if (!wait_full(2 * j + 2, 25)) { ok = false; break; }
@@ -489,8 +499,8 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 // warp-collective, but rows that keep their max use alpha = 1 exactly, so a
                 // row's result never depends on the other rows of its warp.  O_t holds
                 // sum_{i<j} P_i V_i here (S_t(j) was issued after PV_t(j-1)); the rescale
-                // of O_t itself is done after P_t is stored (fewer live registers) and
-                // before the PFULL arrive that lets PV_t(j) start.
+                // of O_t itself is done after the first half of P_t is stored (fewer live
+                // registers) and before the P0 arrive that lets PV_t(j) start.
                 const bool need = mx > m_used + kLazyTau;
                 const bool warp_rescale = __any_sync(0xffffffffu, need) && j > 0;
                 float alpha = 1.0f;
@@ -506,64 +516,72 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 // just before it: (1) exponent arguments, (2) exponentials, (3) row sum and
                 // bf16 packing.
                 uint64_t acc0 = 0, acc1 = 0, acc2 = 0, acc3 = 0;  // packed partial sums
-                uint32_t pk[kBN / 2];
-                auto exp_row = [&](auto emulate) {
+                uint32_t pk[kBN / 4];
+                // Keys 0..63, then 64..127: each half is stored and signalled on its own
+                // (P0, P1), so PV over the first half runs during the second half.  O_t is
+                // rescaled (if needed) before P0 releases the first PV.
+                auto exp_half = [&](auto emulate, auto half_c) {
+                    constexpr int h = decltype(half_c)::value;
+                    float* sh = s + h * (kBN / 2);
                     if constexpr (HAS_MASK) {
                         #pragma unroll
-                        for (int c = 0; c < kBN; ++c) s[c] = s[c] - shift;
+                        for (int c = 0; c < kBN / 2; ++c) sh[c] = sh[c] - shift;
                     } else {
                         #pragma unroll
-                        for (int c = 0; c < kBN / 2; ++c) {
-                            const uint64_t xv = ffma2(pack_f32x2(s[2 * c], s[2 * c + 1]), c2, nshift2);
-                            s[2 * c] = lo_f32(xv);
-                            s[2 * c + 1] = hi_f32(xv);
+                        for (int c = 0; c < kBN / 4; ++c) {
+                            const uint64_t xv = ffma2(pack_f32x2(sh[2 * c], sh[2 * c + 1]), c2, nshift2);
+                            sh[2 * c] = lo_f32(xv);
+                            sh[2 * c + 1] = hi_f32(xv);
                         }
                     }
                     #pragma unroll
-                    for (int c = 0; c < kBN / 2; ++c) {
+                    for (int c = 0; c < kBN / 4; ++c) {
                         if (decltype(emulate)::value &&
                             (c % (kExp2EmuEvery > 0 ? kExp2EmuEvery : 1)) == kExp2EmuEvery - 1) {
-                            exp2_poly_pair(pack_f32x2(s[2 * c], s[2 * c + 1]), s[2 * c], s[2 * c + 1]);
+                            exp2_poly_pair(pack_f32x2(sh[2 * c], sh[2 * c + 1]), sh[2 * c], sh[2 * c + 1]);
                         } else {
-                            s[2 * c] = ex2_approx(s[2 * c]);
-                            s[2 * c + 1] = ex2_approx(s[2 * c + 1]);
+                            sh[2 * c] = ex2_approx(sh[2 * c]);
+                            sh[2 * c + 1] = ex2_approx(sh[2 * c + 1]);
                         }
                     }
                     #pragma unroll
-                    for (int c = 0; c < kBN / 2; ++c) {
-                        const uint64_t e = pack_f32x2(s[2 * c], s[2 * c + 1]);
+                    for (int c = 0; c < kBN / 4; ++c) {
+                        const uint64_t e = pack_f32x2(sh[2 * c], sh[2 * c + 1]);
                         switch (c & 3) {
                             case 0: acc0 = fadd2(acc0, e); break;
                             case 1: acc1 = fadd2(acc1, e); break;
                             case 2: acc2 = fadd2(acc2, e); break;
                             default: acc3 = fadd2(acc3, e); break;
                         }
-                        pk[c] = pack_bf16x2(s[2 * c], s[2 * c + 1]);
+                        pk[c] = pack_bf16x2(sh[2 * c], sh[2 * c + 1]);
                     }
+                    tmem_st32(s_tmem + h * 32, pk);
+                    if (h == 0 && warp_rescale) {
+                        #pragma unroll
+                        for (int c = 0; c < D / 32; ++c) {
+                            uint32_t o[32];
+                            tmem_ld32(o_tmem + c * 32, o);
+                            tmem_wait_ld();
+                            #pragma unroll
+                            for (int v = 0; v < 32; ++v) o[v] = __float_as_uint(__uint_as_float(o[v]) * alpha);
+                            tmem_st32(o_tmem + c * 32, o);
+                        }
+                    }
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(bar((h == 0 ? L::P0 : L::P1) + t));
                 };
-                if (kExp2EmuEvery > 0 && !HAS_MASK && !boundary)
-                    exp_row(std::integral_constant<bool, kExp2EmuEvery != 0>{});
-                else
-                    exp_row(std::false_type{});
+                using Half0 = std::integral_constant<int, 0>;
+                using Half1 = std::integral_constant<int, 1>;
+                if (kExp2EmuEvery > 0 && !HAS_MASK && !boundary) {
+                    exp_half(std::integral_constant<bool, kExp2EmuEvery != 0>{}, Half0{});
+                    exp_half(std::integral_constant<bool, kExp2EmuEvery != 0>{}, Half1{});
+                } else {
+                    exp_half(std::false_type{}, Half0{});
+                    exp_half(std::false_type{}, Half1{});
+                }
                 const uint64_t acc = fadd2(fadd2(acc0, acc2), fadd2(acc1, acc3));
                 l_sum += lo_f32(acc) + hi_f32(acc);
-
-                tmem_st32(s_tmem, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-                tmem_st32(s_tmem + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
-                if (warp_rescale) {
-                    #pragma unroll
-                    for (int c = 0; c < D / 32; ++c) {
-                        uint32_t o[32];
-                        tmem_ld32(o_tmem + c * 32, o);
-                        tmem_wait_ld();
-                        #pragma unroll
-                        for (int v = 0; v < 32; ++v) o[v] = __float_as_uint(__uint_as_float(o[v]) * alpha);
-                        tmem_st32(o_tmem + c * 32, o);
-                    }
-                }
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(bar(L::PFULL + t));
             }
 
             // ------------------------------------------------------------ epilogue
