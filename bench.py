@@ -242,10 +242,24 @@ def run_ours(args, w):
     if in_bytes + out_bytes < 2 * l2_bytes:  # small working set: flush L2 between steps
         flush = torch.empty(2 * l2_bytes // 4, dtype=torch.float32, device=dev)
 
+    # decode-shaped workloads run through the split-KV entry point (workspace allocated once, here)
+    split, ws, per_step_launches = None, None, 1
+    if w.split_kv:
+        split = 0
+        st, n_used, nbytes = ea.attn_splitkv_plan(w.B, w.Hq, w.Nq, w.Nk, w.d, split, 0)
+        if st != ea.ATTN_OK:
+            raise ea.AttnError(st, "attn_splitkv_plan")
+        ws = torch.empty((max(nbytes, 1),), dtype=torch.uint8, device=dev)
+        per_step_launches = 2 if n_used > 1 else 1
+
+    def call():
+        ea.attention(q, k, v, is_causal=w.is_causal, key_lens=kl, out=out, lse=lse, stream=stream,
+                     split_kv=split, workspace=ws)
+
     def step():
         if flush is not None:
             flush.fill_(1.0)
-        ea.attention(q, k, v, is_causal=w.is_causal, key_lens=kl, out=out, lse=lse, stream=stream)
+        call()
 
     for _ in range(args.warmup):
         step()
@@ -263,11 +277,11 @@ def run_ours(args, w):
             if flush is not None:
                 flush.fill_(1.0)
                 ev[2 * i].record(stream)
-                ea.attention(q, k, v, is_causal=w.is_causal, key_lens=kl, out=out, lse=lse, stream=stream)
+                call()
                 ev[2 * i + 1].record(stream)
             else:
-                ea.attention(q, k, v, is_causal=w.is_causal, key_lens=kl, out=out, lse=lse, stream=stream)
-            launches += 1
+                call()
+            launches += per_step_launches
         end.record(stream)
         torch.cuda.synchronize(dev)
     barrier(world, dev)
@@ -286,7 +300,8 @@ def run_ours(args, w):
     klh = None if kl is None else kl.cpu().pin_memory()
     outh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     lseh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-    runner = ea.HostAttention(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, device=dev, with_key_lens=kl is not None)
+    runner = ea.HostAttention(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, device=dev, with_key_lens=kl is not None,
+                              split_kv=split)
     e2e_steps = max(1, min(args.steps, 20))
     for _ in range(min(args.warmup, 3)):
         runner(qh, kh, vh, outh, lseh, klh, is_causal=w.is_causal, stream=stream)
@@ -333,6 +348,7 @@ def run_ours(args, w):
                                f"{' causal' if w.is_causal else ''}",
                    "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Nq": w.Nq, "Nk": w.Nk, "d": w.d,
                    "is_causal": w.is_causal, "key_lens": w.key_lens,
+                   "entry_point": "attn_fwd_splitkv" if w.split_kv else "attn_fwd",
                    "flops_per_step": flops, "parallelism": f"independent batch per GPU x{world}",
                    "l2": ("L2 flushed between steps (kernel time only)" if flush is not None
                           else f"inputs larger than L2 ({in_bytes / 1e6:.0f} MB > {l2_bytes / 1e6:.0f} MB)")},

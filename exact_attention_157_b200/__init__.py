@@ -7,10 +7,16 @@ B200 is missing, calls raise.
     from exact_attention_157_b200 import attention
     out, lse = attention(q, k, v, is_causal=True)        # torch bf16 CUDA tensors
 
+Split-KV (decode-shaped inputs: few queries, many keys):
+
+    out, lse = attention(q, k, v, split_kv=0)            # 0 = automatic range count
+
 Lower level, with the C names and raw pointers:
 
     attn_fwd(q_ptr, k_ptr, v_ptr, out_ptr, lse_ptr, B, Hq, Hkv, Nq, Nk, d,
              scale, is_causal, key_lens_ptr, mask_ptr, mask_strides, stream)
+    attn_splitkv_plan(B, Hq, Nq, Nk, d, n_splits, sm_count) -> (status, n_used, bytes)
+    attn_fwd_splitkv(..., n_splits, workspace_ptr, workspace_bytes, stream)
 """
 from __future__ import annotations
 
@@ -30,8 +36,8 @@ ATTN_ERR_TIMEOUT = 5
 ATTN_ERR_DEVICE = 6
 
 # Every symbol include/attn.h declares.
-EXPORTED = ("attn_fwd", "attn_check_device_status", "attn_set_wait_timeout_ns",
-            "attn_selftest_timeout", "attn_status_string", "attn_last_cuda_error", "attn_version")
+EXPORTED = ("attn_fwd", "attn_splitkv_plan", "attn_fwd_splitkv", "attn_check_device_status",
+            "attn_set_wait_timeout_ns", "attn_selftest_timeout", "attn_status_string", "attn_last_cuda_error", "attn_version")
 
 _lock = threading.Lock()
 _lib = None
@@ -58,6 +64,11 @@ def lib() -> ctypes.CDLL:
             vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
             L.attn_fwd.restype = i
             L.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, vp, vp, vp]
+            L.attn_splitkv_plan.restype = i
+            L.attn_splitkv_plan.argtypes = [i, i, i, i, i, i, i, ctypes.POINTER(i), ctypes.POINTER(ctypes.c_size_t)]
+            L.attn_fwd_splitkv.restype = i
+            L.attn_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, vp, vp,
+                                           i, vp, ctypes.c_size_t, vp]
             L.attn_check_device_status.restype = i
             L.attn_check_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
             L.attn_set_wait_timeout_ns.restype = i
@@ -98,6 +109,28 @@ def attn_fwd(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, is_causal,
                               float(scale), int(bool(is_causal)), key_lens, additive_mask, ms, stream))
 
 
+def attn_splitkv_plan(B, Hq, Nq, Nk, d, n_splits=0, sm_count=0):
+    """The C planner: returns (status, key ranges used, workspace bytes)."""
+    n = ctypes.c_int(0)
+    nb = ctypes.c_size_t(0)
+    st = int(lib().attn_splitkv_plan(int(B), int(Hq), int(Nq), int(Nk), int(d), int(n_splits), int(sm_count),
+                                     ctypes.byref(n), ctypes.byref(nb)))
+    return st, int(n.value), int(nb.value)
+
+
+def attn_fwd_splitkv(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, is_causal,
+                     key_lens=None, additive_mask=None, mask_strides=None, n_splits=0,
+                     workspace=None, workspace_bytes=0, stream=None) -> int:
+    """The C split-KV entry point with raw device pointers (ints); returns the status code."""
+    ms = None
+    if mask_strides is not None:
+        arr = (ctypes.c_int64 * 3)(*[int(x) for x in mask_strides])
+        ms = ctypes.cast(arr, ctypes.c_void_p)
+    return int(lib().attn_fwd_splitkv(q, k, v, out, lse, int(B), int(Hq), int(Hkv), int(Nq), int(Nk), int(d),
+                                      float(scale), int(bool(is_causal)), key_lens, additive_mask, ms,
+                                      int(n_splits), workspace, int(workspace_bytes), stream))
+
+
 def attn_check_device_status(stream=None):
     """Synchronises ``stream``; returns (status, raw error word)."""
     info = ctypes.c_uint32(0)
@@ -132,12 +165,16 @@ def _check_bf16_cuda(name, t, ndim):
 
 
 def attention(q, k, v, *, scale: float | None = None, is_causal: bool = False, key_lens=None,
-              attn_mask=None, out=None, lse=None, return_lse: bool = True, stream=None):
+              attn_mask=None, out=None, lse=None, return_lse: bool = True, stream=None,
+              split_kv: int | None = None, workspace=None):
     """O = softmax(scale * Q K^T + mask) V on bf16 CUDA tensors.
 
     q [B, Hq, Nq, d], k/v [B, Hkv, Nk, d] (contiguous bf16); key_lens int32 [B]
     (CUDA) or None; attn_mask fp32 CUDA tensor broadcastable to [B, Hq, Nq, Nk]
-    with a contiguous last dimension, or None.  Returns (out, lse or None).
+    with a contiguous last dimension, or None.  split_kv=None runs attn_fwd;
+    an int runs attn_fwd_splitkv with at most that many key ranges (0 =
+    automatic), its workspace taken from ``workspace`` (a CUDA tensor of at
+    least the planned bytes) or allocated here.  Returns (out, lse or None).
     """
     import torch
     _check_bf16_cuda("q", q, 4)
@@ -175,12 +212,26 @@ def attention(q, k, v, *, scale: float | None = None, is_causal: bool = False, k
         if m.stride(3) != 1:
             m = m.contiguous()
         m_ptr, m_strides = m.data_ptr(), (m.stride(0), m.stride(1), m.stride(2))
-    st = attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                  None if lse is None else lse.data_ptr(), B, Hq, Hkv, Nq, Nk, d,
-                  0.0 if scale is None else float(scale), is_causal, kl_ptr, m_ptr, m_strides,
-                  _stream_handle(stream))
+    sc = 0.0 if scale is None else float(scale)
+    lse_ptr = None if lse is None else lse.data_ptr()
+    if split_kv is None:
+        st = attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse_ptr, B, Hq, Hkv, Nq, Nk, d,
+                      sc, is_causal, kl_ptr, m_ptr, m_strides, _stream_handle(stream))
+        if st != ATTN_OK:
+            raise AttnError(st, "attn_fwd")
+        return out, lse
+    st, _, nbytes = attn_splitkv_plan(B, Hq, Nq, Nk, d, int(split_kv), 0)
     if st != ATTN_OK:
-        raise AttnError(st, "attn_fwd")
+        raise AttnError(st, "attn_splitkv_plan")
+    if workspace is None:
+        workspace = torch.empty((max(nbytes, 1),), dtype=torch.uint8, device=q.device)
+    elif workspace.device != q.device or workspace.numel() * workspace.element_size() < nbytes:
+        raise ValueError(f"workspace must be a CUDA tensor of at least {nbytes} bytes")
+    st = attn_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse_ptr, B, Hq, Hkv, Nq, Nk,
+                          d, sc, is_causal, kl_ptr, m_ptr, m_strides, int(split_kv), workspace.data_ptr(),
+                          workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd_splitkv")
     return out, lse
 
 
@@ -196,10 +247,12 @@ class HostAttention:
 
     Each call copies Q, K, V (and key lengths) host -> device on ``stream``,
     runs ``attn_fwd`` and copies O and LSE back into the host tensors it was
-    given; the device staging buffers are allocated once, here, and reused.
+    given; the device staging buffers (and a split-KV workspace when
+    ``split_kv`` is not None) are allocated once, here, and reused.
     """
 
-    def __init__(self, B, Hq, Hkv, Nq, Nk, d, device="cuda:0", with_lse=True, with_key_lens=False):
+    def __init__(self, B, Hq, Hkv, Nq, Nk, d, device="cuda:0", with_lse=True, with_key_lens=False,
+                 split_kv=None):
         import torch
         dev = torch.device(device)
         bf = torch.bfloat16
@@ -210,6 +263,13 @@ class HostAttention:
         self.out = torch.empty((B, Hq, Nq, d), dtype=bf, device=dev)
         self.lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=dev) if with_lse else None
         self.key_lens = torch.empty((B,), dtype=torch.int32, device=dev) if with_key_lens else None
+        self.split_kv = split_kv
+        self.workspace = None
+        if split_kv is not None:
+            st, _, nbytes = attn_splitkv_plan(B, Hq, Nq, Nk, d, int(split_kv), 0)
+            if st != ATTN_OK:
+                raise AttnError(st, "attn_splitkv_plan")
+            self.workspace = torch.empty((max(nbytes, 1),), dtype=torch.uint8, device=dev)
 
     def __call__(self, q_h, k_h, v_h, out_h, lse_h=None, key_lens_h=None, *, scale=None,
                  is_causal=False, stream=None):
@@ -224,7 +284,8 @@ class HostAttention:
                 self.key_lens.copy_(key_lens_h, non_blocking=True)
                 kl = self.key_lens
             attention(self.q, self.k, self.v, scale=scale, is_causal=is_causal, key_lens=kl,
-                      out=self.out, lse=self.lse, return_lse=self.lse is not None, stream=s)
+                      out=self.out, lse=self.lse, return_lse=self.lse is not None, stream=s,
+                      split_kv=self.split_kv, workspace=self.workspace)
             out_h.copy_(self.out, non_blocking=True)
             if lse_h is not None and self.lse is not None:
                 lse_h.copy_(self.lse, non_blocking=True)

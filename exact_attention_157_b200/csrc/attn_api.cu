@@ -55,8 +55,11 @@ constexpr int kSlots64 = 8, kQStages64 = 2;
 
 template <int D, int NSLOT, int QS, bool M>
 cudaError_t set_pp_attrs() {
-    return cudaFuncSetAttribute(attn_fwd_pp_kernel<D, NSLOT, QS, M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                SmemPP<D, NSLOT, QS>::kAlloc);
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_pp_kernel<D, NSLOT, QS, M, false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SmemPP<D, NSLOT, QS>::kAlloc);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(attn_fwd_pp_kernel<D, NSLOT, QS, M, true>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, SmemPP<D, NSLOT, QS>::kAlloc);
 }
 
 // One-time per-device set-up: architecture check, SM count, kernel attributes,
@@ -116,21 +119,58 @@ attn_status_t encode_map(CUtensorMap* map, const void* base, int d, int rows, lo
 template <int D, int NSLOT, int QS, bool M>
 cudaError_t launch_pp(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
                       const FwdParams& p, unsigned grid, cudaStream_t stream) {
-    attn_fwd_pp_kernel<D, NSLOT, QS, M><<<grid, kPPThreads, SmemPP<D, NSLOT, QS>::kAlloc, stream>>>(tq, tk, tv, to, p);
+    if (p.n_splits > 1)
+        attn_fwd_pp_kernel<D, NSLOT, QS, M, true>
+            <<<grid, kPPThreads, SmemPP<D, NSLOT, QS>::kAlloc, stream>>>(tq, tk, tv, to, p);
+    else
+        attn_fwd_pp_kernel<D, NSLOT, QS, M, false>
+            <<<grid, kPPThreads, SmemPP<D, NSLOT, QS>::kAlloc, stream>>>(tq, tk, tv, to, p);
     return cudaGetLastError();
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-}  // namespace
+constexpr size_t kWsAlign = 256;
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-extern "C" {
+// Workspace of a split-KV launch: partial O (fp32, [n_splits][B*Hq*Nq][d]) then
+// partial LSE (fp32, [n_splits][B*Hq*Nq]), each rounded up to 256 bytes.
+size_t splitkv_bytes(long long rows, int d, int n_splits) {
+    return round_up(static_cast<size_t>(n_splits) * rows * d * sizeof(float), kWsAlign) +
+           round_up(static_cast<size_t>(n_splits) * rows * sizeof(float), kWsAlign);
+}
 
-attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
+// Number of key ranges: the smallest-cost choice under a plain model in which a
+// wave of `sms` concurrent units takes (key blocks per range + kUnitOverhead)
+// block-times, and a unit count that is not a multiple of `sms` wastes the rest
+// of its last wave.  `requested` > 0 is taken as an upper bound.
+constexpr int kMaxSplits = 128;
+constexpr int kUnitOverheadBlocks = 2;
+int choose_splits(long long base_units, int Nk, int sms, int requested) {
+    const int n_blocks = (Nk + kBN - 1) / kBN;
+    if (requested > 0) return requested < n_blocks ? requested : n_blocks;
+    const int hi = kMaxSplits < n_blocks ? kMaxSplits : n_blocks;
+    int best = 1;
+    long long best_cost = -1;
+    for (int s = 1; s <= hi; ++s) {
+        const int per = (n_blocks + s - 1) / s;
+        const int s_eff = (n_blocks + per - 1) / per;  // ranges that hold keys
+        if (s_eff != s) continue;
+        const long long waves = (base_units * s + sms - 1) / sms;
+        const long long cost = waves * (per + kUnitOverheadBlocks);
+        if (best_cost < 0 || cost < best_cost) { best_cost = cost; best = s; }
+    }
+    return best;
+}
+
+
+// Shared by attn_fwd (n_splits = 1) and attn_fwd_splitkv.
+attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, float* lse,
                        int B, int Hq, int Hkv, int Nq, int Nk, int d,
                        float scale, int is_causal,
                        const int32_t* key_lens,
                        const float* additive_mask, const int64_t* mask_strides,
+                       bool split_kv, int n_splits_req, void* workspace, size_t workspace_bytes,
                        void* stream) {
     // ---- host-side validation (no CUDA call before this passes)
     if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return ATTN_ERR_INVALID_ARG;
@@ -157,6 +197,9 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* out, f
             msb = msh * Hq;
         }
     }
+
+    if (split_kv && (n_splits_req < 0 || (workspace != nullptr && reinterpret_cast<uintptr_t>(workspace) % kWsAlign)))
+        return n_splits_req < 0 ? ATTN_ERR_INVALID_ARG : ATTN_ERR_ALIGNMENT;
 
     int dev = 0;
     attn_status_t st = device_setup(&dev);
@@ -189,9 +232,29 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* out, f
     // Work units of 256 query rows (two tiles sharing each K/V block); one
     // persistent CTA per SM loops over them.
     p.n_qtiles = static_cast<int>((static_cast<long long>(Nq) + 2 * kBM - 1) / (2 * kBM));
-    const long long n_units = static_cast<long long>(B) * Hq * p.n_qtiles;
-    if (n_units > (1LL << 30)) return ATTN_ERR_INVALID_ARG;  // unit sequence positions stay in int range
     const int sms = g_dev[dev].sm_count > 0 ? g_dev[dev].sm_count : 1;
+    const long long rows = static_cast<long long>(B) * Hq * Nq;
+    p.n_splits = 1;
+    p.split_keys = (Nk + kBN - 1) / kBN * kBN;
+    p.ws_o = nullptr;
+    p.ws_lse = nullptr;
+    if (split_kv) {
+        const int n_splits = choose_splits(static_cast<long long>(B) * Hq * p.n_qtiles, Nk, sms, n_splits_req);
+        const int n_blocks = (Nk + kBN - 1) / kBN;
+        const int per = (n_blocks + n_splits - 1) / n_splits;
+        p.n_splits = (n_blocks + per - 1) / per;
+        if (p.n_splits > 1) {
+            p.split_keys = per * kBN;
+            if (workspace == nullptr || workspace_bytes < splitkv_bytes(rows, d, p.n_splits))
+                return ATTN_ERR_INVALID_ARG;
+            p.ws_o = static_cast<float*>(workspace);
+            p.ws_lse = reinterpret_cast<float*>(
+                static_cast<char*>(workspace) +
+                round_up(static_cast<size_t>(p.n_splits) * rows * d * sizeof(float), kWsAlign));
+        }
+    }
+    const long long n_units = static_cast<long long>(B) * Hq * p.n_qtiles * p.n_splits;
+    if (n_units > (1LL << 30)) return ATTN_ERR_INVALID_ARG;  // unit sequence positions stay in int range
     // Causal units differ in cost: with at least two units per SM, each CTA
     // takes heavy/light pairs of one head (equal cost per pair).
     p.unit_run = (is_causal && n_units >= 2LL * sms) ? 2 : 1;
@@ -204,7 +267,65 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* out, f
         e = has_mask ? launch_pp<64, kSlots64, kQStages64, true>(tq, tk, tv, to, p, g, s)
                      : launch_pp<64, kSlots64, kQStages64, false>(tq, tk, tv, to, p, g, s);
     if (e != cudaSuccess) return cuda_fail(e);
+    if (p.n_splits > 1) {
+        // merge the key ranges' partial results into out (bf16) and lse
+        const unsigned cg = static_cast<unsigned>((rows + 7) / 8);
+        if (d == 128)
+            attn_splitkv_combine_kernel<128><<<cg, 256, 0, s>>>(p.ws_o, p.ws_lse, static_cast<__nv_bfloat16*>(out),
+                                                                lse, rows, p.n_splits);
+        else
+            attn_splitkv_combine_kernel<64><<<cg, 256, 0, s>>>(p.ws_o, p.ws_lse, static_cast<__nv_bfloat16*>(out),
+                                                               lse, rows, p.n_splits);
+        if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
+    }
     return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
+                       int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                       float scale, int is_causal,
+                       const int32_t* key_lens,
+                       const float* additive_mask, const int64_t* mask_strides,
+                       void* stream) {
+    return fwd_impl(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, is_causal, key_lens, additive_mask,
+                    mask_strides, false, 1, nullptr, 0, stream);
+}
+
+attn_status_t attn_splitkv_plan(int B, int Hq, int Nq, int Nk, int d, int n_splits, int sm_count,
+                                int* n_splits_out, size_t* workspace_bytes) {
+    if (B <= 0 || Hq <= 0 || Nq <= 0 || Nk <= 0 || d <= 0 || n_splits < 0 || sm_count < 0) return ATTN_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+    int sms = sm_count;
+    if (sms == 0) {
+        int dev = 0;
+        attn_status_t st = device_setup(&dev);
+        if (st != ATTN_OK) return st;
+        sms = g_dev[dev].sm_count > 0 ? g_dev[dev].sm_count : 1;
+    }
+    const long long n_qtiles = (static_cast<long long>(Nq) + 2 * kBM - 1) / (2 * kBM);
+    const int chosen = choose_splits(static_cast<long long>(B) * Hq * n_qtiles, Nk, sms, n_splits);
+    const int n_blocks = (Nk + kBN - 1) / kBN;
+    const int per = (n_blocks + chosen - 1) / chosen;
+    const int used = (n_blocks + per - 1) / per;
+    if (n_splits_out != nullptr) *n_splits_out = used;
+    if (workspace_bytes != nullptr)
+        *workspace_bytes = used > 1 ? splitkv_bytes(static_cast<long long>(B) * Hq * Nq, d, used) : 0;
+    return ATTN_OK;
+}
+
+attn_status_t attn_fwd_splitkv(const void* q, const void* k, const void* v, void* out, float* lse,
+                               int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                               float scale, int is_causal,
+                               const int32_t* key_lens,
+                               const float* additive_mask, const int64_t* mask_strides,
+                               int n_splits, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+    return fwd_impl(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, is_causal, key_lens, additive_mask,
+                    mask_strides, true, n_splits, workspace, workspace_bytes, stream);
 }
 
 attn_status_t attn_check_device_status(void* stream, uint32_t* info) {

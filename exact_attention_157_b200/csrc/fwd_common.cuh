@@ -29,9 +29,60 @@ struct FwdParams {
     float* lse;
     void* out;     // O base (bf16), for rows written without the TMA store
     int unit_run;  // persistent kernel: consecutive units per CTA turn (1 or 2)
+    // split-KV mode: every unit covers one range of split_keys keys (a multiple of
+    // 128); partial results go to the workspace, [n_splits][B*Hq][Nq][d] for O
+    // (fp32, normalised by the partial row sum) and [n_splits][B*Hq][Nq] for LSE
+    int n_splits;
+    int split_keys;
+    float* ws_o;
+    float* ws_lse;
     unsigned long long timeout_ns;
     unsigned int epoch;  // launch id for the launch-wide abort (never 0)
 };
+
+// Split-KV combine: for each output row, merge the n_splits partial results
+// (O_s normalised by its own row sum, LSE_s) of disjoint key ranges:
+//   M = max_s LSE_s,  w_s = exp(LSE_s - M),  O = sum_s w_s O_s / sum_s w_s,
+//   LSE = M + ln sum_s w_s
+// (exact: each w_s is proportional to the sum of exp(score) over range s).  A row
+// with no key in any range gives O = 0, LSE = -inf.  One warp per row; lane i
+// holds columns 4i .. 4i+3 (d = 128) or 2i .. 2i+1 (d = 64).
+template <int D>
+__global__ void __launch_bounds__(256) attn_splitkv_combine_kernel(const float* __restrict__ ws_o,
+                                                                  const float* __restrict__ ws_lse,
+                                                                  __nv_bfloat16* __restrict__ out,
+                                                                  float* __restrict__ lse, long long rows,
+                                                                  int n_splits) {
+    constexpr int kPer = D / 32;
+    const long long r = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (r >= rows) return;
+    float m = -INFINITY;
+    for (int s = lane; s < n_splits; s += 32) m = fmaxf(m, ws_lse[s * rows + r]);
+    #pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float acc[kPer];
+    #pragma unroll
+    for (int i = 0; i < kPer; ++i) acc[i] = 0.0f;
+    float wsum = 0.0f;
+    if (m != -INFINITY) {
+        for (int s = 0; s < n_splits; ++s) {
+            const float ls = ws_lse[s * rows + r];
+            if (ls == -INFINITY) continue;
+            const float w = __expf(ls - m);
+            wsum += w;
+            const float* src = ws_o + (s * rows + r) * D + lane * kPer;
+            #pragma unroll
+            for (int i = 0; i < kPer; ++i) acc[i] = fmaf(w, src[i], acc[i]);
+        }
+    }
+    const float inv = wsum > 0.0f ? 1.0f / wsum : 0.0f;
+    __nv_bfloat16* dst = out + r * D + lane * kPer;
+    #pragma unroll
+    for (int i = 0; i < kPer; i += 2)
+        *reinterpret_cast<__nv_bfloat162*>(dst + i) = __floats2bfloat162_rn(acc[i] * inv, acc[i + 1] * inv);
+    if (lane == 0 && lse != nullptr) lse[r] = wsum > 0.0f ? m + __logf(wsum) : -INFINITY;
+}
 
 // Waits on a barrier nothing arrives at; the bounded wait must expire.
 __global__ void attn_selftest_timeout_kernel(unsigned long long timeout_ns, unsigned int epoch) {

@@ -54,6 +54,15 @@ constexpr int kRegsSoftmax = 200;
 constexpr int kRegsControl = 104;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl <= kPPThreads * 168, "register split");
 
+// P_t(j) is stored and signalled in kPChunks equal chunks of keys, so that the
+// PV over the first chunks runs while the softmax computes the last ones.
+#ifndef ATTN_P_CHUNKS
+#define ATTN_P_CHUNKS 2
+#endif
+constexpr int kPChunks = ATTN_P_CHUNKS;
+static_assert(kPChunks == 2 || kPChunks == 4, "P is released in 2 or 4 chunks");
+constexpr int kChunkKeys = kBN / kPChunks;
+
 template <int D, int NSLOT, int QS>
 struct SmemPP {
     static constexpr int kChunks = D / 64;
@@ -69,11 +78,10 @@ struct SmemPP {
     static constexpr int FULL = 2 * QS;               // NSLOT: K/V slot loaded
     static constexpr int EMPTY = 2 * QS + NSLOT;      // NSLOT: K/V slot released
     static constexpr int SFULL = 2 * QS + 2 * NSLOT;  // 2: S_t(j) complete
-    static constexpr int P0 = SFULL + 2;              // 2: P_t(j) keys 0..63 stored (128 arrivals)
-    static constexpr int P1 = SFULL + 4;              // 2: P_t(j) keys 64..127 stored (128 arrivals)
-    static constexpr int OFINAL = SFULL + 6;          // 2: last PV_t of a unit complete
-    static constexpr int OEMPTY = SFULL + 8;          // 2: O_t read out by the epilogue (128 arrivals)
-    static constexpr int MMAFIN = SFULL + 10;
+    static constexpr int PCH = SFULL + 2;             // 2 x kPChunks: chunk c of P_t(j) stored (128 arrivals)
+    static constexpr int OFINAL = PCH + 2 * kPChunks; // 2: last PV_t of a unit complete
+    static constexpr int OEMPTY = OFINAL + 2;         // 2: O_t read out by the epilogue (128 arrivals)
+    static constexpr int MMAFIN = OEMPTY + 2;
     static constexpr int kNumBars = MMAFIN + 1;
     static constexpr int kMisc = kBars + 8 * kNumBars;
     static constexpr int kBytes = kMisc + 16;
@@ -148,6 +156,7 @@ __device__ __forceinline__ void exp2_poly_pair(uint64_t x, float& e0, float& e1)
 // Everything about one work unit that every role derives identically.
 struct Unit {
     int bh, b, h, bhk, q0, kv_len;
+    int split, j_lo;  // split-KV: key range index and its first key block
     int n_t[2];  // key blocks of tile A / B (0: nothing to compute)
     bool tile_b_valid;
     __device__ __forceinline__ int n_max() const { return n_t[0] > n_t[1] ? n_t[0] : n_t[1]; }
@@ -165,13 +174,18 @@ __device__ __forceinline__ int unit_seq(int c, int k, int G, int P) {
 // the critical path).
 __device__ __forceinline__ int unit_key_len(const FwdParams& p, int s, int n_units) {
     if (p.key_lens == nullptr || s >= n_units) return p.Nk;
-    return __ldg(p.key_lens + (s / p.n_qtiles) / p.Hq);
+    return __ldg(p.key_lens + (s / (p.n_qtiles * p.n_splits)) / p.Hq);
 }
 
+// Units are numbered (head, split, query-unit): the units of one head and key
+// range are adjacent.  Without split-KV, n_splits = 1.
 __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int s, int kv_len, bool report) {
     Unit x;
-    x.bh = s / p.n_qtiles;
-    const int pos = s - x.bh * p.n_qtiles;
+    const int per_head = p.n_qtiles * p.n_splits;
+    x.bh = s / per_head;
+    const int r = s - x.bh * per_head;
+    x.split = r / p.n_qtiles;
+    const int pos = r - x.split * p.n_qtiles;
     // causal: heavy and light query tiles alternate (n-1, 0, n-2, 1, ...)
     const int qt = !p.is_causal ? pos : (pos & 1) ? (pos >> 1) : p.n_qtiles - 1 - (pos >> 1);
     x.b = x.bh / p.Hq;
@@ -184,17 +198,20 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int s, int kv_le
         kv_len = kv_len < 0 ? 0 : p.Nk;
     }
     x.kv_len = kv_len;
+    const int k_lo = x.split * p.split_keys;  // a multiple of kBN
+    x.j_lo = k_lo / kBN;
     #pragma unroll
     for (int t = 0; t < 2; ++t) {
         int end = x.kv_len;
         if (p.is_causal && x.q0 + (t + 1) * kBM < end) end = x.q0 + (t + 1) * kBM;
-        x.n_t[t] = (end + kBN - 1) / kBN;
+        if (k_lo + p.split_keys < end) end = k_lo + p.split_keys;
+        x.n_t[t] = end > k_lo ? (end - k_lo + kBN - 1) / kBN : 0;
     }
     if (!x.tile_b_valid) x.n_t[1] = 0;
     return x;
 }
 
-template <int D, int NSLOT, int QS, bool HAS_MASK>
+template <int D, int NSLOT, int QS, bool HAS_MASK, bool SPLIT>
 __global__ void __launch_bounds__(kPPThreads, 1)
 attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -207,7 +224,8 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int n_units = p.B * p.Hq * p.n_qtiles;  // p.n_qtiles counts 256-row units per head
+    // p.n_qtiles counts 256-row units per head; p.n_splits key ranges per head
+    const int n_units = p.B * p.Hq * p.n_qtiles * p.n_splits;
 
     auto bar = [&](int i) -> uint32_t { return sbase + L::kBars + 8u * i; };
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
@@ -224,8 +242,7 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         }
         for (int t = 0; t < 2; ++t) {
             mbar_init(bar(L::SFULL + t), 1);
-            mbar_init(bar(L::P0 + t), 128);
-            mbar_init(bar(L::P1 + t), 128);
+            for (int c = 0; c < kPChunks; ++c) mbar_init(bar(L::PCH + t * kPChunks + c), 128);
             mbar_init(bar(L::OFINAL + t), 1);
             mbar_init(bar(L::OEMPTY + t), 128);
         }
@@ -299,7 +316,7 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     #pragma unroll
                     for (int c = 0; c < L::kChunks; ++c)
                         tma_load_3d(sbase + L::kRing + s * L::kTileBytes + c * L::kChunkBytes, map, bar(L::FULL + s),
-                                    c * 64, (i >> 1) * kBN, x.bhk);
+                                    c * 64, (x.j_lo + (i >> 1)) * kBN, x.bhk);
                     uses[s] = use + 1;
                 }
             }
@@ -320,7 +337,7 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             #pragma unroll
             for (int q = 0; q < QS; ++q) q_loads[q] = 0;
             int i_glob = 0;      // K/V loads consumed so far
-            int gp[2] = {0, 0};  // P_t blocks consumed so far (P0 / P1 phase)
+            int gp[2] = {0, 0};  // P_t blocks consumed so far (P chunk barrier phase)
             bool ok = true;
             int it = 0;
             int kv_next = unit_key_len(p, unit_seq(cta, 0, G, p.unit_run), n_units);
@@ -347,14 +364,14 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     }
                     mma_commit(bar(L::SFULL + t));
                 };
-                // O_t += P_t(j)[:, keys 64 half .. +63] V_j[those keys, :]
-                auto issue_pv = [&](int t, int j, int half) {
+                // O_t += P_t(j)[:, keys of chunk c] V_j[those keys, :]
+                auto issue_pv = [&](int t, int j, int c) {
                     const uint32_t v_addr = sbase + L::kRing + slot_of(2 * j + 1) * L::kTileBytes;
                     const uint32_t o_tmem = tmem + L::kColO + t * D;
                     const uint32_t p_tmem = tmem + t * 128;
                     #pragma unroll
-                    for (int k4 = 0; k4 < kBN / 32; ++k4) {
-                        const int kk = half * (kBN / 32) + k4;
+                    for (int k4 = 0; k4 < kChunkKeys / 16; ++k4) {
+                        const int kk = c * (kChunkKeys / 16) + k4;
                         mma_ts(o_tmem, p_tmem + kk * 8, smem_desc_sw128(v_addr + kk * 2048, L::kChunkBytes, 1024),
                                kIdescO, (j > 0 || kk > 0) ? 1u : 0u);
                     }
@@ -371,24 +388,26 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     bool v_ready = false, k_next_ready = false;
                     for (int t = 0; t < 2 && ok; ++t) {
                         if (j >= x.n_t[t]) continue;
-                        // first half of P_t(j): PV over keys 0..63 overlaps the rest of the softmax
-                        if (!mbar_wait(bar(L::P0 + t), gp[t] & 1, limit, abort_flag, p.epoch, kRoleMma, 22))
-                            { ok = false; break; }
-                        // the previous unit's epilogue must have read O_t out of TMEM
-                        if (j == 0 && it > 0 &&
-                            !mbar_wait(bar(L::OEMPTY + t), (it - 1) & 1, limit, abort_flag, p.epoch, kRoleMma, 23))
-                            { ok = false; break; }
-                        if (!v_ready) {
-                            if (!wait_full(2 * j + 1, 24)) { ok = false; break; }
-                            v_ready = true;
+                        // P_t(j) arrives in chunks: the PV over the first ones overlaps the rest of
+                        // the softmax
+                        for (int c = 0; ok && c < kPChunks; ++c) {
+                            if (!mbar_wait(bar(L::PCH + t * kPChunks + c), gp[t] & 1, limit, abort_flag, p.epoch,
+                                           kRoleMma, 22)) { ok = false; break; }
+                            if (c == 0) {
+                                // the previous unit's epilogue must have read O_t out of TMEM
+                                if (j == 0 && it > 0 &&
+                                    !mbar_wait(bar(L::OEMPTY + t), (it - 1) & 1, limit, abort_flag, p.epoch, kRoleMma,
+                                               23)) { ok = false; break; }
+                                if (!v_ready) {
+                                    if (!wait_full(2 * j + 1, 24)) { ok = false; break; }
+                                    v_ready = true;
+                                }
+                            }
+                            tc_fence_after();
+                            issue_pv(t, j, c);
                         }
-                        tc_fence_after();
-                        issue_pv(t, j, 0);
-                        if (!mbar_wait(bar(L::P1 + t), gp[t] & 1, limit, abort_flag, p.epoch, kRoleMma, 27))
-                            { ok = false; break; }
+                        if (!ok) break;
                         ++gp[t];
-                        tc_fence_after();
-                        issue_pv(t, j, 1);
                         if (j + 1 < x.n_t[t]) {
                             if (!k_next_ready) {
                                 if (!wait_full(2 * j + 2, 25)) { ok = false; break; }
@@ -454,13 +473,12 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     tmem_ld32(s_tmem + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
                 tmem_wait_ld();
                 float* s = reinterpret_cast<float*>(sr);
-                const int j0 = j * kBN;
+                const int j0 = (x.j_lo + j) * kBN;
                 const bool boundary = (j0 + kBN > kv_len) || (p.is_causal && j0 + kBN - 1 > q0_t);
 
                 float mx;
                 if constexpr (HAS_MASK) {
                     mx = -INFINITY;
-                    #pragma unroll
                     // keys c >= lim are masked (past the end of K, or past the diagonal)
                     int lim = mask_row != nullptr ? kv_len - j0 : 0;
                     if (p.is_causal && q_idx - j0 + 1 < lim) lim = q_idx - j0 + 1;
@@ -499,8 +517,8 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 // warp-collective, but rows that keep their max use alpha = 1 exactly, so a
                 // row's result never depends on the other rows of its warp.  O_t holds
                 // sum_{i<j} P_i V_i here (S_t(j) was issued after PV_t(j-1)); the rescale
-                // of O_t itself is done after the first half of P_t is stored (fewer live
-                // registers) and before the P0 arrive that lets PV_t(j) start.
+                // of O_t itself is done after the first chunk of P_t is stored (fewer live
+                // registers) and before that chunk's signal lets PV_t(j) start.
                 const bool need = mx > m_used + kLazyTau;
                 const bool warp_rescale = __any_sync(0xffffffffu, need) && j > 0;
                 float alpha = 1.0f;
@@ -516,26 +534,26 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 // just before it: (1) exponent arguments, (2) exponentials, (3) row sum and
                 // bf16 packing.
                 uint64_t acc0 = 0, acc1 = 0, acc2 = 0, acc3 = 0;  // packed partial sums
-                uint32_t pk[kBN / 4];
-                // Keys 0..63, then 64..127: each half is stored and signalled on its own
-                // (P0, P1), so PV over the first half runs during the second half.  O_t is
-                // rescaled (if needed) before P0 releases the first PV.
-                auto exp_half = [&](auto emulate, auto half_c) {
-                    constexpr int h = decltype(half_c)::value;
-                    float* sh = s + h * (kBN / 2);
+                uint32_t pk[kChunkKeys / 2];
+                // Chunk by chunk of keys: each chunk is stored and signalled on its own, so
+                // the PV over earlier chunks runs during the later ones.  O_t is rescaled
+                // (if needed) before the first chunk's signal releases the first PV.
+                auto exp_chunk = [&](auto emulate, auto chunk_c) {
+                    constexpr int cc = decltype(chunk_c)::value;
+                    float* sh = s + cc * kChunkKeys;
                     if constexpr (HAS_MASK) {
                         #pragma unroll
-                        for (int c = 0; c < kBN / 2; ++c) sh[c] = sh[c] - shift;
+                        for (int c = 0; c < kChunkKeys; ++c) sh[c] = sh[c] - shift;
                     } else {
                         #pragma unroll
-                        for (int c = 0; c < kBN / 4; ++c) {
+                        for (int c = 0; c < kChunkKeys / 2; ++c) {
                             const uint64_t xv = ffma2(pack_f32x2(sh[2 * c], sh[2 * c + 1]), c2, nshift2);
                             sh[2 * c] = lo_f32(xv);
                             sh[2 * c + 1] = hi_f32(xv);
                         }
                     }
                     #pragma unroll
-                    for (int c = 0; c < kBN / 4; ++c) {
+                    for (int c = 0; c < kChunkKeys / 2; ++c) {
                         if (decltype(emulate)::value &&
                             (c % (kExp2EmuEvery > 0 ? kExp2EmuEvery : 1)) == kExp2EmuEvery - 1) {
                             exp2_poly_pair(pack_f32x2(sh[2 * c], sh[2 * c + 1]), sh[2 * c], sh[2 * c + 1]);
@@ -545,7 +563,7 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         }
                     }
                     #pragma unroll
-                    for (int c = 0; c < kBN / 4; ++c) {
+                    for (int c = 0; c < kChunkKeys / 2; ++c) {
                         const uint64_t e = pack_f32x2(sh[2 * c], sh[2 * c + 1]);
                         switch (c & 3) {
                             case 0: acc0 = fadd2(acc0, e); break;
@@ -555,8 +573,12 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         }
                         pk[c] = pack_bf16x2(sh[2 * c], sh[2 * c + 1]);
                     }
-                    tmem_st32(s_tmem + h * 32, pk);
-                    if (h == 0 && warp_rescale) {
+                    if constexpr (kChunkKeys == 64) {
+                        tmem_st32(s_tmem + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+                    } else {
+                        tmem_st16(s_tmem + cc * (kChunkKeys / 2), pk);
+                    }
+                    if (cc == 0 && warp_rescale) {
                         #pragma unroll
                         for (int c = 0; c < D / 32; ++c) {
                             uint32_t o[32];
@@ -569,34 +591,52 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     }
                     tmem_wait_st();
                     tc_fence_before();
-                    mbar_arrive(bar((h == 0 ? L::P0 : L::P1) + t));
+                    mbar_arrive(bar(L::PCH + t * kPChunks + cc));
                 };
-                using Half0 = std::integral_constant<int, 0>;
-                using Half1 = std::integral_constant<int, 1>;
-                if (kExp2EmuEvery > 0 && !HAS_MASK && !boundary) {
-                    exp_half(std::integral_constant<bool, kExp2EmuEvery != 0>{}, Half0{});
-                    exp_half(std::integral_constant<bool, kExp2EmuEvery != 0>{}, Half1{});
-                } else {
-                    exp_half(std::false_type{}, Half0{});
-                    exp_half(std::false_type{}, Half1{});
-                }
+                auto all_chunks = [&](auto emulate) {
+                    exp_chunk(emulate, std::integral_constant<int, 0>{});
+                    exp_chunk(emulate, std::integral_constant<int, 1>{});
+                    if constexpr (kPChunks == 4) {
+                        exp_chunk(emulate, std::integral_constant<int, 2>{});
+                        exp_chunk(emulate, std::integral_constant<int, 3>{});
+                    }
+                };
+                if (kExp2EmuEvery > 0 && !HAS_MASK && !boundary)
+                    all_chunks(std::integral_constant<bool, kExp2EmuEvery != 0>{});
+                else
+                    all_chunks(std::false_type{});
                 const uint64_t acc = fadd2(fadd2(acc0, acc2), fadd2(acc1, acc3));
                 l_sum += lo_f32(acc) + hi_f32(acc);
             }
 
             // ------------------------------------------------------------ epilogue
             const int qb = it % QS;
+            // QEMPTY expects two arrivals per loaded unit.  Only a tile with key blocks
+            // arrives (on behalf of both when the other tile has none): a tile without
+            // work waits on nothing, so its arrivals could run ahead into a later
+            // unit's phase of the barrier.
+            auto release_q = [&](int b) {
+                if (x.n_t[t] > 0) mbar_arrive_cnt(bar(L::QEMPTY + b), x.n_t[t ^ 1] > 0 ? 1u : 2u);
+            };
             if (x.n_max() == 0) {
                 // No unmasked key at all (key length 0): O = 0, LSE = -inf, written
                 // directly (this unit loaded nothing and owns no Q buffer).
                 tc_fence_before();
                 mbar_arrive(bar(L::OEMPTY + t));
                 if (q_idx < p.Nq && ok && !*abort_flag) {
-                    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) +
-                                                          (static_cast<long long>(x.bh) * p.Nq + q_idx) * D);
-                    #pragma unroll
-                    for (int v = 0; v < D / 8; ++v) dst[v] = make_uint4(0u, 0u, 0u, 0u);
-                    if (p.lse != nullptr) p.lse[static_cast<long long>(x.bh) * p.Nq + q_idx] = -INFINITY;
+                    const long long r = static_cast<long long>(x.bh) * p.Nq + q_idx;
+                    if constexpr (SPLIT) {
+                        const long long rs = static_cast<long long>(x.split) * p.B * p.Hq * p.Nq + r;
+                        float4* dst = reinterpret_cast<float4*>(p.ws_o + rs * D);
+                        #pragma unroll
+                        for (int v = 0; v < D / 4; ++v) dst[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+                        p.ws_lse[rs] = -INFINITY;
+                    } else {
+                        uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + r * D);
+                        #pragma unroll
+                        for (int v = 0; v < D / 8; ++v) dst[v] = make_uint4(0u, 0u, 0u, 0u);
+                        if (p.lse != nullptr) p.lse[r] = -INFINITY;
+                    }
                 }
                 continue;
             }
@@ -609,6 +649,37 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             const bool do_epilogue = __all_sync(0xffffffffu, ok && !*abort_flag) && q0_t < p.Nq;
             uint8_t* stage = smem + L::kQ + qb * L::kQBuf + t * L::kTileBytes;  // Q_t is dead after OFINAL_t
             const float inv_l = l_sum > 0.0f ? 1.0f / l_sum : 0.0f;
+            if constexpr (SPLIT) {
+                // Split-KV: this key range's O (normalised by its own row sum) and LSE go
+                // to the workspace in fp32, row by row; the combine kernel merges them.
+                const long long rs = (static_cast<long long>(x.split) * p.B * p.Hq + x.bh) * p.Nq + q_idx;
+                #pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t o[32];
+                    if (n_blocks > 0 && do_epilogue) {
+                        tmem_ld32(o_tmem + c * 32, o);
+                        tmem_wait_ld();
+                    } else {
+                        #pragma unroll
+                        for (int v = 0; v < 32; ++v) o[v] = 0u;
+                    }
+                    if (c == D / 32 - 1) {
+                        tc_fence_before();
+                        mbar_arrive(bar(L::OEMPTY + t));
+                    }
+                    if (do_epilogue && q_idx < p.Nq) {
+                        float4* dst = reinterpret_cast<float4*>(p.ws_o + rs * D + c * 32);
+                        #pragma unroll
+                        for (int v = 0; v < 8; ++v)
+                            dst[v] = make_float4(__uint_as_float(o[4 * v]) * inv_l, __uint_as_float(o[4 * v + 1]) * inv_l,
+                                                 __uint_as_float(o[4 * v + 2]) * inv_l, __uint_as_float(o[4 * v + 3]) * inv_l);
+                    }
+                }
+                if (do_epilogue && q_idx < p.Nq)
+                    p.ws_lse[rs] = l_sum > 0.0f ? (m_used + __log2f(l_sum)) * kLn2 : -INFINITY;
+                named_barrier_sync(1 + t, 128);
+                if ((threadIdx.x & 127) == 0) release_q(qb);
+            } else {
             #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t o[32];
@@ -655,8 +726,9 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     bulk_commit_group();
                     bulk_wait_group_read0();
                 }
-                mbar_arrive(bar(L::QEMPTY + qb));  // the producer may refill this Q buffer
+                release_q(qb);  // the producer may refill this Q buffer
             }
+            }  // !SPLIT
         }
     }
 

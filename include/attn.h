@@ -27,6 +27,7 @@
 #ifndef ATTN_H_
 #define ATTN_H_
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -82,6 +83,56 @@ attn_status_t attn_fwd(const void *q, const void *k, const void *v, void *out, f
                        const int32_t *key_lens,
                        const float *additive_mask, const int64_t *mask_strides,
                        void *stream);
+
+/*
+ * attn_splitkv_plan -- how attn_fwd_splitkv would split the keys, and the
+ * workspace it then needs.  Host-only arithmetic (no CUDA call) when
+ * sm_count > 0; sm_count == 0 queries the current device's SM count.
+ *   n_splits: 0 = choose automatically; k > 0 = at most k ranges.
+ *   n_splits_out (host, may be NULL): key ranges actually used (1 = no split,
+ *     the launch then writes out directly and needs no workspace).
+ *   workspace_bytes (host, may be NULL): bytes of device workspace needed.
+ * The keys are cut into n_splits_out ranges of equal length (a multiple of
+ * 128 keys; the last may be shorter).  The automatic choice minimises
+ * (waves of units over the SMs) x (key blocks per range + 2).
+ * Errors: ATTN_ERR_INVALID_ARG for non-positive sizes or negative counts,
+ * ATTN_ERR_UNSUPPORTED for d not in {64, 128}.
+ */
+attn_status_t attn_splitkv_plan(int B, int Hq, int Nq, int Nk, int d, int n_splits, int sm_count,
+                                int *n_splits_out, size_t *workspace_bytes);
+
+/*
+ * attn_fwd_splitkv -- attn_fwd with the keys of every (batch, head) cut into
+ * ranges that run as separate work units, then merged: the decoding-phase
+ * scheme that "FlashAttention technical analysis" (jsqmd.com/news/722897),
+ * section 5.2, names FlashDecoding.  It serves short query blocks (Nq of 1 to
+ * a few hundred) over long key sequences, where B * Hq alone leaves SMs idle.
+ *
+ * Range s gives O_s (its rows normalised by the range's own row sum) and
+ * LSE_s; the merge is exact: with M = max_s LSE_s and w_s = exp(LSE_s - M),
+ * O = sum_s w_s O_s / sum_s w_s and LSE = M + ln(sum_s w_s).  A range with no
+ * unmasked key of a row has LSE_s = -inf and weight 0.
+ *
+ * Arguments as attn_fwd, plus:
+ *   n_splits: 0 = automatic (attn_splitkv_plan), k > 0 = at most k ranges.
+ *   workspace: device, 256-byte aligned, at least the bytes attn_splitkv_plan
+ *     reports for the same sizes (may be NULL when that is 0).  The library
+ *     writes it before reading it (nothing needs to start at zero); its
+ *     contents after the call are unspecified.  Two calls in flight at once
+ *     must not share a workspace.
+ * Two kernels run on `stream`: the attention kernel (partials to the
+ * workspace) and the merge (out, lse); with one range only the first, writing
+ * out directly.
+ * Errors: as attn_fwd; ATTN_ERR_INVALID_ARG also for n_splits < 0 or a
+ * missing / short workspace, ATTN_ERR_ALIGNMENT for a misaligned workspace.
+ */
+attn_status_t attn_fwd_splitkv(const void *q, const void *k, const void *v, void *out, float *lse,
+                               int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                               float scale, int is_causal,
+                               const int32_t *key_lens,
+                               const float *additive_mask, const int64_t *mask_strides,
+                               int n_splits, void *workspace, size_t workspace_bytes,
+                               void *stream);
 
 /*
  * attn_check_device_status -- synchronise `stream`, then read and clear the

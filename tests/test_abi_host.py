@@ -85,3 +85,65 @@ def test_package_does_not_import_oracle():
     assert "oracle" not in src
     for f in os.listdir(os.path.join(ROOT, "exact_attention_157_b200", "csrc")):
         assert "oracle" not in open(os.path.join(ROOT, "exact_attention_157_b200", "csrc", f)).read()
+
+
+# ------------------------------------------------------------------ split-KV plan
+def _ws_bytes(rows, d, s):
+    r = lambda x: (x + 255) // 256 * 256
+    return r(s * rows * d * 4) + r(s * rows * 4)
+
+
+@pytest.mark.parametrize("B,Hq,Nq,Nk,d,req,used", [
+    (8, 32, 1, 16384, 128, 1, 1),
+    (8, 32, 1, 16384, 128, 4, 4),
+    (2, 4, 7, 300, 64, 3, 3),     # 3 key blocks, 3 ranges of one block
+    (2, 4, 7, 300, 64, 5, 3),     # capped at the number of key blocks
+    (2, 4, 7, 512, 64, 3, 2),     # 4 blocks in ranges of ceil(4/3) = 2 blocks -> 2 ranges
+    (1, 1, 1, 100, 128, 8, 1),    # a single key block never splits
+])
+def test_splitkv_plan_requested(B, Hq, Nq, Nk, d, req, used):
+    st, n, nbytes = ea.attn_splitkv_plan(B, Hq, Nq, Nk, d, req, 148)
+    assert st == ea.ATTN_OK
+    assert n == used
+    assert nbytes == (_ws_bytes(B * Hq * Nq, d, n) if n > 1 else 0)
+
+
+@pytest.mark.parametrize("B,Hq,Nq,Nk", [(8, 32, 1, 16384), (1, 8, 4, 32768), (8, 32, 4096, 4096),
+                                         (4, 8, 77, 2000), (1, 1, 1, 1 << 20)])
+def test_splitkv_plan_auto_minimises_stated_cost(B, Hq, Nq, Nk):
+    """The automatic range count is the first minimiser of
+    ceil(units * s / SMs) * (key blocks per range + 2) over range counts s
+    that the equal-length cut realises exactly (the header's model)."""
+    sms = 148
+    nb = -(-Nk // 128)
+    units = B * Hq * (-(-Nq // 256))
+    best, best_cost = 1, None
+    for s in range(1, min(128, nb) + 1):
+        per = -(-nb // s)
+        if -(-nb // per) != s:
+            continue
+        cost = -(-(units * s) // sms) * (per + 2)
+        if best_cost is None or cost < best_cost:
+            best, best_cost = s, cost
+    st, n, _ = ea.attn_splitkv_plan(B, Hq, Nq, Nk, 128, 0, sms)
+    assert st == ea.ATTN_OK and n == best
+
+
+def test_splitkv_plan_rejects_bad_sizes():
+    assert ea.attn_splitkv_plan(0, 1, 1, 1, 64, 0, 148)[0] == ea.ATTN_ERR_INVALID_ARG
+    assert ea.attn_splitkv_plan(1, 1, 1, 1, 64, -1, 148)[0] == ea.ATTN_ERR_INVALID_ARG
+    assert ea.attn_splitkv_plan(1, 1, 1, 1, 64, 0, -5)[0] == ea.ATTN_ERR_INVALID_ARG
+    assert ea.attn_splitkv_plan(1, 1, 1, 1, 96, 0, 148)[0] == ea.ATTN_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("args,status", [
+    (dict(n_splits=-1), ea.ATTN_ERR_INVALID_ARG),
+    (dict(workspace=A + 16), ea.ATTN_ERR_ALIGNMENT),
+    (dict(q=0), ea.ATTN_ERR_INVALID_ARG),
+    (dict(d=96), ea.ATTN_ERR_UNSUPPORTED),
+])
+def test_splitkv_validation_is_host_side(args, status):
+    kw = dict(q=A, k=A, v=A, out=A, lse=None, B=1, Hq=2, Hkv=2, Nq=1, Nk=4096, d=128,
+              scale=0.0, is_causal=0, n_splits=4, workspace=A, workspace_bytes=1 << 20)
+    kw.update(args)
+    assert ea.attn_fwd_splitkv(**kw) == status

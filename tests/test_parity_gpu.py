@@ -74,6 +74,20 @@ def test_shapes_vs_oracle(Nq, Nk, d, causal):
     assert_close(out, lse, ro, rl)
 
 
+@pytest.mark.parametrize("Nq,Nk", [(100, 300), (1, 256), (300, 200)])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_many_units_per_cta_with_idle_tile(Nq, Nk, d, causal):
+    """More work units than SMs, where the second 128-row tile of some or all
+    units has no rows (Nq <= 128, or the last unit of each head at Nq = 300):
+    the persistent CTAs run several such units back to back."""
+    B, Hq, Hkv = 48, 8, 4
+    q, k, v = make_qkv(B, Hq, Hkv, Nq, Nk, d, seed=Nq + Nk + d + causal)
+    out, lse = run_gpu(q, k, v, is_causal=causal)
+    ro, rl = oracle.attention(q, k, v, is_causal=causal)
+    assert_close(out, lse, ro, rl)
+
+
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("causal", [False, True])
 def test_key_lens_vs_oracle(d, causal):
@@ -185,7 +199,7 @@ def test_workload_vs_oracle(name):
     w = WORKLOADS[name]
     dev = torch.device("cuda:0")
     q, k, v, kl = make_inputs(w, device=dev)
-    out, lse = ea.attention(q, k, v, is_causal=w.is_causal, key_lens=kl)
+    out, lse = ea.attention(q, k, v, is_causal=w.is_causal, key_lens=kl, split_kv=0 if w.split_kv else None)
     ea.check_device_status()
     full = w.B * w.Hq * w.Nq * w.Nk * w.d <= 2e10
     kl_list = None if kl is None else kl.cpu().tolist()

@@ -19,6 +19,10 @@ used):
                                                (xxmr.cn/news/81028, sections 2.1-2.2)
   prefill_gqa  B1  Hq32 Hkv2 N16384  d128, causal -- grouped-head LLM prefill
                                                (jsqmd.com/news/348824, causal=True)
+  decode_gqa   B8  Hq32 Hkv8 Nq1 Nk16384 d128 -- one decoding step over a 16K-key
+                                               cache, grouped heads (the decoding
+                                               phase of jsqmd.com/news/722897,
+                                               section 5.2); run with split-KV
 """
 from __future__ import annotations
 
@@ -40,6 +44,7 @@ class Workload:
     is_causal: bool = False
     key_lens: tuple | None = None  # (low, high) inclusive range of per-sample key lengths
     seed: int = 0
+    split_kv: bool = False  # run through the split-KV entry point (automatic range count)
 
     @property
     def scale(self) -> float:
@@ -71,6 +76,7 @@ WORKLOADS = {
         Workload("unet_self", 4, 8, 8, 4096, 4096, 64, seed=1003),
         Workload("unet_cross", 4, 8, 8, 4096, 77, 64, key_lens=(8, 77), seed=1013),
         Workload("prefill_gqa", 1, 32, 2, 16384, 16384, 128, is_causal=True, seed=1004),
+        Workload("decode_gqa", 8, 32, 8, 1, 16384, 128, seed=1005, split_kv=True),
     ]
 }
 
