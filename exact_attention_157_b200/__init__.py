@@ -34,10 +34,13 @@ ATTN_ERR_ALIGNMENT = 3
 ATTN_ERR_CUDA = 4
 ATTN_ERR_TIMEOUT = 5
 ATTN_ERR_DEVICE = 6
+ATTN_ERR_SCRATCH = 7
+NOALLOC_SCRATCH_BYTES = 16 << 20  # ATTN_NOALLOC_SCRATCH_BYTES
 
 # Every symbol include/attn.h declares.
-EXPORTED = ("attn_fwd", "attn_splitkv_plan", "attn_fwd_splitkv", "attn_check_device_status",
-            "attn_set_wait_timeout_ns", "attn_selftest_timeout", "attn_status_string", "attn_last_cuda_error", "attn_version")
+EXPORTED = ("attn_fwd", "attn_splitkv_plan", "attn_fwd_splitkv", "attn_fwd_splitkv_noalloc",
+            "attn_check_device_status", "attn_set_wait_timeout_ns", "attn_selftest_timeout",
+            "attn_status_string", "attn_last_cuda_error", "attn_version")
 
 _lock = threading.Lock()
 _lib = None
@@ -69,6 +72,8 @@ def lib() -> ctypes.CDLL:
             L.attn_fwd_splitkv.restype = i
             L.attn_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, vp, vp,
                                            i, vp, ctypes.c_size_t, vp]
+            L.attn_fwd_splitkv_noalloc.restype = i
+            L.attn_fwd_splitkv_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, vp, vp, i, vp]
             L.attn_check_device_status.restype = i
             L.attn_check_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
             L.attn_set_wait_timeout_ns.restype = i
@@ -129,6 +134,20 @@ def attn_fwd_splitkv(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, is_causal,
     return int(lib().attn_fwd_splitkv(q, k, v, out, lse, int(B), int(Hq), int(Hkv), int(Nq), int(Nk), int(d),
                                       float(scale), int(bool(is_causal)), key_lens, additive_mask, ms,
                                       int(n_splits), workspace, int(workspace_bytes), stream))
+
+
+def attn_fwd_splitkv_noalloc(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, is_causal,
+                             key_lens=None, additive_mask=None, mask_strides=None, n_splits=0,
+                             stream=None) -> int:
+    """The C split-KV entry point that uses the library's fixed scratch buffer
+    (raw device pointers as ints); returns the status code."""
+    ms = None
+    if mask_strides is not None:
+        arr = (ctypes.c_int64 * 3)(*[int(x) for x in mask_strides])
+        ms = ctypes.cast(arr, ctypes.c_void_p)
+    return int(lib().attn_fwd_splitkv_noalloc(q, k, v, out, lse, int(B), int(Hq), int(Hkv), int(Nq), int(Nk),
+                                              int(d), float(scale), int(bool(is_causal)), key_lens, additive_mask,
+                                              ms, int(n_splits), stream))
 
 
 def attn_check_device_status(stream=None):

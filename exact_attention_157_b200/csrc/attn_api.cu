@@ -364,6 +364,8 @@ const char* attn_status_string(int status) {
         case ATTN_ERR_CUDA: return "CUDA runtime or driver error (see attn_last_cuda_error)";
         case ATTN_ERR_TIMEOUT: return "a bounded wait inside a kernel expired";
         case ATTN_ERR_DEVICE: return "device-side consistency check failed";
+        case ATTN_ERR_SCRATCH: return "the split plan needs more than the library's fixed scratch buffer "
+                                      "(ATTN_NOALLOC_SCRATCH_BYTES); use attn_fwd_splitkv or fewer ranges";
         default: return "unknown status";
     }
 }
@@ -373,3 +375,57 @@ int attn_last_cuda_error(void) { return g_last_cuda_error.load(); }
 int attn_version(void) { return kVersion; }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------
+// Split-KV without caller memory: the workspace lives in a fixed device array
+// of this library (allocated with the module, never by a call).  Serves
+// callers that cannot provide device memory per call: C hosts that own no
+// device allocator, servers whose memory is fully reserved up front, and
+// decode loops that must not call cudaMalloc / cudaFree (which may
+// synchronise the device).  Calls overlapping on one device share the array
+// and race.
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[ATTN_NOALLOC_SCRATCH_BYTES];
+
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch for the current device, looked up once
+// per device (with that device current).
+attn_status_t noalloc_scratch(int dev, void** out) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void* ptr = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e);
+        if (ptr == nullptr || reinterpret_cast<uintptr_t>(ptr) % kWsAlign != 0) return ATTN_ERR_CUDA;
+        g_noalloc_ptr[dev] = ptr;
+    }
+    *out = g_noalloc_ptr[dev];
+    return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" attn_status_t attn_fwd_splitkv_noalloc(const void* q, const void* k, const void* v, void* out,
+                                                  float* lse, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                                                  float scale, int is_causal, const int32_t* key_lens,
+                                                  const float* additive_mask, const int64_t* mask_strides,
+                                                  int n_splits, void* stream) {
+    if (B <= 0 || Hq <= 0 || Nq <= 0 || Nk <= 0 || n_splits < 0) return ATTN_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+    int dev = 0;
+    attn_status_t st = device_setup(&dev);
+    if (st != ATTN_OK) return st;
+    int used = 1;
+    size_t need = 0;
+    if ((st = attn_splitkv_plan(B, Hq, Nq, Nk, d, n_splits, g_dev[dev].sm_count > 0 ? g_dev[dev].sm_count : 1,
+                                &used, &need)) != ATTN_OK)
+        return st;
+    if (need > static_cast<size_t>(ATTN_NOALLOC_SCRATCH_BYTES)) return ATTN_ERR_SCRATCH;
+    void* scratch = nullptr;
+    if ((st = noalloc_scratch(dev, &scratch)) != ATTN_OK) return st;
+    // the plan above is the one fwd_impl makes for the same sizes and n_splits
+    return fwd_impl(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, is_causal, key_lens, additive_mask,
+                    mask_strides, true, n_splits, scratch, static_cast<size_t>(ATTN_NOALLOC_SCRATCH_BYTES), stream);
+}

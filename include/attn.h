@@ -41,7 +41,9 @@ typedef enum attn_status_t {
     ATTN_ERR_ALIGNMENT = 3,    /* a tensor base is not 16-byte aligned */
     ATTN_ERR_CUDA = 4,         /* a CUDA runtime / driver call failed; see attn_last_cuda_error() */
     ATTN_ERR_TIMEOUT = 5,      /* a bounded wait inside a kernel expired (asynchronous) */
-    ATTN_ERR_DEVICE = 6        /* another device-side consistency check failed (asynchronous) */
+    ATTN_ERR_DEVICE = 6,       /* another device-side consistency check failed (asynchronous) */
+    ATTN_ERR_SCRATCH = 7       /* attn_fwd_splitkv_noalloc: the call needs more than
+                                  ATTN_NOALLOC_SCRATCH_BYTES of scratch */
 } attn_status_t;
 
 /*
@@ -133,6 +135,42 @@ attn_status_t attn_fwd_splitkv(const void *q, const void *k, const void *v, void
                                const float *additive_mask, const int64_t *mask_strides,
                                int n_splits, void *workspace, size_t workspace_bytes,
                                void *stream);
+
+/*
+ * attn_fwd_splitkv_noalloc -- attn_fwd_splitkv with the workspace taken from a
+ * fixed buffer inside the library instead of from the caller.  The pages have
+ * no counterpart: it exists for callers that cannot hand over device memory
+ * per call -- plain C hosts that only receive tensor pointers from another
+ * framework and own no device allocator; servers that have reserved all of
+ * the GPU's memory up front (for example for a key/value cache) so that a
+ * new allocation would fail; and decode loops that must not call
+ * cudaMalloc / cudaFree, which may synchronise the whole device and so stall
+ * the other streams.
+ *
+ * The buffer is a statically sized device array of
+ * ATTN_NOALLOC_SCRATCH_BYTES (16 MiB) per device, part of the library's
+ * device image; nothing is allocated by this call or by the library.  A call
+ * whose split plan (attn_splitkv_plan with the same sizes and n_splits) needs
+ * more than that returns ATTN_ERR_SCRATCH before launching anything; a plan
+ * of one range needs none.  Nothing in the buffer has to start at zero: the
+ * attention kernel writes every partial result before the merge reads it.
+ *
+ * The first call on a device does one-time set-up with that device current
+ * (kernel attributes and the buffer's device address); make it before any
+ * stream capture.  Calls that overlap in time on one device -- on different
+ * streams, or from different host threads -- share the buffer and race:
+ * order them on one stream or synchronise between them.
+ *
+ * Arguments and results as attn_fwd_splitkv without workspace and
+ * workspace_bytes.  Errors: as attn_fwd_splitkv, plus ATTN_ERR_SCRATCH.
+ */
+#define ATTN_NOALLOC_SCRATCH_BYTES (16u << 20)
+attn_status_t attn_fwd_splitkv_noalloc(const void *q, const void *k, const void *v, void *out, float *lse,
+                                       int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                                       float scale, int is_causal,
+                                       const int32_t *key_lens,
+                                       const float *additive_mask, const int64_t *mask_strides,
+                                       int n_splits, void *stream);
 
 /*
  * attn_check_device_status -- synchronise `stream`, then read and clear the

@@ -1,0 +1,100 @@
+"""attn_fwd_splitkv_noalloc: split-KV with the library's fixed scratch buffer,
+called through the C ABI with raw device pointers and compared with the
+caller-workspace entry point attn_fwd_splitkv (and the fp64 oracle) within the
+parity tolerances, on two calls in a row.  Collected last so that it also runs
+after every other GPU test; it must pass on its own in a fresh process too."""
+import pytest
+import torch
+
+import exact_attention_157_b200 as ea
+import oracle
+from workloads import make_qkv
+
+from test_parity_gpu import assert_close
+
+pytestmark = pytest.mark.gpu
+
+DEV = torch.device("cuda:0")
+
+
+def _inputs(B, Hq, Hkv, Nq, Nk, d, seed):
+    q, k, v = make_qkv(B, Hq, Hkv, Nq, Nk, d, seed=seed)
+    return q, k, v, q.to(DEV), k.to(DEV), v.to(DEV)
+
+
+def _noalloc(qd, kd, vd, B, Hq, Hkv, Nq, Nk, d, n_splits, key_lens=None, causal=False):
+    out = torch.empty_like(qd)
+    lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=DEV)
+    st = ea.attn_fwd_splitkv_noalloc(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                     B, Hq, Hkv, Nq, Nk, d, 0.0, causal,
+                                     key_lens=None if key_lens is None else key_lens.data_ptr(),
+                                     n_splits=n_splits, stream=ea._stream_handle(None))
+    assert st == ea.ATTN_OK, ea.status_string(st)
+    ea.check_device_status()
+    return out, lse
+
+
+def _with_workspace(qd, kd, vd, B, Hq, Hkv, Nq, Nk, d, n_splits, key_lens=None, causal=False):
+    st, _, nbytes = ea.attn_splitkv_plan(B, Hq, Nq, Nk, d, n_splits, 0)
+    assert st == ea.ATTN_OK
+    ws = torch.empty((max(nbytes, 1),), dtype=torch.uint8, device=DEV)
+    out = torch.empty_like(qd)
+    lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=DEV)
+    st = ea.attn_fwd_splitkv(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                             B, Hq, Hkv, Nq, Nk, d, 0.0, causal,
+                             key_lens=None if key_lens is None else key_lens.data_ptr(),
+                             n_splits=n_splits, workspace=ws.data_ptr(), workspace_bytes=nbytes,
+                             stream=ea._stream_handle(None))
+    assert st == ea.ATTN_OK, ea.status_string(st)
+    ea.check_device_status()
+    return out, lse
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Nq,Nk,d,n_splits", [
+    (4, 16, 4, 1, 5000, 128, 0),
+    (2, 8, 2, 3, 3000, 64, 6),
+    (1, 4, 4, 200, 1100, 128, 3),
+])
+def test_noalloc_matches_workspace_entry_point_twice(B, Hq, Hkv, Nq, Nk, d, n_splits):
+    q, k, v, qd, kd, vd = _inputs(B, Hq, Hkv, Nq, Nk, d, seed=B * 100 + Nq + Nk + d)
+    ref_o, ref_l = _with_workspace(qd, kd, vd, B, Hq, Hkv, Nq, Nk, d, n_splits)
+    ro, rl = oracle.attention(q, k, v)
+    for _ in range(2):  # two calls in a row reuse the same scratch
+        out, lse = _noalloc(qd, kd, vd, B, Hq, Hkv, Nq, Nk, d, n_splits)
+        assert (out.float() - ref_o.float()).abs().max().item() <= 1e-2
+        assert (lse - ref_l).abs().max().item() <= 1e-3
+        assert_close(out, lse, ro, rl)
+
+
+def test_noalloc_key_lens_twice_and_no_new_device_memory():
+    B, Hq, Hkv, Nq, Nk, d = 3, 8, 8, 2, 4000, 128
+    q, k, v, qd, kd, vd = _inputs(B, Hq, Hkv, Nq, Nk, d, seed=17)
+    lens = torch.tensor([4000, 0, 1500], dtype=torch.int32, device=DEV)
+    ref_o, ref_l = _with_workspace(qd, kd, vd, B, Hq, Hkv, Nq, Nk, d, 5, key_lens=lens)
+    _noalloc(qd, kd, vd, B, Hq, Hkv, Nq, Nk, d, 5, key_lens=lens)  # set-up done by now
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info(DEV)[0]
+    for _ in range(2):
+        out, lse = _noalloc(qd, kd, vd, B, Hq, Hkv, Nq, Nk, d, 5, key_lens=lens)
+        assert (out.float() - ref_o.float()).abs().max().item() <= 1e-2
+        fin = torch.isfinite(ref_l)
+        assert torch.equal(torch.isneginf(lse), torch.isneginf(ref_l))
+        assert (lse[fin] - ref_l[fin]).abs().max().item() <= 1e-3
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info(DEV)[0] == free0
+
+
+def test_noalloc_rejects_plans_beyond_the_fixed_buffer():
+    # 4096 rows x 8 ranges x (128 + 1) fp32 values = 16.9 MB > 16 MiB; real buffers
+    B, Hq, Hkv, Nq, Nk, d = 1, 8, 8, 512, 8192, 128
+    st, used, nbytes = ea.attn_splitkv_plan(B, Hq, Nq, Nk, d, 8, 0)
+    assert st == ea.ATTN_OK and used == 8 and nbytes > ea.NOALLOC_SCRATCH_BYTES
+    _, _, _, qd, kd, vd = _inputs(B, Hq, Hkv, Nq, Nk, d, seed=23)
+    out = torch.zeros_like(qd)
+    st = ea.attn_fwd_splitkv_noalloc(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), out.data_ptr(), None,
+                                     B, Hq, Hkv, Nq, Nk, d, 0.0, False, n_splits=8,
+                                     stream=ea._stream_handle(None))
+    assert st == ea.ATTN_ERR_SCRATCH
+    assert "scratch" in ea.status_string(st)
+    torch.cuda.synchronize()
+    assert int(out.abs().sum().item()) == 0  # nothing was launched
