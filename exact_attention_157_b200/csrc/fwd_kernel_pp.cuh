@@ -54,15 +54,6 @@ constexpr int kRegsSoftmax = 200;
 constexpr int kRegsControl = 104;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl <= kPPThreads * 168, "register split");
 
-// P_t(j) is stored and signalled in kPChunks equal chunks of keys, so that the
-// PV over the first chunks runs while the softmax computes the last ones.
-#ifndef ATTN_P_CHUNKS
-#define ATTN_P_CHUNKS 2
-#endif
-constexpr int kPChunks = ATTN_P_CHUNKS;
-static_assert(kPChunks == 2 || kPChunks == 4, "P is released in 2 or 4 chunks");
-constexpr int kChunkKeys = kBN / kPChunks;
-
 template <int D, int NSLOT, int QS>
 struct SmemPP {
     static constexpr int kChunks = D / 64;
@@ -78,10 +69,11 @@ struct SmemPP {
     static constexpr int FULL = 2 * QS;               // NSLOT: K/V slot loaded
     static constexpr int EMPTY = 2 * QS + NSLOT;      // NSLOT: K/V slot released
     static constexpr int SFULL = 2 * QS + 2 * NSLOT;  // 2: S_t(j) complete
-    static constexpr int PCH = SFULL + 2;             // 2 x kPChunks: chunk c of P_t(j) stored (128 arrivals)
-    static constexpr int OFINAL = PCH + 2 * kPChunks; // 2: last PV_t of a unit complete
-    static constexpr int OEMPTY = OFINAL + 2;         // 2: O_t read out by the epilogue (128 arrivals)
-    static constexpr int MMAFIN = OEMPTY + 2;
+    static constexpr int P0 = SFULL + 2;              // 2: P_t(j) keys 0..63 stored (128 arrivals)
+    static constexpr int P1 = SFULL + 4;              // 2: P_t(j) keys 64..127 stored (128 arrivals)
+    static constexpr int OFINAL = SFULL + 6;          // 2: last PV_t of a unit complete
+    static constexpr int OEMPTY = SFULL + 8;          // 2: O_t read out by the epilogue (128 arrivals)
+    static constexpr int MMAFIN = SFULL + 10;
     static constexpr int kNumBars = MMAFIN + 1;
     static constexpr int kMisc = kBars + 8 * kNumBars;
     static constexpr int kBytes = kMisc + 16;
@@ -178,14 +170,22 @@ __device__ __forceinline__ int unit_key_len(const FwdParams& p, int s, int n_uni
 }
 
 // Units are numbered (head, split, query-unit): the units of one head and key
-// range are adjacent.  Without split-KV, n_splits = 1.
+// range are adjacent.  Without split-KV (SPLIT = false) there is one range.
+template <bool SPLIT>
 __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int s, int kv_len, bool report) {
     Unit x;
-    const int per_head = p.n_qtiles * p.n_splits;
-    x.bh = s / per_head;
-    const int r = s - x.bh * per_head;
-    x.split = r / p.n_qtiles;
-    const int pos = r - x.split * p.n_qtiles;
+    int pos;
+    if constexpr (SPLIT) {
+        const int per_head = p.n_qtiles * p.n_splits;
+        x.bh = s / per_head;
+        const int r = s - x.bh * per_head;
+        x.split = r / p.n_qtiles;
+        pos = r - x.split * p.n_qtiles;
+    } else {
+        x.bh = s / p.n_qtiles;
+        x.split = 0;
+        pos = s - x.bh * p.n_qtiles;
+    }
     // causal: heavy and light query tiles alternate (n-1, 0, n-2, 1, ...)
     const int qt = !p.is_causal ? pos : (pos & 1) ? (pos >> 1) : p.n_qtiles - 1 - (pos >> 1);
     x.b = x.bh / p.Hq;
@@ -198,13 +198,13 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int s, int kv_le
         kv_len = kv_len < 0 ? 0 : p.Nk;
     }
     x.kv_len = kv_len;
-    const int k_lo = x.split * p.split_keys;  // a multiple of kBN
+    const int k_lo = SPLIT ? x.split * p.split_keys : 0;  // a multiple of kBN
     x.j_lo = k_lo / kBN;
     #pragma unroll
     for (int t = 0; t < 2; ++t) {
         int end = x.kv_len;
         if (p.is_causal && x.q0 + (t + 1) * kBM < end) end = x.q0 + (t + 1) * kBM;
-        if (k_lo + p.split_keys < end) end = k_lo + p.split_keys;
+        if (SPLIT && k_lo + p.split_keys < end) end = k_lo + p.split_keys;
         x.n_t[t] = end > k_lo ? (end - k_lo + kBN - 1) / kBN : 0;
     }
     if (!x.tile_b_valid) x.n_t[1] = 0;
@@ -242,7 +242,8 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         }
         for (int t = 0; t < 2; ++t) {
             mbar_init(bar(L::SFULL + t), 1);
-            for (int c = 0; c < kPChunks; ++c) mbar_init(bar(L::PCH + t * kPChunks + c), 128);
+            mbar_init(bar(L::P0 + t), 128);
+            mbar_init(bar(L::P1 + t), 128);
             mbar_init(bar(L::OFINAL + t), 1);
             mbar_init(bar(L::OEMPTY + t), 128);
         }
@@ -287,7 +288,7 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             int it = 0;
             int kv_next = unit_key_len(p, unit_seq(cta, 0, G, p.unit_run), n_units);
             for (int u = unit_seq(cta, 0, G, p.unit_run); ok && u < n_units; ++it, u = unit_seq(cta, it, G, p.unit_run)) {
-                const Unit x = decode_unit(p, u, kv_next, false);
+                const Unit x = decode_unit<SPLIT>(p, u, kv_next, false);
                 kv_next = unit_key_len(p, unit_seq(cta, it + 1, G, p.unit_run), n_units);
                 const int qb = it % QS;
                 const int n_max = x.n_max();
@@ -337,12 +338,12 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             #pragma unroll
             for (int q = 0; q < QS; ++q) q_loads[q] = 0;
             int i_glob = 0;      // K/V loads consumed so far
-            int gp[2] = {0, 0};  // P_t blocks consumed so far (P chunk barrier phase)
+            int gp[2] = {0, 0};  // P_t blocks consumed so far (P0 / P1 phase)
             bool ok = true;
             int it = 0;
             int kv_next = unit_key_len(p, unit_seq(cta, 0, G, p.unit_run), n_units);
             for (int u = unit_seq(cta, 0, G, p.unit_run); ok && u < n_units; ++it, u = unit_seq(cta, it, G, p.unit_run)) {
-                const Unit x = decode_unit(p, u, kv_next, false);
+                const Unit x = decode_unit<SPLIT>(p, u, kv_next, false);
                 kv_next = unit_key_len(p, unit_seq(cta, it + 1, G, p.unit_run), n_units);
                 const int n_max = x.n_max();
                 if (n_max == 0) continue;
@@ -364,14 +365,14 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     }
                     mma_commit(bar(L::SFULL + t));
                 };
-                // O_t += P_t(j)[:, keys of chunk c] V_j[those keys, :]
-                auto issue_pv = [&](int t, int j, int c) {
+                // O_t += P_t(j)[:, keys 64 half .. +63] V_j[those keys, :]
+                auto issue_pv = [&](int t, int j, int half) {
                     const uint32_t v_addr = sbase + L::kRing + slot_of(2 * j + 1) * L::kTileBytes;
                     const uint32_t o_tmem = tmem + L::kColO + t * D;
                     const uint32_t p_tmem = tmem + t * 128;
                     #pragma unroll
-                    for (int k4 = 0; k4 < kChunkKeys / 16; ++k4) {
-                        const int kk = c * (kChunkKeys / 16) + k4;
+                    for (int k4 = 0; k4 < kBN / 32; ++k4) {
+                        const int kk = half * (kBN / 32) + k4;
                         mma_ts(o_tmem, p_tmem + kk * 8, smem_desc_sw128(v_addr + kk * 2048, L::kChunkBytes, 1024),
                                kIdescO, (j > 0 || kk > 0) ? 1u : 0u);
                     }
@@ -388,26 +389,24 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     bool v_ready = false, k_next_ready = false;
                     for (int t = 0; t < 2 && ok; ++t) {
                         if (j >= x.n_t[t]) continue;
-                        // P_t(j) arrives in chunks: the PV over the first ones overlaps the rest of
-                        // the softmax
-                        for (int c = 0; ok && c < kPChunks; ++c) {
-                            if (!mbar_wait(bar(L::PCH + t * kPChunks + c), gp[t] & 1, limit, abort_flag, p.epoch,
-                                           kRoleMma, 22)) { ok = false; break; }
-                            if (c == 0) {
-                                // the previous unit's epilogue must have read O_t out of TMEM
-                                if (j == 0 && it > 0 &&
-                                    !mbar_wait(bar(L::OEMPTY + t), (it - 1) & 1, limit, abort_flag, p.epoch, kRoleMma,
-                                               23)) { ok = false; break; }
-                                if (!v_ready) {
-                                    if (!wait_full(2 * j + 1, 24)) { ok = false; break; }
-                                    v_ready = true;
-                                }
-                            }
-                            tc_fence_after();
-                            issue_pv(t, j, c);
+                        // first half of P_t(j): PV over keys 0..63 overlaps the rest of the softmax
+                        if (!mbar_wait(bar(L::P0 + t), gp[t] & 1, limit, abort_flag, p.epoch, kRoleMma, 22))
+                            { ok = false; break; }
+                        // the previous unit's epilogue must have read O_t out of TMEM
+                        if (j == 0 && it > 0 &&
+                            !mbar_wait(bar(L::OEMPTY + t), (it - 1) & 1, limit, abort_flag, p.epoch, kRoleMma, 23))
+                            { ok = false; break; }
+                        if (!v_ready) {
+                            if (!wait_full(2 * j + 1, 24)) { ok = false; break; }
+                            v_ready = true;
                         }
-                        if (!ok) break;
+                        tc_fence_after();
+                        issue_pv(t, j, 0);
+                        if (!mbar_wait(bar(L::P1 + t), gp[t] & 1, limit, abort_flag, p.epoch, kRoleMma, 27))
+                            { ok = false; break; }
                         ++gp[t];
+                        tc_fence_after();
+                        issue_pv(t, j, 1);
                         if (j + 1 < x.n_t[t]) {
                             if (!k_next_ready) {
                                 if (!wait_full(2 * j + 2, 25)) { ok = false; break; }
@@ -447,7 +446,7 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         int it = 0;
         int kv_next = unit_key_len(p, unit_seq(cta, 0, G, p.unit_run), n_units);
         for (int u = unit_seq(cta, 0, G, p.unit_run); u < n_units; ++it, u = unit_seq(cta, it, G, p.unit_run)) {
-            const Unit x = decode_unit(p, u, kv_next, threadIdx.x == 0);
+            const Unit x = decode_unit<SPLIT>(p, u, kv_next, threadIdx.x == 0);
             kv_next = unit_key_len(p, unit_seq(cta, it + 1, G, p.unit_run), n_units);
             const int q0_t = x.q0 + t * kBM;
             const int q_idx = q0_t + row;
@@ -517,8 +516,8 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 // warp-collective, but rows that keep their max use alpha = 1 exactly, so a
                 // row's result never depends on the other rows of its warp.  O_t holds
                 // sum_{i<j} P_i V_i here (S_t(j) was issued after PV_t(j-1)); the rescale
-                // of O_t itself is done after the first chunk of P_t is stored (fewer live
-                // registers) and before that chunk's signal lets PV_t(j) start.
+                // of O_t itself is done after the first half of P_t is stored (fewer live
+                // registers) and before the P0 arrive that lets PV_t(j) start.
                 const bool need = mx > m_used + kLazyTau;
                 const bool warp_rescale = __any_sync(0xffffffffu, need) && j > 0;
                 float alpha = 1.0f;
@@ -534,26 +533,26 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 // just before it: (1) exponent arguments, (2) exponentials, (3) row sum and
                 // bf16 packing.
                 uint64_t acc0 = 0, acc1 = 0, acc2 = 0, acc3 = 0;  // packed partial sums
-                uint32_t pk[kChunkKeys / 2];
-                // Chunk by chunk of keys: each chunk is stored and signalled on its own, so
-                // the PV over earlier chunks runs during the later ones.  O_t is rescaled
-                // (if needed) before the first chunk's signal releases the first PV.
-                auto exp_chunk = [&](auto emulate, auto chunk_c) {
-                    constexpr int cc = decltype(chunk_c)::value;
-                    float* sh = s + cc * kChunkKeys;
+                uint32_t pk[kBN / 4];
+                // Keys 0..63, then 64..127: each half is stored and signalled on its own
+                // (P0, P1), so PV over the first half runs during the second half.  O_t is
+                // rescaled (if needed) before P0 releases the first PV.
+                auto exp_half = [&](auto emulate, auto half_c) {
+                    constexpr int h = decltype(half_c)::value;
+                    float* sh = s + h * (kBN / 2);
                     if constexpr (HAS_MASK) {
                         #pragma unroll
-                        for (int c = 0; c < kChunkKeys; ++c) sh[c] = sh[c] - shift;
+                        for (int c = 0; c < kBN / 2; ++c) sh[c] = sh[c] - shift;
                     } else {
                         #pragma unroll
-                        for (int c = 0; c < kChunkKeys / 2; ++c) {
+                        for (int c = 0; c < kBN / 4; ++c) {
                             const uint64_t xv = ffma2(pack_f32x2(sh[2 * c], sh[2 * c + 1]), c2, nshift2);
                             sh[2 * c] = lo_f32(xv);
                             sh[2 * c + 1] = hi_f32(xv);
                         }
                     }
                     #pragma unroll
-                    for (int c = 0; c < kChunkKeys / 2; ++c) {
+                    for (int c = 0; c < kBN / 4; ++c) {
                         if (decltype(emulate)::value &&
                             (c % (kExp2EmuEvery > 0 ? kExp2EmuEvery : 1)) == kExp2EmuEvery - 1) {
                             exp2_poly_pair(pack_f32x2(sh[2 * c], sh[2 * c + 1]), sh[2 * c], sh[2 * c + 1]);
@@ -563,7 +562,7 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         }
                     }
                     #pragma unroll
-                    for (int c = 0; c < kChunkKeys / 2; ++c) {
+                    for (int c = 0; c < kBN / 4; ++c) {
                         const uint64_t e = pack_f32x2(sh[2 * c], sh[2 * c + 1]);
                         switch (c & 3) {
                             case 0: acc0 = fadd2(acc0, e); break;
@@ -573,12 +572,8 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         }
                         pk[c] = pack_bf16x2(sh[2 * c], sh[2 * c + 1]);
                     }
-                    if constexpr (kChunkKeys == 64) {
-                        tmem_st32(s_tmem + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-                    } else {
-                        tmem_st16(s_tmem + cc * (kChunkKeys / 2), pk);
-                    }
-                    if (cc == 0 && warp_rescale) {
+                    tmem_st32(s_tmem + h * 32, pk);
+                    if (h == 0 && warp_rescale) {
                         #pragma unroll
                         for (int c = 0; c < D / 32; ++c) {
                             uint32_t o[32];
@@ -591,20 +586,17 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     }
                     tmem_wait_st();
                     tc_fence_before();
-                    mbar_arrive(bar(L::PCH + t * kPChunks + cc));
+                    mbar_arrive(bar((h == 0 ? L::P0 : L::P1) + t));
                 };
-                auto all_chunks = [&](auto emulate) {
-                    exp_chunk(emulate, std::integral_constant<int, 0>{});
-                    exp_chunk(emulate, std::integral_constant<int, 1>{});
-                    if constexpr (kPChunks == 4) {
-                        exp_chunk(emulate, std::integral_constant<int, 2>{});
-                        exp_chunk(emulate, std::integral_constant<int, 3>{});
-                    }
-                };
-                if (kExp2EmuEvery > 0 && !HAS_MASK && !boundary)
-                    all_chunks(std::integral_constant<bool, kExp2EmuEvery != 0>{});
-                else
-                    all_chunks(std::false_type{});
+                using Half0 = std::integral_constant<int, 0>;
+                using Half1 = std::integral_constant<int, 1>;
+                if (kExp2EmuEvery > 0 && !HAS_MASK && !boundary) {
+                    exp_half(std::integral_constant<bool, kExp2EmuEvery != 0>{}, Half0{});
+                    exp_half(std::integral_constant<bool, kExp2EmuEvery != 0>{}, Half1{});
+                } else {
+                    exp_half(std::false_type{}, Half0{});
+                    exp_half(std::false_type{}, Half1{});
+                }
                 const uint64_t acc = fadd2(fadd2(acc0, acc2), fadd2(acc1, acc3));
                 l_sum += lo_f32(acc) + hi_f32(acc);
             }
