@@ -18,7 +18,7 @@
 //   warp 8      TMA producer: Q_A, Q_B of each unit into one of QS Q buffers,
 //               K_0, V_0, K_1, V_1, ... of every unit into one ring of NSLOT
 //               slots (128-byte swizzle, no multicast), in consumption order
-//   warp 9      TMEM owner and MMA issuer (one thread), per unit
+//   warp 9      TMEM owner and MMA issuer (warp-uniform, one elected lane issues), per unit
 //                 S_A(0) S_B(0) | PV_A(0) S_A(1) PV_B(0) S_B(1) | PV_A(1) ...
 //               so that while the softmax of one tile runs, the tensor cores
 //               work on the other tile (two MMAs of cover each way)
@@ -331,7 +331,9 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         }
       } else {
         // =============================== MMA issuer ===============================
-        if (lane == 0) {
+        // The whole warp runs this loop (warp-uniform control flow and operands);
+        // one elected lane issues each tcgen05 instruction.
+        {
             constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kBN, false);
             constexpr uint32_t kIdescO = idesc_bf16_f32(kBM, D, true);
             int q_loads[QS];
@@ -351,7 +353,7 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 const uint32_t qbuf = sbase + L::kQ + qb * L::kQBuf;
                 auto slot_of = [&](int i) { return (i_glob + i) % NSLOT; };
                 auto wait_full = [&](int i, unsigned site) -> bool {
-                    return mbar_wait(bar(L::FULL + slot_of(i)), ((i_glob + i) / NSLOT) & 1, limit, abort_flag,
+                    return mbar_wait_warp(bar(L::FULL + slot_of(i)), ((i_glob + i) / NSLOT) & 1, limit, abort_flag,
                                      p.epoch, kRoleMma, site);
                 };
                 auto issue_s = [&](int t, int j) {
@@ -360,10 +362,10 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint32_t off = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
-                        mma_ss(tmem + t * 128, smem_desc_sw128(q_addr + off, 16, 1024),
+                        mma_ss_warp(tmem + t * 128, smem_desc_sw128(q_addr + off, 16, 1024),
                                smem_desc_sw128(k_addr + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
                     }
-                    mma_commit(bar(L::SFULL + t));
+                    mma_commit_warp(bar(L::SFULL + t));
                 };
                 // O_t += P_t(j)[:, keys 64 half .. +63] V_j[those keys, :]
                 auto issue_pv = [&](int t, int j, int half) {
@@ -373,28 +375,28 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     #pragma unroll
                     for (int k4 = 0; k4 < kBN / 32; ++k4) {
                         const int kk = half * (kBN / 32) + k4;
-                        mma_ts(o_tmem, p_tmem + kk * 8, smem_desc_sw128(v_addr + kk * 2048, L::kChunkBytes, 1024),
+                        mma_ts_warp(o_tmem, p_tmem + kk * 8, smem_desc_sw128(v_addr + kk * 2048, L::kChunkBytes, 1024),
                                kIdescO, (j > 0 || kk > 0) ? 1u : 0u);
                     }
                 };
-                ok = mbar_wait(bar(L::QFULL + qb), q_loads[qb] & 1, limit, abort_flag, p.epoch, kRoleMma, 20) &&
+                ok = mbar_wait_warp(bar(L::QFULL + qb), q_loads[qb] & 1, limit, abort_flag, p.epoch, kRoleMma, 20) &&
                      wait_full(0, 21);
                 ++q_loads[qb];
                 if (!ok) break;
                 tc_fence_after();
                 for (int t = 0; t < 2; ++t)
                     if (x.n_t[t] > 0) issue_s(t, 0);
-                mma_commit(bar(L::EMPTY + slot_of(0)));  // K_0 released once both S(0) complete
+                mma_commit_warp(bar(L::EMPTY + slot_of(0)));  // K_0 released once both S(0) complete
                 for (int j = 0; ok && j < n_max; ++j) {
                     bool v_ready = false, k_next_ready = false;
                     for (int t = 0; t < 2 && ok; ++t) {
                         if (j >= x.n_t[t]) continue;
                         // first half of P_t(j): PV over keys 0..63 overlaps the rest of the softmax
-                        if (!mbar_wait(bar(L::P0 + t), gp[t] & 1, limit, abort_flag, p.epoch, kRoleMma, 22))
+                        if (!mbar_wait_warp(bar(L::P0 + t), gp[t] & 1, limit, abort_flag, p.epoch, kRoleMma, 22))
                             { ok = false; break; }
                         // the previous unit's epilogue must have read O_t out of TMEM
                         if (j == 0 && it > 0 &&
-                            !mbar_wait(bar(L::OEMPTY + t), (it - 1) & 1, limit, abort_flag, p.epoch, kRoleMma, 23))
+                            !mbar_wait_warp(bar(L::OEMPTY + t), (it - 1) & 1, limit, abort_flag, p.epoch, kRoleMma, 23))
                             { ok = false; break; }
                         if (!v_ready) {
                             if (!wait_full(2 * j + 1, 24)) { ok = false; break; }
@@ -402,7 +404,7 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         }
                         tc_fence_after();
                         issue_pv(t, j, 0);
-                        if (!mbar_wait(bar(L::P1 + t), gp[t] & 1, limit, abort_flag, p.epoch, kRoleMma, 27))
+                        if (!mbar_wait_warp(bar(L::P1 + t), gp[t] & 1, limit, abort_flag, p.epoch, kRoleMma, 27))
                             { ok = false; break; }
                         ++gp[t];
                         tc_fence_after();
@@ -415,18 +417,18 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                             }
                             issue_s(t, j + 1);
                         } else {
-                            mma_commit(bar(L::OFINAL + t));
+                            mma_commit_warp(bar(L::OFINAL + t));
                         }
                     }
                     if (!ok) break;
-                    mma_commit(bar(L::EMPTY + slot_of(2 * j + 1)));  // V_j: both PV(j) issued above
+                    mma_commit_warp(bar(L::EMPTY + slot_of(2 * j + 1)));  // V_j: both PV(j) issued above
                     // K_{j+1}: the tile with n_t = n_max uses every block, so k_next_ready
                     // holds exactly when j + 1 < n_max (each load is released once).
-                    if (k_next_ready) mma_commit(bar(L::EMPTY + slot_of(2 * j + 2)));
+                    if (k_next_ready) mma_commit_warp(bar(L::EMPTY + slot_of(2 * j + 2)));
                 }
                 i_glob += 2 * n_max;
             }
-            mma_commit(bar(L::MMAFIN));
+            mma_commit_warp(bar(L::MMAFIN));
             mbar_drain(bar(L::MMAFIN), 0, kRoleMma, 26);
         }
       }
