@@ -7,7 +7,8 @@ with the CUDA library and never imports it.
 Contents
 --------
 ``attention``            the definition (three steps, two-pass softmax) in plain C,
-                         fp64, threaded over rows (``attn_oracle.c``).
+                         fp64, threaded over rows (``attn_oracle.c``); optional
+                         soft-capped scores and 2-D neighbourhood / window masks.
 ``attention_online``     a numpy fp64 re-statement of the tiled algorithm with a
                          running max ``m`` and running sum ``l`` rescaled per key
                          block, used only to cross-check ``attention``.
@@ -64,6 +65,14 @@ def _bind(path):
         ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
         ctypes.c_double, ctypes.c_int,
         ip, dp, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+        ip, ctypes.c_int, ctypes.c_int]
+    lib.oracle_attention_fwd_mod.restype = ctypes.c_int
+    lib.oracle_attention_fwd_mod.argtypes = [
+        dp, dp, dp, dp, dp,
+        ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+        ctypes.c_double, ctypes.c_int,
+        ip, dp, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+        ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
         ip, ctypes.c_int, ctypes.c_int]
     lib.oracle_default_threads.restype = ctypes.c_int
     return lib
@@ -123,13 +132,21 @@ def _mask_view(mask, B, Hq, Nq, Nk):
     return base, Hq * Nq * Nk, Nq * Nk, Nk
 
 
+MASK2D_KINDS = {"neighborhood": 1, "window": 2}
+
+
 def attention(q, k, v, *, scale: float | None = None, is_causal: bool = False,
-              key_lens=None, mask=None, rows=None, n_threads: int = 0, lib=None):
+              key_lens=None, mask=None, rows=None, n_threads: int = 0, lib=None,
+              softcap: float = 0.0, mask2d=None):
     """The definition, in fp64.
 
     q: [B, Hq, Nq, d]; k, v: [B, Hkv, Nk, d]; key_lens: [B] ints or None;
     mask: additive mask broadcastable to [B, Hq, Nq, Nk] or None;
-    rows: optional list of query indices computed in every head (others are NaN).
+    rows: optional list of query indices computed in every head (others are NaN);
+    softcap: > 0 replaces the scaled score x by softcap * tanh(x / softcap);
+    mask2d: None, ("neighborhood", W, R) or ("window", W, w, shift) -- token n
+    of a row-major grid with W tokens per row sits at (n // W, n % W); see
+    ``attn_oracle.c`` for the two rules.
     Returns (O [B, Hq, Nq, d] fp64, LSE [B, Hq, Nq] fp64).
     """
     q, k, v = _f64(q), _f64(k), _f64(v)
@@ -142,11 +159,24 @@ def attention(q, k, v, *, scale: float | None = None, is_causal: bool = False,
     kl = None if key_lens is None else np.ascontiguousarray(np.asarray(key_lens, dtype=np.int32))
     rw = None if rows is None else np.ascontiguousarray(np.asarray(rows, dtype=np.int32))
     mk, sb, sh, sq = (None, 0, 0, 0) if mask is None else _mask_view(_f64(mask), B, Hq, Nq, Nk)
-    rc = (lib or _load()).oracle_attention_fwd(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
-        B, Hq, Hkv, Nq, Nk, d, float(scale), int(bool(is_causal)),
-        _ptr(kl, ctypes.c_int32), _ptr(mk), sb, sh, sq,
-        _ptr(rw, ctypes.c_int32), 0 if rw is None else len(rw), int(n_threads))
+    if softcap == 0.0 and mask2d is None:
+        rc = (lib or _load()).oracle_attention_fwd(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+            B, Hq, Hkv, Nq, Nk, d, float(scale), int(bool(is_causal)),
+            _ptr(kl, ctypes.c_int32), _ptr(mk), sb, sh, sq,
+            _ptr(rw, ctypes.c_int32), 0 if rw is None else len(rw), int(n_threads))
+    else:
+        kind, W, size, shift = 0, 0, 0, 0
+        if mask2d is not None:
+            kind = MASK2D_KINDS[mask2d[0]]
+            W, size = int(mask2d[1]), int(mask2d[2])
+            shift = int(mask2d[3]) if len(mask2d) > 3 else 0
+        rc = (lib or _load()).oracle_attention_fwd_mod(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+            B, Hq, Hkv, Nq, Nk, d, float(scale), int(bool(is_causal)),
+            _ptr(kl, ctypes.c_int32), _ptr(mk), sb, sh, sq,
+            float(softcap), kind, W, size, shift,
+            _ptr(rw, ctypes.c_int32), 0 if rw is None else len(rw), int(n_threads))
     if rc != 0:
         raise ValueError(f"oracle_attention_fwd rejected its arguments (status {rc})")
     return out, lse

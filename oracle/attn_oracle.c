@@ -27,6 +27,23 @@
  *     LSE_i = M_i + ln L_i;
  *   - a row with no unmasked key returns O = 0 and LSE = -infinity.
  *
+ * Score and mask variants (oracle_attention_fwd_mod):
+ *   - soft-capping, the score_mod example of the PyTorch attention article
+ *     (atyun.com/61003.html, "Score Mod example: soft-capping with tanh"):
+ *     the scaled dot product x = scale * <q_i, k_j> becomes cap * tanh(x / cap);
+ *     an additive mask, if any, is added after it (a score_mod acts on the
+ *     score, masking comes after);
+ *   - 2-D neighbourhood, the mask_mod example of the same article: token n of
+ *     a row-major grid with W tokens per row sits at (n / W, n % W); query i
+ *     sees key j iff |r_i - r_j| < R and |c_i - c_j| < R;
+ *   - 2-D windows, the window attention of "Flash Attention in a production
+ *     Stable-Diffusion service" (xxmr.cn/news/81028) section 3.2: the grid is
+ *     cut into non-overlapping w x w windows, displaced by `shift` tokens in
+ *     both directions (0 = plain, w / 2 = the shifted variant; border windows
+ *     are partial, no cyclic wrap), and query i sees key j iff both lie in the
+ *     same window: (r_i + shift) / w == (r_j + shift) / w and the same for
+ *     the columns.
+ *
  * Every arithmetic step is fp64 on the bf16 input values (converted exactly
  * to double by the caller).  Rows are spread over POSIX threads; a row's own
  * arithmetic is the plain sequence below, never blocked or reordered.
@@ -46,6 +63,9 @@ typedef struct {
     const int32_t *key_lens;
     const double *mask;
     int64_t mask_sb, mask_sh, mask_sq; /* element strides of the mask */
+    double softcap;                    /* 0: off */
+    int m2_kind;                       /* 0 none, 1 neighbourhood, 2 windows */
+    int m2_w, m2_size, m2_shift;       /* grid width, R or w, window shift */
     const int32_t *rows;               /* optional subset of query rows */
     int n_rows;
     int64_t n_units;                   /* B * Hq * (rows per head) */
@@ -57,6 +77,24 @@ typedef struct {
     int64_t first, last; /* [first, last) in unit index space */
     int status;
 } oracle_job;
+
+/* Whether the 2-D mask lets query i see key j. */
+static int allowed_2d(const oracle_args *a, int i, int j)
+{
+    if (a->m2_kind == 0) return 1;
+    const int W = a->m2_w;
+    const int ri = i / W, ci = i % W, rj = j / W, cj = j % W;
+    if (a->m2_kind == 1) {
+        const int dr = ri > rj ? ri - rj : rj - ri;
+        const int dc = ci > cj ? ci - cj : cj - ci;
+        return dr < a->m2_size && dc < a->m2_size;
+    }
+    if (a->m2_kind == 2) {
+        const int w = a->m2_size, sh = a->m2_shift;
+        return (ri + sh) / w == (rj + sh) / w && (ci + sh) / w == (cj + sh) / w;
+    }
+    return 1;
+}
 
 /* One query row of one head: the three steps of the definition. */
 static void oracle_row(const oracle_args *a, int b, int h, int i, double *s)
@@ -73,15 +111,17 @@ static void oracle_row(const oracle_args *a, int b, int h, int i, double *s)
         ? a->mask + (int64_t)b * a->mask_sb + (int64_t)h * a->mask_sh + (int64_t)i * a->mask_sq
         : NULL;
 
-    /* Step 1: scores s_ij = scale * <q_i, k_j> (+ mask_ij); masked keys -> -inf. */
+    /* Step 1: scores s_ij = scale * <q_i, k_j>, soft-capped if asked, (+ mask_ij);
+     * masked keys -> -inf. */
     for (int j = 0; j < a->Nk; ++j) {
-        if (j >= len || (a->is_causal && j > i)) {
+        if (j >= len || (a->is_causal && j > i) || !allowed_2d(a, i, j)) {
             s[j] = -INFINITY;
             continue;
         }
         double dot = 0.0;
         for (int t = 0; t < d; ++t) dot += qi[t] * kh[(int64_t)j * d + t];
         s[j] = a->scale * dot;
+        if (a->softcap > 0.0) s[j] = a->softcap * tanh(s[j] / a->softcap);
         if (mrow) s[j] += mrow[j];
     }
 
@@ -135,24 +175,31 @@ static void *oracle_worker(void *p)
 }
 
 /*
- * oracle_attention_fwd
+ * oracle_attention_fwd_mod
  *   q   [B, Hq, Nq, d], k/v [B, Hkv, Nk, d], out [B, Hq, Nq, d]: fp64, contiguous.
  *   lse [B, Hq, Nq] fp64 or NULL.
  *   key_lens [B] (0 <= len <= Nk) or NULL; mask fp64 with element strides
  *   (sb, sh, sq) and a contiguous last dimension, or NULL.
  *   rows: if non-NULL, only these query indices (in every head) are computed.
  *   n_threads <= 0 uses every online core.
+ *   softcap > 0 applies cap * tanh(x / cap) to the scaled score (0: off);
+ *   m2_kind 1 (neighbourhood, m2_size = R) or 2 (windows, m2_size = w,
+ *   m2_shift) on a grid of m2_w tokens per row; 0: no 2-D mask.
  * Returns 0 on success, -1 on invalid arguments, -2 on allocation failure.
  */
-int oracle_attention_fwd(const double *q, const double *k, const double *v,
-                         double *out, double *lse,
-                         int B, int Hq, int Hkv, int Nq, int Nk, int d,
-                         double scale, int is_causal,
-                         const int32_t *key_lens,
-                         const double *mask, int64_t mask_sb, int64_t mask_sh, int64_t mask_sq,
-                         const int32_t *rows, int n_rows, int n_threads)
+int oracle_attention_fwd_mod(const double *q, const double *k, const double *v,
+                             double *out, double *lse,
+                             int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                             double scale, int is_causal,
+                             const int32_t *key_lens,
+                             const double *mask, int64_t mask_sb, int64_t mask_sh, int64_t mask_sq,
+                             double softcap, int m2_kind, int m2_w, int m2_size, int m2_shift,
+                             const int32_t *rows, int n_rows, int n_threads)
 {
     if (!q || !k || !v || !out) return -1;
+    if (!(softcap >= 0.0)) return -1;
+    if (m2_kind < 0 || m2_kind > 2) return -1;
+    if (m2_kind != 0 && (m2_w <= 0 || m2_size <= 0 || m2_shift < 0)) return -1;
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nk <= 0 || d <= 0) return -1;
     if (Hq % Hkv != 0) return -1;
     if (rows) {
@@ -170,6 +217,7 @@ int oracle_attention_fwd(const double *q, const double *k, const double *v,
     a.scale = scale; a.is_causal = is_causal;
     a.key_lens = key_lens;
     a.mask = mask; a.mask_sb = mask_sb; a.mask_sh = mask_sh; a.mask_sq = mask_sq;
+    a.softcap = softcap; a.m2_kind = m2_kind; a.m2_w = m2_w; a.m2_size = m2_size; a.m2_shift = m2_shift;
     a.rows = rows; a.n_rows = n_rows;
     a.n_units = (int64_t)B * Hq * (rows ? n_rows : Nq);
 
@@ -208,6 +256,19 @@ int oracle_attention_fwd(const double *q, const double *k, const double *v,
     free(jobs);
     free(tids);
     return status;
+}
+
+/* The plain definition: no soft-cap, no 2-D mask. */
+int oracle_attention_fwd(const double *q, const double *k, const double *v,
+                         double *out, double *lse,
+                         int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                         double scale, int is_causal,
+                         const int32_t *key_lens,
+                         const double *mask, int64_t mask_sb, int64_t mask_sh, int64_t mask_sq,
+                         const int32_t *rows, int n_rows, int n_threads)
+{
+    return oracle_attention_fwd_mod(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, is_causal, key_lens,
+                                    mask, mask_sb, mask_sh, mask_sq, 0.0, 0, 0, 0, 0, rows, n_rows, n_threads);
 }
 
 /* Number of threads oracle_attention_fwd would use for n_threads <= 0. */

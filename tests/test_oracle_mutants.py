@@ -20,7 +20,7 @@ MUTANTS = {
     "lse_log2": ("M + log(L)", "M + log2(L)"),
     "v_transposed": ("oi[t] += s[j] * vj[t];", "oi[t] += s[j] * vh[(int64_t)t * a->Nk + j % a->Nk];"),
     "no_normalisation": ("oi[t] /= L;", "oi[t] /= 1.0;"),
-    "mask_before_scale": ("s[j] = a->scale * dot;\n        if (mrow) s[j] += mrow[j];",
+    "mask_before_scale": ("s[j] = a->scale * dot;\n        if (a->softcap > 0.0) s[j] = a->softcap * tanh(s[j] / a->softcap);\n        if (mrow) s[j] += mrow[j];",
                           "s[j] = dot;\n        if (mrow) s[j] += mrow[j];\n        s[j] *= a->scale;"),
 }
 
