@@ -109,42 +109,6 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
 __device__ __forceinline__ float lo_f32(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v)); }
 __device__ __forceinline__ float hi_f32(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
 
-// Part of the exponentials can run on the FMA pipe instead of the MUFU unit:
-// one pair in every kExp2EmuEvery (0 disables; measured neutral to negative
-// on B200 at d = 128, where the softmax is latency- rather than MUFU-bound).
-// Used only on blocks without a masked key, so masked probabilities stay
-// exactly 0 (ex2(-inf)).
-#ifndef ATTN_EXP2_EMU_EVERY
-#define ATTN_EXP2_EMU_EVERY 0
-#endif
-constexpr int kExp2EmuEvery = ATTN_EXP2_EMU_EVERY;
-
-constexpr uint64_t splat2(uint32_t bits) { return (static_cast<uint64_t>(bits) << 32) | bits; }
-
-// 2^x for a pair, x <= ~9: Cody-Waite reduction x = n + f, n = round(x) (the
-// 1.5 * 2^23 rounding constant leaves n in the low mantissa bits), then a
-// degree-3 minimax polynomial for 2^f on [-1/2, 1/2] (max relative error
-// 7.5e-5; coefficients fitted by csrc/fit_exp2_poly.py) and n added to the
-// exponent field.  x is clamped at -120, where the result (~1e-36) is zero for
-// every practical purpose next to the row maximum (>= 1).
-__device__ __forceinline__ void exp2_poly_pair(uint64_t x, float& e0, float& e1) {
-    constexpr uint64_t kMagic = splat2(0x4B400000u);     //  12582912.0f
-    constexpr uint64_t kNegMagic = splat2(0xCB400000u);  // -12582912.0f
-    constexpr uint64_t kNegOne = splat2(0xBF800000u);    // -1.0f
-    constexpr uint64_t kC0 = splat2(0x3F7FFB49u);        // 0.99992806
-    constexpr uint64_t kC1 = splat2(0x3F31798Du);        // 0.69326097
-    constexpr uint64_t kC2 = splat2(0x3E786F0Du);        // 0.24261113
-    constexpr uint64_t kC3 = splat2(0x3D61FBB0u);        // 0.05517167
-    const uint64_t xx = pack_f32x2(fmaxf(lo_f32(x), -120.0f), fmaxf(hi_f32(x), -120.0f));
-    const uint64_t t = fadd2(xx, kMagic);
-    const uint64_t f = ffma2(fadd2(t, kNegMagic), kNegOne, xx);  // x - n, in [-1/2, 1/2]
-    uint64_t p = ffma2(f, kC3, kC2);
-    p = ffma2(p, f, kC1);
-    p = ffma2(p, f, kC0);
-    e0 = __uint_as_float(static_cast<uint32_t>(p) + (static_cast<uint32_t>(t) << 23));
-    e1 = __uint_as_float(static_cast<uint32_t>(p >> 32) + (static_cast<uint32_t>(t >> 32) << 23));
-}
-
 // Everything about one work unit that every role derives identically.
 struct Unit {
     int bh, b, h, bhk, q0, kv_len;
@@ -477,28 +441,34 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 const int j0 = (x.j_lo + j) * kBN;
                 const bool boundary = (j0 + kBN > kv_len) || (p.is_causal && j0 + kBN - 1 > q0_t);
 
-                float mx;
-                if constexpr (HAS_MASK) {
-                    mx = -INFINITY;
-                    // keys c >= lim are masked (past the end of K, or past the diagonal)
-                    int lim = mask_row != nullptr ? kv_len - j0 : 0;
-                    if (p.is_causal && q_idx - j0 + 1 < lim) lim = q_idx - j0 + 1;
-                    #pragma unroll
-                    for (int c = 0; c < kBN; ++c) {
-                        const bool valid = c < lim;
-                        const float mv = valid ? __ldg(mask_row + j0 + c) : 0.0f;
-                        s[c] = valid ? fmaf(s[c], c_log2, mv * kLog2e) : -INFINITY;
-                        mx = fmaxf(mx, s[c]);
-                    }
-                } else {
+                // keys c >= lim of this block are masked (padding / past the diagonal)
+                int lim = kv_len - j0;
+                if (p.is_causal && q_idx - j0 + 1 < lim) lim = q_idx - j0 + 1;
+                if constexpr (!HAS_MASK) {
                     if (boundary) {
-                        // keys c >= lim of this block are masked (padding / past the diagonal);
                         // one compare and select per element, c a compile-time constant
-                        int lim = kv_len - j0;
-                        if (p.is_causal && q_idx - j0 + 1 < lim) lim = q_idx - j0 + 1;
                         #pragma unroll
                         for (int c = 0; c < kBN; ++c) s[c] = (c < lim) ? s[c] : -INFINITY;
                     }
+                }
+                // exponent arguments and exponentials of keys [64h, 64h + 64) in place
+                auto exp_keys = [&](auto half_c, uint64_t ns2) {
+                    constexpr int kN = kBN / 2;
+                    float* sh = s + decltype(half_c)::value * kN;
+                    if constexpr (HAS_MASK) {
+                        const float sft = -lo_f32(ns2);
+                        #pragma unroll
+                        for (int c = 0; c < kN; ++c) sh[c] = ex2_approx(sh[c] - sft);
+                    } else {
+                        #pragma unroll
+                        for (int c = 0; c < kN / 2; ++c) {
+                            const uint64_t xv = ffma2(pack_f32x2(sh[2 * c], sh[2 * c + 1]), c2, ns2);
+                            sh[2 * c] = ex2_approx(lo_f32(xv));
+                            sh[2 * c + 1] = ex2_approx(hi_f32(xv));
+                        }
+                    }
+                };
+                auto row_max = [&]() -> float {
                     float m0 = fmax3(s[0], s[1], s[2]), m1 = fmax3(s[3], s[4], s[5]);
                     float m2 = fmax3(s[6], s[7], s[8]), m3 = fmax3(s[9], s[10], s[11]);
                     #pragma unroll
@@ -510,7 +480,22 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     }
                     m0 = fmax3(m0, s[kBN - 4], s[kBN - 3]);
                     m1 = fmax3(m1, s[kBN - 2], s[kBN - 1]);
-                    mx = fmax3(m0, m1, fmaxf(m2, m3)) * c_log2;
+                    return fmax3(m0, m1, fmaxf(m2, m3));
+                };
+
+                float mx;
+                if constexpr (HAS_MASK) {
+                    mx = -INFINITY;
+                    const int mlim = mask_row != nullptr ? lim : 0;
+                    #pragma unroll
+                    for (int c = 0; c < kBN; ++c) {
+                        const bool valid = c < mlim;
+                        const float mv = valid ? __ldg(mask_row + j0 + c) : 0.0f;
+                        s[c] = valid ? fmaf(s[c], c_log2, mv * kLog2e) : -INFINITY;
+                        mx = fmaxf(mx, s[c]);
+                    }
+                } else {
+                    mx = row_max() * c_log2;
                 }
 
                 // Lazy correction, decided per row: a row moves its reference max only when
@@ -531,38 +516,11 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 const float shift = (m_used == -INFINITY) ? 0.0f : m_used;
                 const uint64_t nshift2 = pack_f32x2(-shift, -shift);
 
-                // Three stages over the whole row, so that no instruction waits on the one
-                // just before it: (1) exponent arguments, (2) exponentials, (3) row sum and
-                // bf16 packing.
                 uint64_t acc0 = 0, acc1 = 0, acc2 = 0, acc3 = 0;  // packed partial sums
                 uint32_t pk[kBN / 4];
-                // Keys 0..63, then 64..127: each half is stored and signalled on its own
-                // (P0, P1), so PV over the first half runs during the second half.  O_t is
-                // rescaled (if needed) before P0 releases the first PV.
-                auto exp_half = [&](auto emulate, auto half_c) {
-                    constexpr int h = decltype(half_c)::value;
-                    float* sh = s + h * (kBN / 2);
-                    if constexpr (HAS_MASK) {
-                        #pragma unroll
-                        for (int c = 0; c < kBN / 2; ++c) sh[c] = sh[c] - shift;
-                    } else {
-                        #pragma unroll
-                        for (int c = 0; c < kBN / 4; ++c) {
-                            const uint64_t xv = ffma2(pack_f32x2(sh[2 * c], sh[2 * c + 1]), c2, nshift2);
-                            sh[2 * c] = lo_f32(xv);
-                            sh[2 * c + 1] = hi_f32(xv);
-                        }
-                    }
-                    #pragma unroll
-                    for (int c = 0; c < kBN / 4; ++c) {
-                        if (decltype(emulate)::value &&
-                            (c % (kExp2EmuEvery > 0 ? kExp2EmuEvery : 1)) == kExp2EmuEvery - 1) {
-                            exp2_poly_pair(pack_f32x2(sh[2 * c], sh[2 * c + 1]), sh[2 * c], sh[2 * c + 1]);
-                        } else {
-                            sh[2 * c] = ex2_approx(sh[2 * c]);
-                            sh[2 * c + 1] = ex2_approx(sh[2 * c + 1]);
-                        }
-                    }
+                // row-sum terms and bf16 pairs of keys [64h, 64h + 64)
+                auto pack_half = [&](auto half_c) {
+                    float* sh = s + decltype(half_c)::value * (kBN / 2);
                     #pragma unroll
                     for (int c = 0; c < kBN / 4; ++c) {
                         const uint64_t e = pack_f32x2(sh[2 * c], sh[2 * c + 1]);
@@ -574,6 +532,15 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         }
                         pk[c] = pack_bf16x2(sh[2 * c], sh[2 * c + 1]);
                     }
+                };
+                exp_keys(std::integral_constant<int, 0>{}, nshift2);
+                pack_half(std::integral_constant<int, 0>{});
+
+                // Keys 0..63, then 64..127: each half is stored and signalled on its own
+                // (P0, P1), so PV over the first half runs during the second half.  O_t is
+                // rescaled (if needed) before P0 releases the first PV.
+                auto store_half = [&](auto half_c) {
+                    constexpr int h = decltype(half_c)::value;
                     tmem_st32(s_tmem + h * 32, pk);
                     if (h == 0 && warp_rescale) {
                         #pragma unroll
@@ -590,15 +557,10 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     tc_fence_before();
                     mbar_arrive(bar((h == 0 ? L::P0 : L::P1) + t));
                 };
-                using Half0 = std::integral_constant<int, 0>;
-                using Half1 = std::integral_constant<int, 1>;
-                if (kExp2EmuEvery > 0 && !HAS_MASK && !boundary) {
-                    exp_half(std::integral_constant<bool, kExp2EmuEvery != 0>{}, Half0{});
-                    exp_half(std::integral_constant<bool, kExp2EmuEvery != 0>{}, Half1{});
-                } else {
-                    exp_half(std::false_type{}, Half0{});
-                    exp_half(std::false_type{}, Half1{});
-                }
+                store_half(std::integral_constant<int, 0>{});
+                exp_keys(std::integral_constant<int, 1>{}, nshift2);
+                pack_half(std::integral_constant<int, 1>{});
+                store_half(std::integral_constant<int, 1>{});
                 const uint64_t acc = fadd2(fadd2(acc0, acc2), fadd2(acc1, acc3));
                 l_sum += lo_f32(acc) + hi_f32(acc);
             }
