@@ -152,6 +152,33 @@ def barrier(world: int, device=None):
             dist.barrier()
 
 
+def mask2d_keys_per_row(w):
+    """Keys each query row may see under the workload's 2-D mask (numpy int
+    array of length Nq): the algorithmic work of a masked workload counts only
+    these (query, key) pairs."""
+    import numpy as np
+    kind, W, size = w.mask2d[0], int(w.mask2d[1]), int(w.mask2d[2])
+    shift = int(w.mask2d[3]) if len(w.mask2d) > 3 else 0
+    i = np.arange(w.Nq)[:, None]
+    j = np.arange(w.Nk)[None, :]
+    ri, ci, rj, cj = i // W, i % W, j // W, j % W
+    if kind == "neighborhood":
+        ok = (np.abs(ri - rj) < size) & (np.abs(ci - cj) < size)
+    else:
+        ok = ((ri + shift) // size == (rj + shift) // size) & ((ci + shift) // size == (cj + shift) // size)
+    if w.is_causal:
+        ok &= j <= i
+    return ok.sum(axis=1)
+
+
+def workload_flops(w):
+    """Forward FLOPs of one step: the metric's 4*B*Hq*Nq*Nk*d (halved when
+    causal) for dense workloads; 4*d per visible (query, key) pair under a 2-D mask."""
+    if w.mask2d is None:
+        return w.flops()
+    return 4.0 * w.d * w.B * w.Hq * float(mask2d_keys_per_row(w).sum())
+
+
 # ---------------------------------------------------------- CPU baseline
 def oracle_sample(w, q, k, v, kl, target_s: float, max_rows=None):
     """Runs the fp64 oracle on a bounded sample of the workload: whole query
@@ -168,11 +195,17 @@ def oracle_sample(w, q, k, v, kl, target_s: float, max_rows=None):
         return (q[b:b + 1, h:h + 1].cpu().double().numpy(), k[b:b + 1, hk:hk + 1].cpu().double().numpy(),
                 v[b:b + 1, hk:hk + 1].cpu().double().numpy(), None if kl_list is None else [kl_list[b]])
 
+    per_row = None if w.mask2d is None else mask2d_keys_per_row(w)
+    var = dict(softcap=w.softcap, mask2d=w.mask2d)
+
     def flops_of(b, rows):
         nk = w.Nk if kl_list is None else kl_list[b]
         total = 0.0
         for i in rows:
-            keys = min(nk, i + 1) if w.is_causal else nk
+            if per_row is not None:
+                keys = int(per_row[i])
+            else:
+                keys = min(nk, i + 1) if w.is_causal else nk
             total += 4.0 * keys * w.d
         return total
 
@@ -180,7 +213,7 @@ def oracle_sample(w, q, k, v, kl, target_s: float, max_rows=None):
     qh, kh, vh, klh = head_inputs(0, 0)
     cal_rows = list(range(0, w.Nq, max(1, w.Nq // max(1, min(w.Nq, 4 * threads)))))[: 4 * threads]
     t0 = time.perf_counter()
-    oracle.attention(qh, kh, vh, is_causal=w.is_causal, key_lens=klh, rows=cal_rows)
+    oracle.attention(qh, kh, vh, is_causal=w.is_causal, key_lens=klh, rows=cal_rows, **var)
     t_cal = max(time.perf_counter() - t0, 1e-6)
     per_flop = t_cal / max(flops_of(0, cal_rows), 1.0)
     budget = target_s / per_flop  # flops we can afford
@@ -207,7 +240,7 @@ def oracle_sample(w, q, k, v, kl, target_s: float, max_rows=None):
     for b, h, rows in plan:
         qh, kh, vh, klh = head_inputs(b, h)
         oracle.attention(qh, kh, vh, is_causal=w.is_causal, key_lens=klh,
-                         rows=None if len(rows) == w.Nq else rows)
+                         rows=None if len(rows) == w.Nq else rows, **var)
         total += flops_of(b, rows)
     dt = time.perf_counter() - t0
     n_rows = sum(len(r) for _, _, r in plan)
@@ -234,7 +267,7 @@ def run_ours(args, w):
     out = torch.empty_like(q)
     lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
-    flops = w.flops()
+    flops = workload_flops(w)
     in_bytes = q.numel() * 2 + k.numel() * 2 + v.numel() * 2 + (0 if kl is None else kl.numel() * 4)
     out_bytes = out.numel() * 2 + lse.numel() * 4
     l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
@@ -254,7 +287,7 @@ def run_ours(args, w):
 
     def call():
         ea.attention(q, k, v, is_causal=w.is_causal, key_lens=kl, out=out, lse=lse, stream=stream,
-                     split_kv=split, workspace=ws)
+                     split_kv=split, workspace=ws, softcap=w.softcap, mask2d=w.mask2d)
 
     def step():
         if flush is not None:
@@ -304,13 +337,15 @@ def run_ours(args, w):
                               split_kv=split)
     e2e_steps = max(1, min(args.steps, 20))
     for _ in range(min(args.warmup, 3)):
-        runner(qh, kh, vh, outh, lseh, klh, is_causal=w.is_causal, stream=stream)
+        runner(qh, kh, vh, outh, lseh, klh, is_causal=w.is_causal, stream=stream, softcap=w.softcap,
+               mask2d=w.mask2d)
     barrier(world, dev)
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(e2e_steps):
-        runner(qh, kh, vh, outh, lseh, klh, is_causal=w.is_causal, stream=stream)
+        runner(qh, kh, vh, outh, lseh, klh, is_causal=w.is_causal, stream=stream, softcap=w.softcap,
+               mask2d=w.mask2d)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / e2e_steps
@@ -348,7 +383,9 @@ def run_ours(args, w):
                                f"{' causal' if w.is_causal else ''}",
                    "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Nq": w.Nq, "Nk": w.Nk, "d": w.d,
                    "is_causal": w.is_causal, "key_lens": w.key_lens,
-                   "entry_point": "attn_fwd_splitkv" if w.split_kv else "attn_fwd",
+                   "entry_point": ("attn_fwd_splitkv" if w.split_kv else
+                                   "attn_fwd_mod" if (w.softcap or w.mask2d) else "attn_fwd"),
+                   "softcap": w.softcap, "mask2d": w.mask2d,
                    "flops_per_step": flops, "parallelism": f"independent batch per GPU x{world}",
                    "l2": ("L2 flushed between steps (kernel time only)" if flush is not None
                           else f"inputs larger than L2 ({in_bytes / 1e6:.0f} MB > {l2_bytes / 1e6:.0f} MB)")},

@@ -38,9 +38,29 @@ ATTN_ERR_SCRATCH = 7
 NOALLOC_SCRATCH_BYTES = 16 << 20  # ATTN_NOALLOC_SCRATCH_BYTES
 
 # Every symbol include/attn.h declares.
-EXPORTED = ("attn_fwd", "attn_splitkv_plan", "attn_fwd_splitkv", "attn_fwd_splitkv_noalloc",
+EXPORTED = ("attn_fwd", "attn_fwd_mod", "attn_splitkv_plan", "attn_fwd_splitkv", "attn_fwd_splitkv_noalloc",
             "attn_check_device_status", "attn_set_wait_timeout_ns", "attn_selftest_timeout",
             "attn_status_string", "attn_last_cuda_error", "attn_version")
+
+MASK2D_KINDS = {None: 0, "neighborhood": 1, "window": 2}
+
+
+class AttnScoreMod(ctypes.Structure):
+    """attn_score_mod_t of include/attn.h."""
+    _fields_ = [("softcap", ctypes.c_float), ("mask2d_kind", ctypes.c_int), ("grid_w", ctypes.c_int),
+                ("size", ctypes.c_int), ("shift", ctypes.c_int)]
+
+
+def score_mod(softcap=0.0, mask2d=None) -> AttnScoreMod:
+    """Build an attn_score_mod_t: mask2d is None, ("neighborhood", W, R) or
+    ("window", W, w[, shift])."""
+    m = AttnScoreMod(float(softcap or 0.0), 0, 0, 0, 0)
+    if mask2d is not None:
+        m.mask2d_kind = MASK2D_KINDS[mask2d[0]]
+        m.grid_w, m.size = int(mask2d[1]), int(mask2d[2])
+        m.shift = int(mask2d[3]) if len(mask2d) > 3 else 0
+    return m
+
 
 _lock = threading.Lock()
 _lib = None
@@ -67,6 +87,8 @@ def lib() -> ctypes.CDLL:
             vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
             L.attn_fwd.restype = i
             L.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, vp, vp, vp]
+            L.attn_fwd_mod.restype = i
+            L.attn_fwd_mod.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, ctypes.POINTER(AttnScoreMod), vp]
             L.attn_splitkv_plan.restype = i
             L.attn_splitkv_plan.argtypes = [i, i, i, i, i, i, i, ctypes.POINTER(i), ctypes.POINTER(ctypes.c_size_t)]
             L.attn_fwd_splitkv.restype = i
@@ -112,6 +134,15 @@ def attn_fwd(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, is_causal,
         ms = ctypes.cast(arr, ctypes.c_void_p)
     return int(lib().attn_fwd(q, k, v, out, lse, int(B), int(Hq), int(Hkv), int(Nq), int(Nk), int(d),
                               float(scale), int(bool(is_causal)), key_lens, additive_mask, ms, stream))
+
+
+def attn_fwd_mod(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, is_causal, key_lens=None, mod=None,
+                 stream=None) -> int:
+    """The C variant entry point with raw device pointers (ints) and an
+    AttnScoreMod (or None, passed as NULL); returns the status code."""
+    return int(lib().attn_fwd_mod(q, k, v, out, lse, int(B), int(Hq), int(Hkv), int(Nq), int(Nk), int(d),
+                                  float(scale), int(bool(is_causal)), key_lens,
+                                  None if mod is None else ctypes.byref(mod), stream))
 
 
 def attn_splitkv_plan(B, Hq, Nq, Nk, d, n_splits=0, sm_count=0):
@@ -185,7 +216,7 @@ def _check_bf16_cuda(name, t, ndim):
 
 def attention(q, k, v, *, scale: float | None = None, is_causal: bool = False, key_lens=None,
               attn_mask=None, out=None, lse=None, return_lse: bool = True, stream=None,
-              split_kv: int | None = None, workspace=None):
+              split_kv: int | None = None, workspace=None, softcap: float = 0.0, mask2d=None):
     """O = softmax(scale * Q K^T + mask) V on bf16 CUDA tensors.
 
     q [B, Hq, Nq, d], k/v [B, Hkv, Nk, d] (contiguous bf16); key_lens int32 [B]
@@ -193,7 +224,9 @@ def attention(q, k, v, *, scale: float | None = None, is_causal: bool = False, k
     with a contiguous last dimension, or None.  split_kv=None runs attn_fwd;
     an int runs attn_fwd_splitkv with at most that many key ranges (0 =
     automatic), its workspace taken from ``workspace`` (a CUDA tensor of at
-    least the planned bytes) or allocated here.  Returns (out, lse or None).
+    least the planned bytes) or allocated here.  softcap > 0 or a mask2d
+    (("neighborhood", W, R) or ("window", W, w[, shift])) runs attn_fwd_mod.
+    Returns (out, lse or None).
     """
     import torch
     _check_bf16_cuda("q", q, 4)
@@ -233,6 +266,14 @@ def attention(q, k, v, *, scale: float | None = None, is_causal: bool = False, k
         m_ptr, m_strides = m.data_ptr(), (m.stride(0), m.stride(1), m.stride(2))
     sc = 0.0 if scale is None else float(scale)
     lse_ptr = None if lse is None else lse.data_ptr()
+    if softcap or mask2d is not None:
+        if split_kv is not None or attn_mask is not None:
+            raise ValueError("softcap / mask2d combine with neither split_kv nor attn_mask")
+        st = attn_fwd_mod(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse_ptr, B, Hq, Hkv, Nq, Nk, d,
+                          sc, is_causal, kl_ptr, score_mod(softcap, mask2d), _stream_handle(stream))
+        if st != ATTN_OK:
+            raise AttnError(st, "attn_fwd_mod")
+        return out, lse
     if split_kv is None:
         st = attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse_ptr, B, Hq, Hkv, Nq, Nk, d,
                       sc, is_causal, kl_ptr, m_ptr, m_strides, _stream_handle(stream))
@@ -291,7 +332,7 @@ class HostAttention:
             self.workspace = torch.empty((max(nbytes, 1),), dtype=torch.uint8, device=dev)
 
     def __call__(self, q_h, k_h, v_h, out_h, lse_h=None, key_lens_h=None, *, scale=None,
-                 is_causal=False, stream=None):
+                 is_causal=False, stream=None, softcap=0.0, mask2d=None):
         import torch
         s = torch.cuda.current_stream() if stream is None else stream
         with torch.cuda.stream(s):
@@ -304,7 +345,7 @@ class HostAttention:
                 kl = self.key_lens
             attention(self.q, self.k, self.v, scale=scale, is_causal=is_causal, key_lens=kl,
                       out=self.out, lse=self.lse, return_lse=self.lse is not None, stream=s,
-                      split_kv=self.split_kv, workspace=self.workspace)
+                      split_kv=self.split_kv, workspace=self.workspace, softcap=softcap, mask2d=mask2d)
             out_h.copy_(self.out, non_blocking=True)
             if lse_h is not None and self.lse is not None:
                 lse_h.copy_(self.lse, non_blocking=True)

@@ -55,11 +55,15 @@ constexpr int kSlots64 = 8, kQStages64 = 2;
 
 template <int D, int NSLOT, int QS, bool M>
 cudaError_t set_pp_attrs() {
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_pp_kernel<D, NSLOT, QS, M, false>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SmemPP<D, NSLOT, QS>::kAlloc);
+    constexpr int kSmem = SmemPP<D, NSLOT, QS>::kAlloc;
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_pp_kernel<D, NSLOT, QS, M, false, false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(attn_fwd_pp_kernel<D, NSLOT, QS, M, true>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize, SmemPP<D, NSLOT, QS>::kAlloc);
+    e = cudaFuncSetAttribute(attn_fwd_pp_kernel<D, NSLOT, QS, M, true, false>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    if (e != cudaSuccess || M) return e;
+    return cudaFuncSetAttribute(attn_fwd_pp_kernel<D, NSLOT, QS, false, false, true>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
 }
 
 // One-time per-device set-up: architecture check, SM count, kernel attributes,
@@ -119,12 +123,13 @@ attn_status_t encode_map(CUtensorMap* map, const void* base, int d, int rows, lo
 template <int D, int NSLOT, int QS, bool M>
 cudaError_t launch_pp(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
                       const FwdParams& p, unsigned grid, cudaStream_t stream) {
+    constexpr int kSmem = SmemPP<D, NSLOT, QS>::kAlloc;
     if (p.n_splits > 1)
-        attn_fwd_pp_kernel<D, NSLOT, QS, M, true>
-            <<<grid, kPPThreads, SmemPP<D, NSLOT, QS>::kAlloc, stream>>>(tq, tk, tv, to, p);
+        attn_fwd_pp_kernel<D, NSLOT, QS, M, true, false><<<grid, kPPThreads, kSmem, stream>>>(tq, tk, tv, to, p);
+    else if (!M && (p.softcap_on || p.m2_kind != 0))
+        attn_fwd_pp_kernel<D, NSLOT, QS, false, false, true><<<grid, kPPThreads, kSmem, stream>>>(tq, tk, tv, to, p);
     else
-        attn_fwd_pp_kernel<D, NSLOT, QS, M, false>
-            <<<grid, kPPThreads, SmemPP<D, NSLOT, QS>::kAlloc, stream>>>(tq, tk, tv, to, p);
+        attn_fwd_pp_kernel<D, NSLOT, QS, M, false, false><<<grid, kPPThreads, kSmem, stream>>>(tq, tk, tv, to, p);
     return cudaGetLastError();
 }
 
@@ -171,7 +176,7 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, f
                        const int32_t* key_lens,
                        const float* additive_mask, const int64_t* mask_strides,
                        bool split_kv, int n_splits_req, void* workspace, size_t workspace_bytes,
-                       void* stream) {
+                       const attn_score_mod_t* mod, void* stream) {
     // ---- host-side validation (no CUDA call before this passes)
     if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return ATTN_ERR_INVALID_ARG;
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nk <= 0 || d <= 0) return ATTN_ERR_INVALID_ARG;
@@ -200,6 +205,16 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, f
 
     if (split_kv && (n_splits_req < 0 || (workspace != nullptr && reinterpret_cast<uintptr_t>(workspace) % kWsAlign)))
         return n_splits_req < 0 ? ATTN_ERR_INVALID_ARG : ATTN_ERR_ALIGNMENT;
+    const bool use_mod = mod != nullptr && (mod->softcap != 0.0f || mod->mask2d_kind != ATTN_MASK2D_NONE);
+    if (mod != nullptr) {
+        if (!std::isfinite(mod->softcap) || mod->softcap < 0.0f) return ATTN_ERR_INVALID_ARG;
+        if (mod->mask2d_kind != ATTN_MASK2D_NONE && mod->mask2d_kind != ATTN_MASK2D_NEIGHBORHOOD &&
+            mod->mask2d_kind != ATTN_MASK2D_WINDOW)
+            return ATTN_ERR_INVALID_ARG;
+        if (mod->mask2d_kind != ATTN_MASK2D_NONE && (mod->grid_w <= 0 || mod->size <= 0 || mod->shift < 0))
+            return ATTN_ERR_INVALID_ARG;
+    }
+    if (use_mod && (additive_mask != nullptr || split_kv)) return ATTN_ERR_UNSUPPORTED;
 
     int dev = 0;
     attn_status_t st = device_setup(&dev);
@@ -217,6 +232,29 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, f
     p.lse = lse;
     p.out = out;
     p.unit_run = 1;
+    p.softcap_on = 0;
+    p.sc_in = 0.0f;
+    p.sc_out = 0.0f;
+    p.m2_kind = 0;
+    p.m2_w = 1;
+    p.m2_size = 1;
+    p.m2_shift = 0;
+    if (use_mod) {
+        if (mod->softcap > 0.0f) {
+            // the kernel turns each raw score into the base-2 logit cap*log2(e)*tanh(scale*s/cap),
+            // so the later steps use a unit scale
+            p.softcap_on = 1;
+            p.sc_in = static_cast<float>(2.0 * scale_eff * 1.4426950408889634 / mod->softcap);
+            p.sc_out = static_cast<float>(static_cast<double>(mod->softcap) * 1.4426950408889634);
+            p.scale_log2 = 1.0f;
+        }
+        p.m2_kind = mod->mask2d_kind;
+        if (p.m2_kind != ATTN_MASK2D_NONE) {
+            p.m2_w = mod->grid_w;
+            p.m2_size = mod->size;
+            p.m2_shift = mod->shift;
+        }
+    }
     p.timeout_ns = g_timeout_ns.load();
     p.epoch = next_epoch();
 
@@ -292,7 +330,18 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* out, f
                        const float* additive_mask, const int64_t* mask_strides,
                        void* stream) {
     return fwd_impl(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, is_causal, key_lens, additive_mask,
-                    mask_strides, false, 1, nullptr, 0, stream);
+                    mask_strides, false, 1, nullptr, 0, nullptr, stream);
+}
+
+attn_status_t attn_fwd_mod(const void* q, const void* k, const void* v, void* out, float* lse,
+                           int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                           float scale, int is_causal,
+                           const int32_t* key_lens,
+                           const attn_score_mod_t* mod,
+                           void* stream) {
+    if (mod == nullptr) return ATTN_ERR_INVALID_ARG;
+    return fwd_impl(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, is_causal, key_lens, nullptr, nullptr,
+                    false, 1, nullptr, 0, mod, stream);
 }
 
 attn_status_t attn_splitkv_plan(int B, int Hq, int Nq, int Nk, int d, int n_splits, int sm_count,
@@ -325,7 +374,7 @@ attn_status_t attn_fwd_splitkv(const void* q, const void* k, const void* v, void
                                int n_splits, void* workspace, size_t workspace_bytes,
                                void* stream) {
     return fwd_impl(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, is_causal, key_lens, additive_mask,
-                    mask_strides, true, n_splits, workspace, workspace_bytes, stream);
+                    mask_strides, true, n_splits, workspace, workspace_bytes, nullptr, stream);
 }
 
 attn_status_t attn_check_device_status(void* stream, uint32_t* info) {
@@ -427,5 +476,6 @@ extern "C" attn_status_t attn_fwd_splitkv_noalloc(const void* q, const void* k, 
     if ((st = noalloc_scratch(dev, &scratch)) != ATTN_OK) return st;
     // the plan above is the one fwd_impl makes for the same sizes and n_splits
     return fwd_impl(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, is_causal, key_lens, additive_mask,
-                    mask_strides, true, n_splits, scratch, static_cast<size_t>(ATTN_NOALLOC_SCRATCH_BYTES), stream);
+                    mask_strides, true, n_splits, scratch, static_cast<size_t>(ATTN_NOALLOC_SCRATCH_BYTES), nullptr,
+                    stream);
 }

@@ -36,9 +36,48 @@ struct FwdParams {
     int split_keys;
     float* ws_o;
     float* ws_lse;
+    // score and mask variants (the MOD instantiation): soft-capped scores
+    // cap * tanh(x / cap) of the scaled score x, and 2-D masks on a row-major
+    // token grid of m2_w tokens per row (kind 1: neighbourhood of radius
+    // m2_size, kind 2: m2_size x m2_size windows displaced by m2_shift)
+    int softcap_on;
+    float sc_in;   // 2 * scale * log2(e) / cap: base-2 exponent of e^(2x / cap) per raw score
+    float sc_out;  // cap * log2(e)
+    int m2_kind, m2_w, m2_size, m2_shift;
     unsigned long long timeout_ns;
     unsigned int epoch;  // launch id for the launch-wide abort (never 0)
 };
+
+// Rectangle of the token grid that query row i may see under a 2-D mask: key
+// rows [r_lo, r_hi] and, within each, columns [c_lo, c_hi] (clipped to the grid).
+struct Rect2D {
+    int r_lo, r_hi, c_lo, c_hi;
+};
+
+__device__ __forceinline__ Rect2D rect_2d(const FwdParams& p, int i) {
+    const long long W = p.m2_w;
+    const long long qr = i / W, qc = i - qr * W;
+    long long r_lo, r_hi, c_lo, c_hi;
+    if (p.m2_kind == 1) {  // |dr| < R and |dc| < R
+        r_lo = qr - p.m2_size + 1;
+        r_hi = qr + p.m2_size - 1;
+        c_lo = qc - p.m2_size + 1;
+        c_hi = qc + p.m2_size - 1;
+    } else {  // same displaced window
+        const long long w = p.m2_size, sh = p.m2_shift;
+        r_lo = ((qr + sh) / w) * w - sh;
+        r_hi = r_lo + w - 1;
+        c_lo = ((qc + sh) / w) * w - sh;
+        c_hi = c_lo + w - 1;
+    }
+    const long long last_row = (static_cast<long long>(p.Nk) - 1) / W;  // key rows that exist
+    Rect2D r;
+    r.r_lo = static_cast<int>(r_lo < 0 ? 0 : r_lo);
+    r.r_hi = static_cast<int>(r_hi > last_row ? last_row : r_hi);
+    r.c_lo = static_cast<int>(c_lo < 0 ? 0 : c_lo);
+    r.c_hi = static_cast<int>(c_hi > W - 1 ? W - 1 : c_hi);
+    return r;
+}
 
 // Split-KV combine: for each output row, merge the n_splits partial results
 // (O_s normalised by its own row sum, LSE_s) of disjoint key ranges:

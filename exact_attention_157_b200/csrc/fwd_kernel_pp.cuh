@@ -135,7 +135,7 @@ __device__ __forceinline__ int unit_key_len(const FwdParams& p, int s, int n_uni
 
 // Units are numbered (head, split, query-unit): the units of one head and key
 // range are adjacent.  Without split-KV (SPLIT = false) there is one range.
-template <bool SPLIT>
+template <bool SPLIT, bool MOD>
 __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int s, int kv_len, bool report) {
     Unit x;
     int pos;
@@ -162,11 +162,22 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int s, int kv_le
         kv_len = kv_len < 0 ? 0 : p.Nk;
     }
     x.kv_len = kv_len;
-    const int k_lo = SPLIT ? x.split * p.split_keys : 0;  // a multiple of kBN
+    int k_lo = SPLIT ? x.split * p.split_keys : 0;  // a multiple of kBN
+    int k_hi = x.kv_len;
+    if constexpr (MOD) {
+        if (p.m2_kind != 0) {
+            // keys of the grid rows that the unit's first and last query rows may see
+            const int q_last = (x.q0 + 2 * kBM - 1 < p.Nq - 1) ? x.q0 + 2 * kBM - 1 : p.Nq - 1;
+            const Rect2D a = rect_2d(p, x.q0), z = rect_2d(p, q_last);
+            k_lo = (a.r_lo * p.m2_w) / kBN * kBN;
+            const long long hi = (static_cast<long long>(z.r_hi) + 1) * p.m2_w;
+            if (hi < k_hi) k_hi = static_cast<int>(hi);
+        }
+    }
     x.j_lo = k_lo / kBN;
     #pragma unroll
     for (int t = 0; t < 2; ++t) {
-        int end = x.kv_len;
+        int end = k_hi;
         if (p.is_causal && x.q0 + (t + 1) * kBM < end) end = x.q0 + (t + 1) * kBM;
         if (SPLIT && k_lo + p.split_keys < end) end = k_lo + p.split_keys;
         x.n_t[t] = end > k_lo ? (end - k_lo + kBN - 1) / kBN : 0;
@@ -175,7 +186,7 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int s, int kv_le
     return x;
 }
 
-template <int D, int NSLOT, int QS, bool HAS_MASK, bool SPLIT>
+template <int D, int NSLOT, int QS, bool HAS_MASK, bool SPLIT, bool MOD>
 __global__ void __launch_bounds__(kPPThreads, 1)
 attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -252,7 +263,7 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             int it = 0;
             int kv_next = unit_key_len(p, unit_seq(cta, 0, G, p.unit_run), n_units);
             for (int u = unit_seq(cta, 0, G, p.unit_run); ok && u < n_units; ++it, u = unit_seq(cta, it, G, p.unit_run)) {
-                const Unit x = decode_unit<SPLIT>(p, u, kv_next, false);
+                const Unit x = decode_unit<SPLIT, MOD>(p, u, kv_next, false);
                 kv_next = unit_key_len(p, unit_seq(cta, it + 1, G, p.unit_run), n_units);
                 const int qb = it % QS;
                 const int n_max = x.n_max();
@@ -309,7 +320,7 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             int it = 0;
             int kv_next = unit_key_len(p, unit_seq(cta, 0, G, p.unit_run), n_units);
             for (int u = unit_seq(cta, 0, G, p.unit_run); ok && u < n_units; ++it, u = unit_seq(cta, it, G, p.unit_run)) {
-                const Unit x = decode_unit<SPLIT>(p, u, kv_next, false);
+                const Unit x = decode_unit<SPLIT, MOD>(p, u, kv_next, false);
                 kv_next = unit_key_len(p, unit_seq(cta, it + 1, G, p.unit_run), n_units);
                 const int n_max = x.n_max();
                 if (n_max == 0) continue;
@@ -412,7 +423,7 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         int it = 0;
         int kv_next = unit_key_len(p, unit_seq(cta, 0, G, p.unit_run), n_units);
         for (int u = unit_seq(cta, 0, G, p.unit_run); u < n_units; ++it, u = unit_seq(cta, it, G, p.unit_run)) {
-            const Unit x = decode_unit<SPLIT>(p, u, kv_next, threadIdx.x == 0);
+            const Unit x = decode_unit<SPLIT, MOD>(p, u, kv_next, threadIdx.x == 0);
             kv_next = unit_key_len(p, unit_seq(cta, it + 1, G, p.unit_run), n_units);
             const int q0_t = x.q0 + t * kBM;
             const int q_idx = q0_t + row;
@@ -420,6 +431,10 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             const int kv_len = x.kv_len;
             float m_used = -INFINITY;  // running max (base-2, scaled), possibly stale by < tau
             float l_sum = 0.0f;        // running sum of exp2(t - m_used)
+            Rect2D rq{0, 0, 0, 0};
+            if constexpr (MOD) {
+                if (p.m2_kind != 0) rq = rect_2d(p, q_idx);
+            }
             const float* mask_row = nullptr;
             if constexpr (HAS_MASK) {
                 if (q_idx < p.Nq)
@@ -444,7 +459,40 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 // keys c >= lim of this block are masked (padding / past the diagonal)
                 int lim = kv_len - j0;
                 if (p.is_causal && q_idx - j0 + 1 < lim) lim = q_idx - j0 + 1;
-                if constexpr (!HAS_MASK) {
+                if constexpr (MOD) {
+                    if (p.softcap_on) {
+                        // base-2 logit cap * log2(e) * tanh(x / cap), with tanh(u) = 1 - 2 / (1 + e^(2u))
+                        #pragma unroll
+                        for (int c = 0; c < kBN; ++c)
+                            s[c] = fmaf(rcp_approx(1.0f + ex2_approx(s[c] * p.sc_in)), -2.0f * p.sc_out, p.sc_out);
+                    }
+                    if (p.m2_kind != 0) {
+                        // keys of this block inside the row's grid rectangle, as a 128-bit set:
+                        // one run of columns per key row the block touches
+                        uint32_t mw[kBN / 32] = {0u, 0u, 0u, 0u};
+                        const int W = p.m2_w;
+                        int kr = j0 / W;
+                        const int kr_end = (j0 + kBN - 1) / W;
+                        if (kr < rq.r_lo) kr = rq.r_lo;
+                        for (; kr <= kr_end && kr <= rq.r_hi; ++kr) {
+                            int a = kr * W + rq.c_lo - j0, b = kr * W + rq.c_hi - j0;
+                            if (a < 0) a = 0;
+                            if (b > kBN - 1) b = kBN - 1;
+                            #pragma unroll
+                            for (int w = 0; w < kBN / 32; ++w) {
+                                const int lo = a - 32 * w > 0 ? a - 32 * w : 0;
+                                const int hi = b - 32 * w < 31 ? b - 32 * w : 31;
+                                if (lo <= hi) mw[w] |= ((2u << (hi - lo)) - 1u) << lo;
+                            }
+                        }
+                        #pragma unroll
+                        for (int c = 0; c < kBN; ++c)
+                            s[c] = (((mw[c >> 5] >> (c & 31)) & 1u) && c < lim) ? s[c] : -INFINITY;
+                    } else if (boundary) {
+                        #pragma unroll
+                        for (int c = 0; c < kBN; ++c) s[c] = (c < lim) ? s[c] : -INFINITY;
+                    }
+                } else if constexpr (!HAS_MASK) {
                     if (boundary) {
                         // one compare and select per element, c a compile-time constant
                         #pragma unroll

@@ -87,6 +87,59 @@ attn_status_t attn_fwd(const void *q, const void *k, const void *v, void *out, f
                        void *stream);
 
 /*
+ * Score and mask variants for attn_fwd_mod.
+ *
+ * softcap > 0 replaces the scaled score x = scale * q.k by softcap * tanh(x /
+ * softcap) before the softmax: the score_mod example ("soft-capping with
+ * tanh", cap 30) of the PyTorch attention article (atyun.com/61003.html).
+ * 0 disables it.
+ *
+ * mask2d_kind treats the tokens as a row-major grid with grid_w tokens per
+ * row, token n at (n / grid_w, n % grid_w):
+ *   ATTN_MASK2D_NEIGHBORHOOD: query i sees key j iff |r_i - r_j| < size and
+ *     |c_i - c_j| < size -- the mask_mod example ("neighbourhood masking",
+ *     grid 56 wide, size 5) of the same article;
+ *   ATTN_MASK2D_WINDOW: the grid is cut into non-overlapping size x size
+ *     windows displaced by `shift` tokens in both directions (0 = plain,
+ *     size / 2 = shifted; border windows are partial, no cyclic wrap); query i
+ *     sees key j iff both lie in the same window -- the window attention of
+ *     "Flash Attention in a production Stable-Diffusion service"
+ *     (xxmr.cn/news/81028), section 3.2.
+ * Key blocks that no query of a work unit may see are skipped, as causal
+ * attention skips the blocks above the diagonal.
+ */
+enum {
+    ATTN_MASK2D_NONE = 0,
+    ATTN_MASK2D_NEIGHBORHOOD = 1,
+    ATTN_MASK2D_WINDOW = 2
+};
+
+typedef struct attn_score_mod_t {
+    float softcap;   /* >= 0, finite; 0 = off */
+    int mask2d_kind; /* ATTN_MASK2D_* */
+    int grid_w;      /* tokens per grid row, >= 1 (2-D masks only) */
+    int size;        /* neighbourhood radius or window side, >= 1 (2-D masks only) */
+    int shift;       /* window displacement, >= 0 (windows only) */
+} attn_score_mod_t;
+
+/*
+ * attn_fwd_mod -- attn_fwd with the variants of `mod` (host pointer, read
+ * during the call only).  Soft-capping and 2-D masks combine with each other,
+ * with is_causal and with key_lens (all masks intersect); an additive mask is
+ * not accepted here.  With softcap = 0 and no 2-D mask it computes exactly
+ * what attn_fwd computes.
+ * Errors: as attn_fwd; ATTN_ERR_INVALID_ARG also for mod == NULL, a negative
+ * or non-finite softcap, an unknown kind, or grid_w / size < 1 or shift < 0
+ * with a 2-D mask.
+ */
+attn_status_t attn_fwd_mod(const void *q, const void *k, const void *v, void *out, float *lse,
+                           int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                           float scale, int is_causal,
+                           const int32_t *key_lens,
+                           const attn_score_mod_t *mod,
+                           void *stream);
+
+/*
  * attn_splitkv_plan -- how attn_fwd_splitkv would split the keys, and the
  * workspace it then needs.  Host-only arithmetic (no CUDA call) when
  * sm_count > 0; sm_count == 0 queries the current device's SM count.

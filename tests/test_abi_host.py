@@ -147,3 +147,26 @@ def test_splitkv_validation_is_host_side(args, status):
               scale=0.0, is_causal=0, n_splits=4, workspace=A, workspace_bytes=1 << 20)
     kw.update(args)
     assert ea.attn_fwd_splitkv(**kw) == status
+
+
+# ------------------------------------------------------------ score / mask variants
+@pytest.mark.parametrize("mod,status", [
+    (None, ea.ATTN_ERR_INVALID_ARG),
+    (ea.score_mod(softcap=-1.0), ea.ATTN_ERR_INVALID_ARG),
+    (ea.score_mod(softcap=float("inf")), ea.ATTN_ERR_INVALID_ARG),
+    (ea.AttnScoreMod(0.0, 3, 8, 2, 0), ea.ATTN_ERR_INVALID_ARG),
+    (ea.score_mod(mask2d=("neighborhood", 0, 2)), ea.ATTN_ERR_INVALID_ARG),
+    (ea.score_mod(mask2d=("window", 8, 0)), ea.ATTN_ERR_INVALID_ARG),
+    (ea.score_mod(mask2d=("window", 8, 4, -1)), ea.ATTN_ERR_INVALID_ARG),
+])
+def test_score_mod_validation_is_host_side(mod, status):
+    assert ea.attn_fwd_mod(A, A, A, A, None, 1, 2, 2, 64, 64, 64, 0.0, 0, mod=mod) == status
+
+
+def test_score_mod_struct_layout_matches_header():
+    import re
+    text = open(HEADER).read()
+    body = re.search(r"typedef struct attn_score_mod_t \{(.*?)\} attn_score_mod_t;", text, re.S).group(1)
+    names = re.findall(r"\b(?:float|int)\s+(\w+);", body)
+    assert names == [f[0] for f in ea.AttnScoreMod._fields_]
+    assert ctypes.sizeof(ea.AttnScoreMod) == 20

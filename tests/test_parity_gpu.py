@@ -199,12 +199,14 @@ def test_workload_vs_oracle(name):
     w = WORKLOADS[name]
     dev = torch.device("cuda:0")
     q, k, v, kl = make_inputs(w, device=dev)
-    out, lse = ea.attention(q, k, v, is_causal=w.is_causal, key_lens=kl, split_kv=0 if w.split_kv else None)
+    out, lse = ea.attention(q, k, v, is_causal=w.is_causal, key_lens=kl, split_kv=0 if w.split_kv else None,
+                            softcap=w.softcap, mask2d=w.mask2d)
     ea.check_device_status()
     full = w.B * w.Hq * w.Nq * w.Nk * w.d <= 2e10
     kl_list = None if kl is None else kl.cpu().tolist()
+    var = dict(softcap=w.softcap, mask2d=w.mask2d)
     if full:
-        ro, rl = oracle.attention(q.cpu(), k.cpu(), v.cpu(), is_causal=w.is_causal, key_lens=kl_list)
+        ro, rl = oracle.attention(q.cpu(), k.cpu(), v.cpu(), is_causal=w.is_causal, key_lens=kl_list, **var)
         assert_close(out.cpu(), lse.cpu(), ro, rl)
         return
     group = w.Hq // w.Hkv
@@ -213,7 +215,7 @@ def test_workload_vs_oracle(name):
         rows = sample_rows(w.Nq, 512, seed=b * 1000 + h)
         ro, rl = oracle.attention(q[b:b + 1, h:h + 1].cpu(), k[b:b + 1, hk:hk + 1].cpu(),
                                   v[b:b + 1, hk:hk + 1].cpu(), is_causal=w.is_causal,
-                                  key_lens=None if kl_list is None else [kl_list[b]], rows=rows)
+                                  key_lens=None if kl_list is None else [kl_list[b]], rows=rows, **var)
         assert_close(out[b:b + 1, h:h + 1].cpu(), lse[b:b + 1, h:h + 1].cpu(), ro, rl, rows=rows)
     assert torch.isfinite(out).all()
 

@@ -23,6 +23,10 @@ used):
                                                cache, grouped heads (the decoding
                                                phase of jsqmd.com/news/722897,
                                                section 5.2); run with split-KV
+  vit3136_softcap       B8 H12 N3136 d64, soft-cap 30 -- the 56 x 56-patch ViT of
+  vit3136_neighborhood  B8 H12 N3136 d64, radius-5      the PyTorch attention article
+                        neighbourhood on the 56-wide    (atyun.com/61003.html: its
+                        token grid                      score_mod and mask_mod examples)
 """
 from __future__ import annotations
 
@@ -45,6 +49,8 @@ class Workload:
     key_lens: tuple | None = None  # (low, high) inclusive range of per-sample key lengths
     seed: int = 0
     split_kv: bool = False  # run through the split-KV entry point (automatic range count)
+    softcap: float = 0.0    # > 0: soft-capped scores (attn_fwd_mod)
+    mask2d: tuple | None = None  # ("neighborhood", W, R) or ("window", W, w, shift) (attn_fwd_mod)
 
     @property
     def scale(self) -> float:
@@ -77,6 +83,8 @@ WORKLOADS = {
         Workload("unet_cross", 4, 8, 8, 4096, 77, 64, key_lens=(8, 77), seed=1013),
         Workload("prefill_gqa", 1, 32, 2, 16384, 16384, 128, is_causal=True, seed=1004),
         Workload("decode_gqa", 8, 32, 8, 1, 16384, 128, seed=1005, split_kv=True),
+        Workload("vit3136_softcap", 8, 12, 12, 3136, 3136, 64, seed=1006, softcap=30.0),
+        Workload("vit3136_neighborhood", 8, 12, 12, 3136, 3136, 64, seed=1007, mask2d=("neighborhood", 56, 5)),
     ]
 }
 
