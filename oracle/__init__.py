@@ -15,6 +15,8 @@ Contents
 ``probabilities``        the materialised probability matrix P (numpy fp64), for
                          the row-sum invariant.
 ``attention_loops``      pure-Python loops for tiny inputs (brute force).
+``attention_bwd``        the gradients dQ, dK, dV of the definition for a given dO, in
+                         plain C, fp64 (``attn_oracle_bwd.c``).
 
 Sources: "FlashAttention technical analysis" (jsqmd.com/news/722897) section 2.1
 (the three steps), section 2.2 (tiling plus online softmax with running max and
@@ -37,21 +39,30 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "attn_oracle.c")
+_SRC_BWD = os.path.join(_HERE, "attn_oracle_bwd.c")
 _LIB_DIR = os.path.join(_HERE, "_build")
 _LIB = os.path.join(_LIB_DIR, "liboracle.so")
+_LIB_BWD = os.path.join(_LIB_DIR, "liboracle_bwd.so")
 _lock = threading.Lock()
 _lib = None
+_lib_bwd = None
+
+
+def _gcc(src: str, out: str, force: bool):
+    if force or not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(src):
+        tmp = out + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math",
+             "-ffp-contract=off", "-o", tmp, src, "-lm", "-lpthread"])
+        os.replace(tmp, out)
 
 
 def build(force: bool = False) -> str:
-    """Compile ``attn_oracle.c`` into ``_build/liboracle.so`` with gcc (no fast-math)."""
+    """Compile ``attn_oracle.c`` and ``attn_oracle_bwd.c`` into ``_build/`` with gcc
+    (no fast-math, no contraction)."""
     os.makedirs(_LIB_DIR, exist_ok=True)
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        tmp = _LIB + f".tmp{os.getpid()}"
-        subprocess.check_call(
-            ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math",
-             "-ffp-contract=off", "-o", tmp, _SRC, "-lm", "-lpthread"])
-        os.replace(tmp, _LIB)
+    _gcc(_SRC, _LIB, force)
+    _gcc(_SRC_BWD, _LIB_BWD, force)
     return _LIB
 
 
@@ -84,6 +95,69 @@ def _load():
         if _lib is None:
             _lib = _bind(build())
     return _lib
+
+
+def _bind_bwd(path):
+    lib = ctypes.CDLL(path)
+    dp = ctypes.POINTER(ctypes.c_double)
+    ip = ctypes.POINTER(ctypes.c_int32)
+    lib.oracle_attention_bwd.restype = ctypes.c_int
+    lib.oracle_attention_bwd.argtypes = [
+        dp, dp, dp, dp, dp, dp, dp,
+        ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+        ctypes.c_double, ctypes.c_int, ip, ip, ctypes.c_int, ctypes.c_int]
+    return lib
+
+
+def _load_bwd():
+    global _lib_bwd
+    with _lock:
+        if _lib_bwd is None:
+            build()
+            _lib_bwd = _bind_bwd(_LIB_BWD)
+    return _lib_bwd
+
+
+def source_text_bwd() -> str:
+    with open(_SRC_BWD) as f:
+        return f.read()
+
+
+def compile_variant_bwd(src_text: str, out_path: str):
+    """Compile a modified copy of the backward oracle (mutant tests only)."""
+    c_path = out_path + ".c"
+    with open(c_path, "w") as f:
+        f.write(src_text)
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math",
+                           "-ffp-contract=off", "-o", out_path, c_path, "-lm", "-lpthread"])
+    return _bind_bwd(out_path)
+
+
+def attention_bwd(q, k, v, dout, *, scale: float | None = None, is_causal: bool = False, key_lens=None,
+                  units=None, n_threads: int = 0, lib=None):
+    """Gradients of the definition for the upstream gradient ``dout`` (fp64).
+
+    q, dout: [B, Hq, Nq, d]; k, v: [B, Hkv, Nk, d]; key_lens: [B] or None;
+    units: optional list of b * Hkv + hkv pairs to compute (others are NaN).
+    Returns (dQ [B, Hq, Nq, d], dK [B, Hkv, Nk, d], dV [B, Hkv, Nk, d]).
+    """
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, Hq, Nq, d = q.shape
+    _, Hkv, Nk, _ = k.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = np.full(q.shape, np.nan)
+    dk = np.full(k.shape, np.nan)
+    dv = np.full(v.shape, np.nan)
+    kl = None if key_lens is None else np.ascontiguousarray(np.asarray(key_lens, dtype=np.int32))
+    un = None if units is None else np.ascontiguousarray(np.asarray(units, dtype=np.int32))
+    rc = (lib or _load_bwd()).oracle_attention_bwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv),
+        B, Hq, Hkv, Nq, Nk, d, float(scale), int(bool(is_causal)),
+        _ptr(kl, ctypes.c_int32), _ptr(un, ctypes.c_int32), 0 if un is None else len(un), int(n_threads))
+    if rc != 0:
+        raise ValueError(f"oracle_attention_bwd rejected its arguments (status {rc})")
+    return dq, dk, dv
 
 
 def compile_variant(src_text: str, out_path: str):
