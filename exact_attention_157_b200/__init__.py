@@ -38,7 +38,7 @@ ATTN_ERR_SCRATCH = 7
 NOALLOC_SCRATCH_BYTES = 16 << 20  # ATTN_NOALLOC_SCRATCH_BYTES
 
 # Every symbol include/attn.h declares.
-EXPORTED = ("attn_fwd", "attn_fwd_mod", "attn_splitkv_plan", "attn_fwd_splitkv", "attn_fwd_splitkv_noalloc",
+EXPORTED = ("attn_fwd", "attn_fwd_mod", "attn_bwd_plan", "attn_bwd", "attn_splitkv_plan", "attn_fwd_splitkv", "attn_fwd_splitkv_noalloc",
             "attn_check_device_status", "attn_set_wait_timeout_ns", "attn_selftest_timeout",
             "attn_status_string", "attn_last_cuda_error", "attn_version")
 
@@ -89,6 +89,11 @@ def lib() -> ctypes.CDLL:
             L.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, vp, vp, vp]
             L.attn_fwd_mod.restype = i
             L.attn_fwd_mod.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, ctypes.POINTER(AttnScoreMod), vp]
+            L.attn_bwd_plan.restype = i
+            L.attn_bwd_plan.argtypes = [i, i, i, ctypes.POINTER(ctypes.c_size_t)]
+            L.attn_bwd.restype = i
+            L.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, vp,
+                                   ctypes.c_size_t, vp]
             L.attn_splitkv_plan.restype = i
             L.attn_splitkv_plan.argtypes = [i, i, i, i, i, i, i, ctypes.POINTER(i), ctypes.POINTER(ctypes.c_size_t)]
             L.attn_fwd_splitkv.restype = i
@@ -143,6 +148,21 @@ def attn_fwd_mod(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, is_causal, key
     return int(lib().attn_fwd_mod(q, k, v, out, lse, int(B), int(Hq), int(Hkv), int(Nq), int(Nk), int(d),
                                   float(scale), int(bool(is_causal)), key_lens,
                                   None if mod is None else ctypes.byref(mod), stream))
+
+
+def attn_bwd_plan(B, Hq, Nq):
+    """The C planner of the backward pass: returns (status, workspace bytes)."""
+    nb = ctypes.c_size_t(0)
+    st = int(lib().attn_bwd_plan(int(B), int(Hq), int(Nq), ctypes.byref(nb)))
+    return st, int(nb.value)
+
+
+def attn_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale, is_causal,
+             key_lens=None, workspace=None, workspace_bytes=0, stream=None) -> int:
+    """The C backward entry point with raw device pointers (ints); returns the status code."""
+    return int(lib().attn_bwd(q, k, v, out, lse, dout, dq, dk, dv, int(B), int(Hq), int(Hkv), int(Nq), int(Nk),
+                              int(d), float(scale), int(bool(is_causal)), key_lens, workspace,
+                              int(workspace_bytes), stream))
 
 
 def attn_splitkv_plan(B, Hq, Nq, Nk, d, n_splits=0, sm_count=0):
@@ -293,6 +313,39 @@ def attention(q, k, v, *, scale: float | None = None, is_causal: bool = False, k
     if st != ATTN_OK:
         raise AttnError(st, "attn_fwd_splitkv")
     return out, lse
+
+
+def attention_backward(q, k, v, out, lse, dout, *, scale: float | None = None, is_causal: bool = False,
+                       key_lens=None, workspace=None, stream=None):
+    """dQ, dK, dV of ``attention`` for the upstream gradient ``dout`` (bf16 CUDA
+    tensors shaped like q / k / v); ``out`` and ``lse`` are the forward results
+    for the same inputs.  Returns (dq, dk, dv)."""
+    import torch
+    for name, t, nd in (("q", q, 4), ("k", k, 4), ("v", v, 4), ("out", out, 4), ("dout", dout, 4)):
+        _check_bf16_cuda(name, t, nd)
+    B, Hq, Nq, d = q.shape
+    _, Hkv, Nk, _ = k.shape
+    if tuple(out.shape) != tuple(q.shape) or tuple(dout.shape) != tuple(q.shape) or tuple(v.shape) != tuple(k.shape):
+        raise ValueError("q / out / dout or k / v shapes disagree")
+    if lse is None or lse.dtype != torch.float32 or tuple(lse.shape) != (B, Hq, Nq) or not lse.is_contiguous():
+        raise ValueError("lse must be the contiguous fp32 [B, Hq, Nq] LSE of the forward pass")
+    st, nbytes = attn_bwd_plan(B, Hq, Nq)
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_bwd_plan")
+    if workspace is None:
+        workspace = torch.empty((nbytes,), dtype=torch.uint8, device=q.device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    kl_ptr = None
+    if key_lens is not None:
+        key_lens = key_lens.contiguous()
+        kl_ptr = key_lens.data_ptr()
+    st = attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), dout.data_ptr(),
+                  dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, Nq, Nk, d,
+                  0.0 if scale is None else float(scale), is_causal, kl_ptr, workspace.data_ptr(),
+                  workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_bwd")
+    return dq, dk, dv
 
 
 def check_device_status(stream=None):

@@ -13,6 +13,7 @@
 #include "attn.h"
 #include "fwd_common.cuh"
 #include "fwd_kernel_pp.cuh"
+#include "bwd_kernels.cuh"
 
 using namespace attn_sm100;
 
@@ -66,6 +67,15 @@ cudaError_t set_pp_attrs() {
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
 }
 
+template <int D>
+cudaError_t set_bwd_attrs() {
+    cudaError_t e = cudaFuncSetAttribute(attn_bwd_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         SmemBwd<D>::kAlloc);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(attn_bwd_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                SmemBwd<D>::kAlloc);
+}
+
 // One-time per-device set-up: architecture check, SM count, kernel attributes,
 // and the driver's tensor-map encoder.
 attn_status_t device_setup(int* dev_out) {
@@ -98,6 +108,8 @@ attn_status_t device_setup(int* dev_out) {
     if ((e = set_pp_attrs<128, kSlots128, kQStages128, true>()) != cudaSuccess) return cuda_fail(e);
     if ((e = set_pp_attrs<64, kSlots64, kQStages64, false>()) != cudaSuccess) return cuda_fail(e);
     if ((e = set_pp_attrs<64, kSlots64, kQStages64, true>()) != cudaSuccess) return cuda_fail(e);
+    if ((e = set_bwd_attrs<128>()) != cudaSuccess) return cuda_fail(e);
+    if ((e = set_bwd_attrs<64>()) != cudaSuccess) return cuda_fail(e);
     st.ready = true;
     st.status = ATTN_OK;
     return ATTN_OK;
@@ -424,6 +436,91 @@ int attn_last_cuda_error(void) { return g_last_cuda_error.load(); }
 int attn_version(void) { return kVersion; }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------
+// Backward pass.
+namespace {
+
+constexpr int kBwdRowPad = 128;
+
+size_t bwd_bytes(int B, int Hq, int Nq) {
+    const long long nq_pad = (static_cast<long long>(Nq) + kBwdRowPad - 1) / kBwdRowPad * kBwdRowPad;
+    return 2 * round_up(static_cast<size_t>(B) * Hq * nq_pad * sizeof(float), kWsAlign);
+}
+
+template <int D>
+cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
+                       const BwdParams& p, cudaStream_t s) {
+    const long long rows = static_cast<long long>(p.B) * p.Hq * p.nq_pad;
+    attn_bwd_prep_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, s>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const dim3 g_kv((p.Nk + kBN - 1) / kBN, p.B * p.Hkv);
+    attn_bwd_kernel<D, true><<<g_kv, kBwdThreads, SmemBwd<D>::kAlloc, s>>>(tq, tk, tv, tdo, p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const dim3 g_q((p.Nq + kBM - 1) / kBM, p.B * p.Hq);
+    attn_bwd_kernel<D, false><<<g_q, kBwdThreads, SmemBwd<D>::kAlloc, s>>>(tq, tk, tv, tdo, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+extern "C" attn_status_t attn_bwd_plan(int B, int Hq, int Nq, size_t* workspace_bytes) {
+    if (B <= 0 || Hq <= 0 || Nq <= 0 || workspace_bytes == nullptr) return ATTN_ERR_INVALID_ARG;
+    *workspace_bytes = bwd_bytes(B, Hq, Nq);
+    return ATTN_OK;
+}
+
+extern "C" attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                                  const void* dout, void* dq, void* dk, void* dv,
+                                  int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                                  float scale, int is_causal, const int32_t* key_lens,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+    if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || lse == nullptr || dout == nullptr ||
+        dq == nullptr || dk == nullptr || dv == nullptr || workspace == nullptr)
+        return ATTN_ERR_INVALID_ARG;
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nk <= 0 || d <= 0 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+    if (!(std::isfinite(scale)) || scale < 0.0f) return ATTN_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) || !aligned16(dq) ||
+        !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(lse) & 3u) ||
+        (key_lens != nullptr && (reinterpret_cast<uintptr_t>(key_lens) & 3u)) ||
+        reinterpret_cast<uintptr_t>(workspace) % kWsAlign != 0)
+        return ATTN_ERR_ALIGNMENT;
+    if (workspace_bytes < bwd_bytes(B, Hq, Nq)) return ATTN_ERR_INVALID_ARG;
+    int dev = 0;
+    attn_status_t st = device_setup(&dev);
+    if (st != ATTN_OK) return st;
+
+    const float scale_eff = scale == 0.0f ? static_cast<float>(1.0 / std::sqrt(static_cast<double>(d))) : scale;
+    BwdParams p;
+    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Nq = Nq; p.Nk = Nk; p.group = Hq / Hkv;
+    p.nq_pad = (Nq + kBwdRowPad - 1) / kBwdRowPad * kBwdRowPad;
+    p.scale_log2 = static_cast<float>(static_cast<double>(scale_eff) * 1.4426950408889634);
+    p.scale = scale_eff;
+    p.is_causal = is_causal ? 1 : 0;
+    p.key_lens = key_lens;
+    p.lse = lse;
+    p.o = static_cast<const uint16_t*>(out);
+    p.dout = static_cast<const uint16_t*>(dout);
+    p.delta = static_cast<float*>(workspace);
+    p.lse2 = reinterpret_cast<float*>(static_cast<char*>(workspace) + bwd_bytes(B, Hq, Nq) / 2);
+    p.dq = static_cast<uint16_t*>(dq);
+    p.dk = static_cast<uint16_t*>(dk);
+    p.dv = static_cast<uint16_t*>(dv);
+    p.timeout_ns = g_timeout_ns.load();
+    p.epoch = next_epoch();
+
+    CUtensorMap tq, tk, tv, tdo;
+    if ((st = encode_map(&tq, q, d, Nq, static_cast<long long>(B) * Hq)) != ATTN_OK) return st;
+    if ((st = encode_map(&tk, k, d, Nk, static_cast<long long>(B) * Hkv)) != ATTN_OK) return st;
+    if ((st = encode_map(&tv, v, d, Nk, static_cast<long long>(B) * Hkv)) != ATTN_OK) return st;
+    if ((st = encode_map(&tdo, dout, d, Nq, static_cast<long long>(B) * Hq)) != ATTN_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const cudaError_t e = d == 128 ? launch_bwd<128>(tq, tk, tv, tdo, p, s) : launch_bwd<64>(tq, tk, tv, tdo, p, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return ATTN_OK;
+}
 
 // ------------------------------------------------------------------------
 // Split-KV without caller memory: the workspace lives in a fixed device array

@@ -1,0 +1,426 @@
+// bwd_kernels.cuh -- backward pass of exact attention for sm_100a.
+//
+// "FlashAttention technical analysis" (jsqmd.com/news/722897), section 3.3:
+// the forward pass keeps only O(N) statistics per row (here the LSE); the
+// backward pass recomputes each block of P from Q, K and those statistics
+// instead of reading a stored N x N matrix.  With S = scale * Q K^T,
+// P = exp(S - LSE), D_i = sum_t dO_it O_it:
+//
+//   dV = P^T dO,   dP = dO V^T,   dS = P o (dP - D),   dQ = scale dS K,   dK = scale dS^T Q
+//
+// Three launches:
+//   attn_bwd_prep_kernel         D and LSE * log2(e) per query row (HBM-bound, a warp per row)
+//   attn_bwd_kernel<D, true>     dK, dV: one CTA per 128-key block of one K/V head, looping
+//                                over the query blocks of every query head of its group (K/V
+//                                blocks in the outer loop, section 4.1 of the same page);
+//                                S^T = K Q^T and dP^T = V dO^T on the tensor cores, P^T and
+//                                dS^T written back to TMEM as bf16, then dV += P^T dO and
+//                                dK += dS^T Q accumulate in TMEM
+//   attn_bwd_kernel<D, false>    dQ: one CTA per 128-row query block, looping over key
+//                                blocks; S = Q K^T, dP = dO V^T, dS to TMEM, dQ += dS K
+// Splitting dQ from dK/dV keeps every accumulator in one CTA's TMEM: no atomics.
+//
+// Warps (192 threads): 0-3 elementwise (thread = TMEM lane = row), 4 TMA producer,
+// 5 TMEM owner and MMA issuer (warp-uniform, elect.sync).  Every wait is bounded.
+#pragma once
+
+#include "fwd_common.cuh"
+
+namespace attn_sm100 {
+
+struct BwdParams {
+    int B, Hq, Hkv, Nq, Nk, group;
+    int nq_pad;          // row stride of the per-head D / LSE2 workspace (multiple of 128)
+    float scale_log2;    // scale * log2(e)
+    float scale;         // multiplies dQ and dK
+    int is_causal;
+    const int32_t* key_lens;
+    const float* lse;    // forward LSE [B*Hq*Nq] (natural log)
+    const uint16_t* o;   // forward O, bf16 [B*Hq*Nq*d]
+    const uint16_t* dout;
+    float* delta;        // workspace: D [B*Hq][nq_pad]
+    float* lse2;         // workspace: LSE * log2(e); +inf for rows without keys and padding rows
+    uint16_t* dq;        // bf16 [B*Hq*Nq*d]
+    uint16_t* dk;        // bf16 [B*Hkv*Nk*d]
+    uint16_t* dv;
+    unsigned long long timeout_ns;
+    unsigned int epoch;
+};
+
+constexpr int kBwdThreads = 192;
+enum : unsigned int { kRoleBwdElem = 4, kRoleBwdProducer = 5, kRoleBwdMma = 6, kRoleBwdPrep = 7 };
+
+// D_i = sum_t dO_it O_it and LSE2_i, one warp per (head, padded row).
+template <int D>
+__global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const BwdParams p) {
+    const long long r = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    const long long total = static_cast<long long>(p.B) * p.Hq * p.nq_pad;
+    if (r >= total) return;
+    const long long bh = r / p.nq_pad;
+    const int i = static_cast<int>(r - bh * p.nq_pad);
+    if (i >= p.Nq) {
+        if (lane == 0) {
+            p.delta[r] = 0.0f;
+            p.lse2[r] = INFINITY;
+        }
+        return;
+    }
+    const long long row = bh * p.Nq + i;
+    constexpr int kPer = D / 32;  // bf16 per lane
+    const uint16_t* o = p.o + row * D + lane * kPer;
+    const uint16_t* g = p.dout + row * D + lane * kPer;
+    float acc = 0.0f;
+    #pragma unroll
+    for (int e = 0; e < kPer; e += 2) {
+        const uint32_t ov = *reinterpret_cast<const uint32_t*>(o + e);
+        const uint32_t gv = *reinterpret_cast<const uint32_t*>(g + e);
+        acc = fmaf(__uint_as_float(ov << 16), __uint_as_float(gv << 16), acc);
+        acc = fmaf(__uint_as_float(ov & 0xffff0000u), __uint_as_float(gv & 0xffff0000u), acc);
+    }
+    #pragma unroll
+    for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+    if (lane == 0) {
+        const float l = p.lse[row];
+        p.delta[r] = acc;
+        p.lse2[r] = (l == -INFINITY) ? INFINITY : l * kLog2e;
+    }
+}
+
+template <int D>
+struct SmemBwd {
+    static constexpr int kChunks = D / 64;
+    static constexpr int kChunkBytes = 128 * 128;
+    static constexpr int kTile = kChunks * kChunkBytes;  // 128 rows x D bf16, 128-byte swizzle
+    // dK/dV kernel: K, V, then 2 stages of (Q, dO).  dQ kernel: Q, dO, then 2 stages of (K, V).
+    static constexpr int kFixed0 = 0, kFixed1 = kTile;
+    static constexpr int kStage = 2 * kTile;
+    static constexpr int kStages = 2 * kTile;
+    static constexpr int kBars = kStages + 2 * kStage;
+    // barriers
+    static constexpr int FIXFULL = 0, STFULL_ = 1, PFULL = 2, DONE = 3, RFULL = 4, REMPTY = 6;
+    static constexpr int kNumBars = 8;
+    static constexpr int kMisc = kBars + 8 * kNumBars;
+    static constexpr int kBytes = kMisc + 16;
+    static constexpr int kAlloc = kBytes + 1024;
+    static constexpr int kColA = 0, kColB = 128, kColAcc0 = 256, kColAcc1 = 256 + D;
+    static_assert(kColAcc1 + D <= kTmemCols, "TMEM budget");
+    static_assert(kAlloc <= 232448, "shared memory budget");
+};
+
+// Writes one row of `D` fp32 TMEM columns, times `mul`, as bf16 to global `dst`
+// (or zeros when `zero`), 32 columns per TMEM load.
+template <int D>
+__device__ __forceinline__ void store_row_bf16(uint32_t taddr, uint16_t* dst, float mul, bool zero, bool write) {
+    #pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[32];
+        if (!zero) {
+            tmem_ld32(taddr + c * 32, v);
+            tmem_wait_ld();
+        }
+        uint32_t w[16];
+        #pragma unroll
+        for (int e = 0; e < 16; ++e)
+            w[e] = zero ? 0u : pack_bf16x2(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
+        if (write) {
+            uint4* out = reinterpret_cast<uint4*>(dst + c * 32);
+            #pragma unroll
+            for (int e = 0; e < 4; ++e) out[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+        }
+    }
+}
+
+// Shared structure of the two main kernels.  DKDV = true: rows of the TMEM
+// tiles are keys, the fixed operands are K and V of one 128-key block, the
+// streamed stages hold Q and dO of one query block.  DKDV = false: rows are
+// queries, fixed Q and dO, streamed K and V.
+template <int D, bool DKDV>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                const BwdParams p) {
+    using L = SmemBwd<D>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t raw_base = smem_u32(smem_raw);
+    const uint32_t sbase = (raw_base + 1023u) & ~1023u;
+    uint8_t* smem = smem_raw + (sbase - raw_base);
+    auto bar = [&](int i) -> uint32_t { return sbase + L::kBars + 8u * i; };
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint64_t limit = p.timeout_ns;
+
+    // ---- the CTA's block and its loop
+    const int blk = blockIdx.x;  // key block (DKDV) or query block
+    int b, hk, h0;               // batch, K/V head, first query head
+    int bh_fixed;                // z of the fixed operands' maps
+    if constexpr (DKDV) {
+        b = blockIdx.y / p.Hkv;
+        hk = blockIdx.y - b * p.Hkv;
+        h0 = hk * p.group;
+        bh_fixed = blockIdx.y;  // b * Hkv + hk
+    } else {
+        b = blockIdx.y / p.Hq;
+        h0 = blockIdx.y - b * p.Hq;
+        hk = h0 / p.group;
+        bh_fixed = blockIdx.y;  // b * Hq + h
+    }
+    int kv_len = p.key_lens != nullptr ? __ldg(p.key_lens + b) : p.Nk;
+    if (kv_len < 0 || kv_len > p.Nk) {
+        if (threadIdx.x == 0) record_error(kErrDevice, kRoleBwdElem, 1);
+        kv_len = kv_len < 0 ? 0 : p.Nk;
+    }
+    const int n_qblk = (p.Nq + kBM - 1) / kBM;
+    int n_iter, first;  // iterations: (query head, query block) pairs or key blocks
+    if constexpr (DKDV) {
+        first = p.is_causal ? blk : 0;  // query blocks that can see a key of this block
+        const int per_head = blk * kBN < kv_len && first < n_qblk ? n_qblk - first : 0;
+        n_iter = per_head * p.group;
+    } else {
+        int end = kv_len;
+        if (p.is_causal && (blk + 1) * kBM < end) end = (blk + 1) * kBM;
+        first = 0;
+        n_iter = (end + kBN - 1) / kBN;
+    }
+    const int per_head = DKDV ? (n_qblk - first) : 1;
+    auto iter_head = [&](int it) { return DKDV ? h0 + it / per_head : h0; };
+    auto iter_blk = [&](int it) { return DKDV ? first + it % per_head : it; };
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(L::FIXFULL), 1);
+        mbar_init(bar(L::STFULL_), 1);
+        mbar_init(bar(L::PFULL), 128);
+        mbar_init(bar(L::DONE), 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar(L::RFULL + s), 1);
+            mbar_init(bar(L::REMPTY + s), 1);
+        }
+        *abort_flag = launch_aborted(p.epoch) ? 1 : 0;
+        fence_mbar_init();
+    }
+    if (warp == 5) {
+        tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+        tmem_relinquish();
+    }
+    if (warp == 4 && lane == 0) {
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+        prefetch_tmap(&tm_do);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 4) {
+        // =============================== TMA producer ===============================
+        if (lane == 0 && n_iter > 0 && !*abort_flag) {
+            bool ok = true;
+            int loads[2] = {0, 0};  // stage loads issued (RFULL phases)
+            const uint32_t f0 = sbase + L::kFixed0, f1 = sbase + L::kFixed1;
+            mbar_arrive_expect_tx(bar(L::FIXFULL), 2 * L::kTile);
+            #pragma unroll
+            for (int c = 0; c < L::kChunks; ++c) {
+                if constexpr (DKDV) {
+                    tma_load_3d(f0 + c * L::kChunkBytes, &tm_k, bar(L::FIXFULL), c * 64, blk * kBN, bh_fixed);
+                    tma_load_3d(f1 + c * L::kChunkBytes, &tm_v, bar(L::FIXFULL), c * 64, blk * kBN, bh_fixed);
+                } else {
+                    tma_load_3d(f0 + c * L::kChunkBytes, &tm_q, bar(L::FIXFULL), c * 64, blk * kBM, bh_fixed);
+                    tma_load_3d(f1 + c * L::kChunkBytes, &tm_do, bar(L::FIXFULL), c * 64, blk * kBM, bh_fixed);
+                }
+            }
+            for (int it = 0; ok && it < n_iter; ++it) {
+                const int s = it & 1;
+                if (it >= 2 &&
+                    !mbar_wait(bar(L::REMPTY + s), ((it >> 1) - 1) & 1, limit, abort_flag, p.epoch, kRoleBwdProducer, 1))
+                    { ok = false; break; }
+                const uint32_t st0 = sbase + L::kStages + s * L::kStage, st1 = st0 + L::kTile;
+                const int ib = iter_blk(it);
+                mbar_arrive_expect_tx(bar(L::RFULL + s), 2 * L::kTile);
+                ++loads[s];
+                #pragma unroll
+                for (int c = 0; c < L::kChunks; ++c) {
+                    if constexpr (DKDV) {
+                        const int z = b * p.Hq + iter_head(it);
+                        tma_load_3d(st0 + c * L::kChunkBytes, &tm_q, bar(L::RFULL + s), c * 64, ib * kBM, z);
+                        tma_load_3d(st1 + c * L::kChunkBytes, &tm_do, bar(L::RFULL + s), c * 64, ib * kBM, z);
+                    } else {
+                        const int z = b * p.Hkv + hk;
+                        tma_load_3d(st0 + c * L::kChunkBytes, &tm_k, bar(L::RFULL + s), c * 64, ib * kBN, z);
+                        tma_load_3d(st1 + c * L::kChunkBytes, &tm_v, bar(L::RFULL + s), c * 64, ib * kBN, z);
+                    }
+                }
+            }
+            // every load issued has landed before the CTA may exit
+            mbar_drain(bar(L::FIXFULL), 0, kRoleBwdProducer, 2);
+            for (int s = 0; s < 2; ++s)
+                if (loads[s] > 0) mbar_drain(bar(L::RFULL + s), (loads[s] - 1) & 1, kRoleBwdProducer, 3);
+        }
+    } else if (warp == 5) {
+        // ================================ MMA issuer ================================
+        constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, false);
+        constexpr uint32_t kIdescAcc = idesc_bf16_f32(128, D, true);
+        bool ok = n_iter > 0 && !*abort_flag;
+        if (ok) ok = mbar_wait_warp(bar(L::FIXFULL), 0, limit, abort_flag, p.epoch, kRoleBwdMma, 1);
+        const uint32_t f0 = sbase + L::kFixed0, f1 = sbase + L::kFixed1;
+        for (int it = 0; ok && it < n_iter; ++it) {
+            const int s = it & 1;
+            const uint32_t st0 = sbase + L::kStages + s * L::kStage, st1 = st0 + L::kTile;
+            if (!mbar_wait_warp(bar(L::RFULL + s), (it >> 1) & 1, limit, abort_flag, p.epoch, kRoleBwdMma, 2))
+                { ok = false; break; }
+            tc_fence_after();
+            // DKDV: S^T = K Q^T, dP^T = V dO^T.  dQ: S = Q K^T, dP = dO V^T.
+            // A = fixed (f0 / f1), B = streamed (st0 / st1), both K-major over d.
+            #pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
+                mma_ss_warp(tmem + L::kColA, smem_desc_sw128(f0 + off, 16, 1024), smem_desc_sw128(st0 + off, 16, 1024),
+                            kIdescS, kk > 0 ? 1u : 0u);
+            }
+            #pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
+                mma_ss_warp(tmem + L::kColB, smem_desc_sw128(f1 + off, 16, 1024), smem_desc_sw128(st1 + off, 16, 1024),
+                            kIdescS, kk > 0 ? 1u : 0u);
+            }
+            mma_commit_warp(bar(L::STFULL_));
+            if (!mbar_wait_warp(bar(L::PFULL), it & 1, limit, abort_flag, p.epoch, kRoleBwdMma, 3)) { ok = false; break; }
+            tc_fence_after();
+            // bf16 operands in TMEM (A) times a streamed tile as B (MN-major, 16 rows per step):
+            // DKDV: dV += P^T dO (P^T in kColA), dK += dS^T Q (dS^T in kColB).
+            // dQ:   dQ += dS K (dS in kColA).
+            #pragma unroll
+            for (int kk = 0; kk < kBN / 16; ++kk) {
+                const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
+                if constexpr (DKDV) {
+                    mma_ts_warp(tmem + L::kColAcc0, tmem + L::kColA + kk * 8,
+                                smem_desc_sw128(st1 + kk * 2048, L::kChunkBytes, 1024), kIdescAcc, acc);
+                    mma_ts_warp(tmem + L::kColAcc1, tmem + L::kColB + kk * 8,
+                                smem_desc_sw128(st0 + kk * 2048, L::kChunkBytes, 1024), kIdescAcc, acc);
+                } else {
+                    mma_ts_warp(tmem + L::kColAcc0, tmem + L::kColA + kk * 8,
+                                smem_desc_sw128(st0 + kk * 2048, L::kChunkBytes, 1024), kIdescAcc, acc);
+                }
+            }
+            mma_commit_warp(bar(L::REMPTY + s));  // the stage may be refilled once these complete
+        }
+        mma_commit_warp(bar(L::DONE));
+        mbar_drain(bar(L::DONE), 0, kRoleBwdMma, 4);
+    } else {
+        // ============================ elementwise warps =============================
+        const int row = warp * 32 + lane;  // TMEM lane
+        const uint32_t lane_tmem = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+        const float c2 = p.scale_log2;
+        // per-row constants of the dQ kernel (rows are queries)
+        const int q_row = DKDV ? 0 : blk * kBM + row;
+        float my_lse2 = 0.0f, my_d = 0.0f;
+        if constexpr (!DKDV) {
+            const long long r = static_cast<long long>(blockIdx.y) * p.nq_pad + q_row;
+            my_lse2 = p.lse2[r];
+            my_d = p.delta[r];
+        }
+        const int key_row = DKDV ? blk * kBN + row : 0;
+        bool ok = !*abort_flag;
+        for (int it = 0; ok && it < n_iter; ++it) {
+            const int ib = iter_blk(it);
+            // DKDV: LSE2 and D of this iteration's 128 queries (the same addresses in every
+            // lane: broadcast loads; rows are padded to 128, so 16-byte aligned)
+            const float* l2row = nullptr;
+            const float* ddrow = nullptr;
+            if constexpr (DKDV) {
+                const long long r = static_cast<long long>(b * p.Hq + iter_head(it)) * p.nq_pad + ib * kBM;
+                l2row = p.lse2 + r;
+                ddrow = p.delta + r;
+            }
+            const bool got = mbar_wait(bar(L::STFULL_), it & 1, limit, abort_flag, p.epoch, kRoleBwdElem, 2);
+            if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+            tc_fence_after();
+            #pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t sv[32], dv[32];
+                tmem_ld32(lane_tmem + L::kColA + c * 32, sv);
+                tmem_ld32(lane_tmem + L::kColB + c * 32, dv);
+                tmem_wait_ld();
+                float l2c[32], ddc[32];
+                if constexpr (DKDV) {
+                    #pragma unroll
+                    for (int v = 0; v < 8; ++v) {
+                        const float4 a = __ldg(reinterpret_cast<const float4*>(l2row + c * 32) + v);
+                        const float4 z = __ldg(reinterpret_cast<const float4*>(ddrow + c * 32) + v);
+                        l2c[4 * v] = a.x; l2c[4 * v + 1] = a.y; l2c[4 * v + 2] = a.z; l2c[4 * v + 3] = a.w;
+                        ddc[4 * v] = z.x; ddc[4 * v + 1] = z.y; ddc[4 * v + 2] = z.z; ddc[4 * v + 3] = z.w;
+                    }
+                }
+                uint32_t pw[16], dw[16];
+                #pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    float pp[2], ds[2];
+                    #pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int col = c * 32 + e + u;  // query (DKDV) or key (dQ) within the block
+                        float l2, dd;
+                        bool vis;
+                        if constexpr (DKDV) {
+                            const int qi = ib * kBM + col;
+                            l2 = l2c[e + u];
+                            dd = ddc[e + u];
+                            vis = key_row < kv_len && (!p.is_causal || key_row <= qi);
+                        } else {
+                            const int kj = ib * kBN + col;
+                            l2 = my_lse2;
+                            dd = my_d;
+                            vis = kj < kv_len && (!p.is_causal || kj <= q_row);
+                        }
+                        const float pv = vis ? ex2_approx(fmaf(__uint_as_float(sv[e + u]), c2, -l2)) : 0.0f;
+                        pp[u] = pv;
+                        ds[u] = pv * (__uint_as_float(dv[e + u]) - dd);
+                    }
+                    pw[e / 2] = pack_bf16x2(pp[0], pp[1]);
+                    dw[e / 2] = pack_bf16x2(ds[0], ds[1]);
+                }
+                if constexpr (DKDV) {
+                    tmem_st16(lane_tmem + L::kColA + c * 16, pw);  // P^T over S^T columns already read
+                    tmem_st16(lane_tmem + L::kColB + c * 16, dw);  // dS^T over dP^T columns already read
+                } else {
+                    tmem_st16(lane_tmem + L::kColA + c * 16, dw);  // dS over S columns already read
+                }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(L::PFULL));
+        }
+        // ------------------------------------------------------------- epilogue
+        bool have = n_iter > 0 && ok;
+        if (have) {
+            const bool got = mbar_wait(bar(L::DONE), 0, limit, abort_flag, p.epoch, kRoleBwdElem, 3);
+            have = __all_sync(0xffffffffu, got);
+            tc_fence_after();
+        }
+        const bool failed = n_iter > 0 && !have;
+        if (!failed) {
+            if constexpr (DKDV) {
+                const bool write = key_row < p.Nk;
+                const long long base = (static_cast<long long>(b * p.Hkv + hk) * p.Nk + key_row) * D;
+                store_row_bf16<D>(lane_tmem + L::kColAcc0, p.dv + base, 1.0f, n_iter == 0, write);
+                store_row_bf16<D>(lane_tmem + L::kColAcc1, p.dk + base, p.scale, n_iter == 0, write);
+            } else {
+                const bool write = q_row < p.Nq;
+                const long long base = (static_cast<long long>(blockIdx.y) * p.Nq + q_row) * D;
+                store_row_bf16<D>(lane_tmem + L::kColAcc0, p.dq + base, p.scale, n_iter == 0, write);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace attn_sm100

@@ -1,7 +1,8 @@
 /*
- * attn.h -- C ABI of the B200 (sm_100a) exact attention forward library.
+ * attn.h -- C ABI of the B200 (sm_100a) exact attention library.
  *
- * The operation is exact scaled-dot-product attention, forward only:
+ * The operation is exact scaled-dot-product attention (the forward pass, and
+ * its gradients in attn_bwd):
  *
  *     O = softmax(scale * Q K^T + mask) V,     LSE = logsumexp(scale * Q K^T + mask)
  *
@@ -224,6 +225,42 @@ attn_status_t attn_fwd_splitkv_noalloc(const void *q, const void *k, const void 
                                        const int32_t *key_lens,
                                        const float *additive_mask, const int64_t *mask_strides,
                                        int n_splits, void *stream);
+
+/*
+ * attn_bwd_plan -- device workspace bytes attn_bwd needs (host-only).  The
+ * workspace holds two fp32 values per query row (D = rowsum(dO * O) and the
+ * base-2 LSE), rows padded to a multiple of 128 per head.
+ * Errors: ATTN_ERR_INVALID_ARG for non-positive sizes or a NULL output.
+ */
+attn_status_t attn_bwd_plan(int B, int Hq, int Nq, size_t *workspace_bytes);
+
+/*
+ * attn_bwd -- gradients of attn_fwd: given the forward inputs, its outputs O
+ * and LSE, and dO = dLoss/dO, writes dQ, dK, dV.
+ *
+ * "FlashAttention technical analysis" (jsqmd.com/news/722897), section 3.3:
+ * the forward keeps only per-row statistics; the backward recomputes each
+ * block of P = exp(scale * Q K^T - LSE) and never stores an N x N matrix.
+ * dV = P^T dO, dS = P o (dO V^T - D) with D_i = sum_t dO_it O_it,
+ * dQ = scale dS K, dK = scale dS^T Q.  Grouped heads: dK and dV of a K/V head
+ * sum the contributions of all query heads that read it.
+ *
+ * Layout as attn_fwd, all device, contiguous, 16-byte-aligned bases:
+ *   q, out, dout, dq   bf16 [B, Hq, Nq, d]     (dq written)
+ *   k, v, dk, dv       bf16 [B, Hkv, Nk, d]    (dk, dv written)
+ *   lse                fp32 [B, Hq, Nq], as written by attn_fwd for the same inputs
+ * scale, is_causal, key_lens: as attn_fwd (additive masks are not supported
+ * here).  Rows of dq with no visible key and keys no query sees get 0.
+ * workspace: device, 256-byte aligned, >= attn_bwd_plan bytes; scratch whose
+ * contents need not be initialised; calls in flight at once must not share it.
+ * Three kernels run on `stream` (row statistics, dK/dV, dQ).
+ * Errors: as attn_fwd; ATTN_ERR_INVALID_ARG also for a NULL or short workspace.
+ */
+attn_status_t attn_bwd(const void *q, const void *k, const void *v, const void *out, const float *lse,
+                       const void *dout, void *dq, void *dk, void *dv,
+                       int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                       float scale, int is_causal, const int32_t *key_lens,
+                       void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * attn_check_device_status -- synchronise `stream`, then read and clear the

@@ -170,3 +170,29 @@ def test_score_mod_struct_layout_matches_header():
     names = re.findall(r"\b(?:float|int)\s+(\w+);", body)
     assert names == [f[0] for f in ea.AttnScoreMod._fields_]
     assert ctypes.sizeof(ea.AttnScoreMod) == 20
+
+
+# ------------------------------------------------------------------- backward
+def test_bwd_plan_bytes():
+    st, nb = ea.attn_bwd_plan(2, 4, 300)
+    assert st == ea.ATTN_OK
+    rows = 2 * 4 * 384  # rows padded to a multiple of 128 per head
+    assert nb == 2 * ((rows * 4 + 255) // 256 * 256)
+    assert ea.attn_bwd_plan(0, 4, 300)[0] == ea.ATTN_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("args,status", [
+    (dict(dq=0), ea.ATTN_ERR_INVALID_ARG),
+    (dict(workspace=0), ea.ATTN_ERR_INVALID_ARG),
+    (dict(workspace_bytes=16), ea.ATTN_ERR_INVALID_ARG),
+    (dict(Hq=3, Hkv=2), ea.ATTN_ERR_INVALID_ARG),
+    (dict(d=96), ea.ATTN_ERR_UNSUPPORTED),
+    (dict(dk=A + 8), ea.ATTN_ERR_ALIGNMENT),
+    (dict(workspace=A + 16), ea.ATTN_ERR_ALIGNMENT),
+    (dict(scale=-2.0), ea.ATTN_ERR_INVALID_ARG),
+])
+def test_bwd_validation_is_host_side(args, status):
+    kw = dict(q=A, k=A, v=A, out=A, lse=A, dout=A, dq=A, dk=A, dv=A, B=1, Hq=2, Hkv=2, Nq=64, Nk=64, d=64,
+              scale=0.0, is_causal=0, key_lens=None, workspace=A, workspace_bytes=1 << 20)
+    kw.update(args)
+    assert ea.attn_bwd(**kw) == status
