@@ -249,6 +249,46 @@ def oracle_sample(w, q, k, v, kl, target_s: float, max_rows=None):
     return total, dt, desc, threads
 
 
+def oracle_sample_bwd(w, q, k, v, do, kl, target_s: float):
+    """The fp64 backward oracle on a bounded sample: the first R query rows of
+    the first (batch, K/V head) pairs (every query head of the group), R chosen
+    to fill ~target_s.  Returns (flops, seconds, description, threads)."""
+    import oracle
+    threads = oracle.default_threads()
+    kl_list = None if kl is None else kl.cpu().tolist()
+    G = w.Hq // w.Hkv
+
+    def inputs(b, hk, R):
+        h0 = hk * G
+        cut = lambda t, a, z: t[b:b + 1, a:z].cpu().double().numpy()
+        return (cut(q, h0, h0 + G)[:, :, :R], cut(k, hk, hk + 1), cut(v, hk, hk + 1), cut(do, h0, h0 + G)[:, :, :R],
+                None if kl_list is None else [kl_list[b]])
+
+    def flops_of(b, R):
+        nk = w.Nk if kl_list is None else kl_list[b]
+        return sum(10.0 * w.d * G * (min(nk, i + 1) if w.is_causal else nk) for i in range(R))
+
+    R0 = min(w.Nq, 16)
+    t0 = time.perf_counter()
+    qq, kk, vv, dd, ll = inputs(0, 0, R0)
+    oracle.attention_bwd(qq, kk, vv, dd, is_causal=w.is_causal, key_lens=ll, n_threads=1)
+    per_flop = max(time.perf_counter() - t0, 1e-6) / max(flops_of(0, R0), 1.0)
+    # units run one per thread: give each thread ~target_s of rows
+    n_units = min(threads, w.B * w.Hkv)
+    R = max(1, min(w.Nq, int(R0 * target_s / max(per_flop * flops_of(0, R0), 1e-9))))
+    units = [divmod(u, w.Hkv) for u in range(n_units)]
+    t0 = time.perf_counter()
+    import concurrent.futures as cf
+    with cf.ThreadPoolExecutor(max_workers=n_units) as ex:
+        list(ex.map(lambda bk: oracle.attention_bwd(*inputs(bk[0], bk[1], R)[:4], is_causal=w.is_causal,
+                                                     key_lens=inputs(bk[0], bk[1], 1)[4], n_threads=1), units))
+    dt = time.perf_counter() - t0
+    total = sum(flops_of(b, R) for b, _ in units)
+    desc = (f"backward of the first {R} query rows of {n_units} (batch, K/V head) pairs of the {w.name} "
+            f"workload, every query head of each group, fp64, one pair per thread")
+    return total, dt, desc, n_units
+
+
 # -------------------------------------------------------------- our arm
 def run_ours(args, w):
     import torch
@@ -270,6 +310,16 @@ def run_ours(args, w):
     flops = workload_flops(w)
     in_bytes = q.numel() * 2 + k.numel() * 2 + v.numel() * 2 + (0 if kl is None else kl.numel() * 4)
     out_bytes = out.numel() * 2 + lse.numel() * 4
+    if w.backward:
+        # the forward results and an upstream gradient are inputs of the timed backward step
+        from workloads import make_qkv
+        dout = make_qkv(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, seed=w.seed + 7 * rank + 1, device=dev)[0]
+        ea.attention(q, k, v, is_causal=w.is_causal, key_lens=kl, out=out, lse=lse, stream=stream)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        st, bw_bytes = ea.attn_bwd_plan(w.B, w.Hq, w.Nq)
+        bws = torch.empty((bw_bytes,), dtype=torch.uint8, device=dev)
+        in_bytes += out.numel() * 2 + lse.numel() * 4 + dout.numel() * 2
+        out_bytes = (dq.numel() + dk.numel() + dv.numel()) * 2
     l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = None
     if in_bytes + out_bytes < 2 * l2_bytes:  # small working set: flush L2 between steps
@@ -286,8 +336,15 @@ def run_ours(args, w):
         per_step_launches = 2 if n_used > 1 else 1
 
     def call():
+        if w.backward:
+            ea.attention_backward(q, k, v, out, lse, dout, is_causal=w.is_causal, key_lens=kl, workspace=bws,
+                                  stream=stream, dq=dq, dk=dk, dv=dv)
+            return
         ea.attention(q, k, v, is_causal=w.is_causal, key_lens=kl, out=out, lse=lse, stream=stream,
                      split_kv=split, workspace=ws, softcap=w.softcap, mask2d=w.mask2d)
+
+    if w.backward:
+        per_step_launches = 3  # row statistics, dK / dV, dQ
 
     def step():
         if flush is not None:
@@ -329,23 +386,40 @@ def run_ours(args, w):
     value = flops * world / (ms_per_step * 1e-3) / 1e12
 
     # --- end to end through the public API with pinned host buffers
-    qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
-    klh = None if kl is None else kl.cpu().pin_memory()
-    outh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    lseh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-    runner = ea.HostAttention(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, device=dev, with_key_lens=kl is not None,
-                              split_kv=split)
     e2e_steps = max(1, min(args.steps, 20))
+    if w.backward:
+        host_in = [t.cpu().pin_memory() for t in (q, k, v, out, lse, dout)]
+        host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (dq, dk, dv)]
+        klh = None if kl is None else kl.cpu().pin_memory()
+
+        def e2e_step():
+            with torch.cuda.stream(stream):
+                for dst, src in zip((q, k, v, out, lse, dout), host_in):
+                    dst.copy_(src, non_blocking=True)
+                if klh is not None:
+                    kl.copy_(klh, non_blocking=True)
+                call()
+                for dst, src in zip(host_out, (dq, dk, dv)):
+                    dst.copy_(src, non_blocking=True)
+    else:
+        qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
+        klh = None if kl is None else kl.cpu().pin_memory()
+        outh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        lseh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        runner = ea.HostAttention(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, device=dev, with_key_lens=kl is not None,
+                                  split_kv=split)
+
+        def e2e_step():
+            runner(qh, kh, vh, outh, lseh, klh, is_causal=w.is_causal, stream=stream, softcap=w.softcap,
+                   mask2d=w.mask2d)
     for _ in range(min(args.warmup, 3)):
-        runner(qh, kh, vh, outh, lseh, klh, is_causal=w.is_causal, stream=stream, softcap=w.softcap,
-               mask2d=w.mask2d)
+        e2e_step()
     barrier(world, dev)
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(e2e_steps):
-        runner(qh, kh, vh, outh, lseh, klh, is_causal=w.is_causal, stream=stream, softcap=w.softcap,
-               mask2d=w.mask2d)
+        e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / e2e_steps
@@ -355,6 +429,8 @@ def run_ours(args, w):
     peaks = load_peaks()
     per_launch_flops = flops
     per_launch_bytes = w.qkvo_bytes() + w.lse_bytes()
+    if w.backward:  # read Q, K, V, O, dO, LSE; write dQ, dK, dV
+        per_launch_bytes = 2 * w.qkvo_bytes() + w.lse_bytes()
     t_launch = ms_per_step * 1e-3
     compute_floor = per_launch_flops / (peaks["bf16_tflops"] * 1e12)
     hbm_floor = per_launch_bytes / (peaks["hbm_gbs"] * 1e9)
@@ -371,7 +447,10 @@ def run_ours(args, w):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        f, dt, desc, threads = oracle_sample(w, q, k, v, kl, target_s=args.cpu_seconds)
+        if w.backward:
+            f, dt, desc, threads = oracle_sample_bwd(w, q, k, v, dout, kl, target_s=args.cpu_seconds)
+        else:
+            f, dt, desc, threads = oracle_sample(w, q, k, v, kl, target_s=args.cpu_seconds)
         cpu = {"value": f / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc,
                "seconds": dt}
 
@@ -383,7 +462,7 @@ def run_ours(args, w):
                                f"{' causal' if w.is_causal else ''}",
                    "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Nq": w.Nq, "Nk": w.Nk, "d": w.d,
                    "is_causal": w.is_causal, "key_lens": w.key_lens,
-                   "entry_point": ("attn_fwd_splitkv" if w.split_kv else
+                   "entry_point": ("attn_bwd" if w.backward else "attn_fwd_splitkv" if w.split_kv else
                                    "attn_fwd_mod" if (w.softcap or w.mask2d) else "attn_fwd"),
                    "softcap": w.softcap, "mask2d": w.mask2d,
                    "flops_per_step": flops, "parallelism": f"independent batch per GPU x{world}",
@@ -412,11 +491,18 @@ def run_reference(args, w):
     import torch
     from workloads import make_inputs
     q, k, v, kl = make_inputs(w, device="cpu")
+    do = None
+    if w.backward:
+        from workloads import make_qkv
+        do = make_qkv(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, seed=w.seed + 1)[0]
     steps, warmup = max(1, args.steps), max(0, args.warmup)
     per_step = max(0.2, min(10.0, args.reference_seconds / (steps + warmup)))
     times, flops_total, desc, threads = [], 0.0, "", 1
     for i in range(warmup + steps):
-        f, dt, desc, threads = oracle_sample(w, q, k, v, kl, target_s=per_step)
+        if w.backward:
+            f, dt, desc, threads = oracle_sample_bwd(w, q, k, v, do, kl, target_s=per_step)
+        else:
+            f, dt, desc, threads = oracle_sample(w, q, k, v, kl, target_s=per_step)
         if i >= warmup:
             times.append(dt)
             flops_total += f

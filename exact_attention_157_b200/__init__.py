@@ -316,7 +316,7 @@ def attention(q, k, v, *, scale: float | None = None, is_causal: bool = False, k
 
 
 def attention_backward(q, k, v, out, lse, dout, *, scale: float | None = None, is_causal: bool = False,
-                       key_lens=None, workspace=None, stream=None):
+                       key_lens=None, workspace=None, stream=None, dq=None, dk=None, dv=None):
     """dQ, dK, dV of ``attention`` for the upstream gradient ``dout`` (bf16 CUDA
     tensors shaped like q / k / v); ``out`` and ``lse`` are the forward results
     for the same inputs.  Returns (dq, dk, dv)."""
@@ -334,7 +334,13 @@ def attention_backward(q, k, v, out, lse, dout, *, scale: float | None = None, i
         raise AttnError(st, "attn_bwd_plan")
     if workspace is None:
         workspace = torch.empty((nbytes,), dtype=torch.uint8, device=q.device)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for name, t, ref in (("dq", dq, q), ("dk", dk, k), ("dv", dv, v)):
+        _check_bf16_cuda(name, t, 4)
+        if tuple(t.shape) != tuple(ref.shape):
+            raise ValueError(f"{name} has the wrong shape")
     kl_ptr = None
     if key_lens is not None:
         key_lens = key_lens.contiguous()

@@ -23,6 +23,9 @@ used):
                                                cache, grouped heads (the decoding
                                                phase of jsqmd.com/news/722897,
                                                section 5.2); run with split-KV
+  long_bwd, long_causal_bwd, prefill_gqa_bwd -- the backward pass (dQ, dK, dV) of the
+                        same shapes (section 3.3 of jsqmd.com/news/722897: training
+                        recomputes P from the saved statistics)
   vit3136_softcap       B8 H12 N3136 d64, soft-cap 30 -- the 56 x 56-patch ViT of
   vit3136_neighborhood  B8 H12 N3136 d64, radius-5      the PyTorch attention article
                         neighbourhood on the 56-wide    (atyun.com/61003.html: its
@@ -51,18 +54,23 @@ class Workload:
     split_kv: bool = False  # run through the split-KV entry point (automatic range count)
     softcap: float = 0.0    # > 0: soft-capped scores (attn_fwd_mod)
     mask2d: tuple | None = None  # ("neighborhood", W, R) or ("window", W, w, shift) (attn_fwd_mod)
+    backward: bool = False  # the step is the backward pass (attn_bwd) of this shape
 
     @property
     def scale(self) -> float:
         return 1.0 / math.sqrt(self.d)
 
     def flops(self) -> float:
-        """Forward FLOPs as the metric counts them: 4*B*Hq*Nq*Nk*d, halved when causal.
+        """FLOPs as the metric counts them: forward 4*B*Hq*Nq*Nk*d, halved when causal.
 
         The count 4*N^2*d for one head is the one "FlashAttention technical analysis"
-        (jsqmd.com/news/722897) section 3.1 uses (8.6 GFLOP at N=4096, d=128).
+        (jsqmd.com/news/722897) section 3.1 uses (8.6 GFLOP at N=4096, d=128).  The
+        backward pass counts its five N x N x d products (S recomputed, dP, dV, dQ,
+        dK): 2.5 times the forward count.
         """
         f = 4.0 * self.B * self.Hq * self.Nq * self.Nk * self.d
+        if self.backward:
+            f *= 2.5
         return f / 2.0 if self.is_causal else f
 
     def qkvo_bytes(self) -> int:
@@ -83,6 +91,9 @@ WORKLOADS = {
         Workload("unet_cross", 4, 8, 8, 4096, 77, 64, key_lens=(8, 77), seed=1013),
         Workload("prefill_gqa", 1, 32, 2, 16384, 16384, 128, is_causal=True, seed=1004),
         Workload("decode_gqa", 8, 32, 8, 1, 16384, 128, seed=1005, split_kv=True),
+        Workload("long_bwd", 8, 32, 32, 4096, 4096, 128, seed=1008, backward=True),
+        Workload("long_causal_bwd", 8, 32, 32, 4096, 4096, 128, is_causal=True, seed=1009, backward=True),
+        Workload("prefill_gqa_bwd", 1, 32, 2, 16384, 16384, 128, is_causal=True, seed=1010, backward=True),
         Workload("vit3136_softcap", 8, 12, 12, 3136, 3136, 64, seed=1006, softcap=30.0),
         Workload("vit3136_neighborhood", 8, 12, 12, 3136, 3136, 64, seed=1007, mask2d=("neighborhood", 56, 5)),
     ]
