@@ -329,11 +329,12 @@ def run_ours(args, w):
     split, ws, per_step_launches = None, None, 1
     if w.split_kv:
         split = 0
-        st, n_used, nbytes = ea.attn_splitkv_plan(w.B, w.Hq, w.Nq, w.Nk, w.d, split, 0)
+        st, n_used, nbytes = ea.attn_splitkv_plan(w.B, w.Hq, w.Nq, w.Nk, w.d, split, 0, Hkv=w.Hkv,
+                                                  is_causal=w.is_causal)
         if st != ea.ATTN_OK:
             raise ea.AttnError(st, "attn_splitkv_plan")
         ws = torch.empty((max(nbytes, 1),), dtype=torch.uint8, device=dev)
-        per_step_launches = 2 if n_used > 1 else 1
+        per_step_launches = 2 if nbytes > 0 else 1  # attention kernel + merge
 
     def call():
         if w.backward:
@@ -407,7 +408,7 @@ def run_ours(args, w):
         outh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
         lseh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
         runner = ea.HostAttention(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, device=dev, with_key_lens=kl is not None,
-                                  split_kv=split)
+                                  split_kv=split, is_causal=w.is_causal)
 
         def e2e_step():
             runner(qh, kh, vh, outh, lseh, klh, is_causal=w.is_causal, stream=stream, softcap=w.softcap,

@@ -95,7 +95,8 @@ def lib() -> ctypes.CDLL:
             L.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, vp,
                                    ctypes.c_size_t, vp]
             L.attn_splitkv_plan.restype = i
-            L.attn_splitkv_plan.argtypes = [i, i, i, i, i, i, i, ctypes.POINTER(i), ctypes.POINTER(ctypes.c_size_t)]
+            L.attn_splitkv_plan.argtypes = [i, i, i, i, i, i, i, i, i, ctypes.POINTER(i),
+                                            ctypes.POINTER(ctypes.c_size_t)]
             L.attn_fwd_splitkv.restype = i
             L.attn_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, vp, vp,
                                            i, vp, ctypes.c_size_t, vp]
@@ -165,11 +166,13 @@ def attn_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale, 
                               int(workspace_bytes), stream))
 
 
-def attn_splitkv_plan(B, Hq, Nq, Nk, d, n_splits=0, sm_count=0):
-    """The C planner: returns (status, key ranges used, workspace bytes)."""
+def attn_splitkv_plan(B, Hq, Nq, Nk, d, n_splits=0, sm_count=0, *, Hkv=None, is_causal=False):
+    """The C planner: returns (status, key ranges planned, workspace bytes).
+    Hkv defaults to Hq (no grouped heads)."""
     n = ctypes.c_int(0)
     nb = ctypes.c_size_t(0)
-    st = int(lib().attn_splitkv_plan(int(B), int(Hq), int(Nq), int(Nk), int(d), int(n_splits), int(sm_count),
+    st = int(lib().attn_splitkv_plan(int(B), int(Hq), int(Hq if Hkv is None else Hkv), int(Nq), int(Nk), int(d),
+                                     int(bool(is_causal)), int(n_splits), int(sm_count),
                                      ctypes.byref(n), ctypes.byref(nb)))
     return st, int(n.value), int(nb.value)
 
@@ -300,7 +303,7 @@ def attention(q, k, v, *, scale: float | None = None, is_causal: bool = False, k
         if st != ATTN_OK:
             raise AttnError(st, "attn_fwd")
         return out, lse
-    st, _, nbytes = attn_splitkv_plan(B, Hq, Nq, Nk, d, int(split_kv), 0)
+    st, _, nbytes = attn_splitkv_plan(B, Hq, Nq, Nk, d, int(split_kv), 0, Hkv=Hkv, is_causal=is_causal)
     if st != ATTN_OK:
         raise AttnError(st, "attn_splitkv_plan")
     if workspace is None:
@@ -367,11 +370,12 @@ class HostAttention:
     Each call copies Q, K, V (and key lengths) host -> device on ``stream``,
     runs ``attn_fwd`` and copies O and LSE back into the host tensors it was
     given; the device staging buffers (and a split-KV workspace when
-    ``split_kv`` is not None) are allocated once, here, and reused.
+    ``split_kv`` is not None, planned for ``is_causal``) are allocated once,
+    here, and reused.
     """
 
     def __init__(self, B, Hq, Hkv, Nq, Nk, d, device="cuda:0", with_lse=True, with_key_lens=False,
-                 split_kv=None):
+                 split_kv=None, is_causal=False):
         import torch
         dev = torch.device(device)
         bf = torch.bfloat16
@@ -385,7 +389,7 @@ class HostAttention:
         self.split_kv = split_kv
         self.workspace = None
         if split_kv is not None:
-            st, _, nbytes = attn_splitkv_plan(B, Hq, Nq, Nk, d, int(split_kv), 0)
+            st, _, nbytes = attn_splitkv_plan(B, Hq, Nq, Nk, d, int(split_kv), 0, Hkv=Hkv, is_causal=is_causal)
             if st != ATTN_OK:
                 raise AttnError(st, "attn_splitkv_plan")
             self.workspace = torch.empty((max(nbytes, 1),), dtype=torch.uint8, device=dev)

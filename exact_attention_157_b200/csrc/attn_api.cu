@@ -14,6 +14,7 @@
 #include "fwd_common.cuh"
 #include "fwd_kernel_pp.cuh"
 #include "bwd_kernels.cuh"
+#include "decode_kernel.cuh"
 
 using namespace attn_sm100;
 
@@ -76,6 +77,19 @@ cudaError_t set_bwd_attrs() {
                                 SmemBwd<D>::kAlloc);
 }
 
+template <int D>
+cudaError_t set_decode_attrs() {
+    return cudaFuncSetAttribute(attn_decode_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                SmemDec<D>::kAlloc);
+}
+
+template <int D>
+cudaError_t launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const DecParams& dp, unsigned grid,
+                          cudaStream_t s) {
+    attn_decode_kernel<D><<<grid, kDecThreads, SmemDec<D>::kAlloc, s>>>(tk, tv, dp);
+    return cudaGetLastError();
+}
+
 // One-time per-device set-up: architecture check, SM count, kernel attributes,
 // and the driver's tensor-map encoder.
 attn_status_t device_setup(int* dev_out) {
@@ -109,6 +123,8 @@ attn_status_t device_setup(int* dev_out) {
     if ((e = set_pp_attrs<64, kSlots64, kQStages64, false>()) != cudaSuccess) return cuda_fail(e);
     if ((e = set_pp_attrs<64, kSlots64, kQStages64, true>()) != cudaSuccess) return cuda_fail(e);
     if ((e = set_bwd_attrs<128>()) != cudaSuccess) return cuda_fail(e);
+    if ((e = set_decode_attrs<128>()) != cudaSuccess) return cuda_fail(e);
+    if ((e = set_decode_attrs<64>()) != cudaSuccess) return cuda_fail(e);
     if ((e = set_bwd_attrs<64>()) != cudaSuccess) return cuda_fail(e);
     st.ready = true;
     st.status = ATTN_OK;
@@ -117,10 +133,11 @@ attn_status_t device_setup(int* dev_out) {
 
 // 3-D map over a [heads, rows, d] bf16 tensor, box = 64 columns x 128 rows x 1,
 // 128-byte swizzle (the layout the UMMA shared-memory descriptors expect).
-attn_status_t encode_map(CUtensorMap* map, const void* base, int d, int rows, long long heads) {
+attn_status_t encode_map(CUtensorMap* map, const void* base, int d, int rows, long long heads,
+                         unsigned box_rows = 128u) {
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(heads)};
     cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2u, static_cast<cuuint64_t>(rows) * d * 2u};
-    cuuint32_t box[3] = {64u, 128u, 1u};
+    cuuint32_t box[3] = {64u, box_rows, 1u};
     cuuint32_t estr[3] = {1u, 1u, 1u};
     CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -162,6 +179,7 @@ size_t splitkv_bytes(long long rows, int d, int n_splits) {
 // block-times, and a unit count that is not a multiple of `sms` wastes the rest
 // of its last wave.  `requested` > 0 is taken as an upper bound.
 constexpr int kMaxSplits = 128;
+constexpr int kDecRangeCost = 15;  // chunks' worth of fixed cost per decode CTA (fitted on B200)
 constexpr int kUnitOverheadBlocks = 2;
 int choose_splits(long long base_units, int Nk, int sms, int requested) {
     const int n_blocks = (Nk + kBN - 1) / kBN;
@@ -178,6 +196,68 @@ int choose_splits(long long base_units, int Nk, int sms, int requested) {
         if (best_cost < 0 || cost < best_cost) { best_cost = cost; best = s; }
     }
     return best;
+}
+
+// Whether a split-KV call can run on the decode kernel: every query head of a
+// K/V head times Nq fits its row limit, no causal or additive mask.
+bool decode_shape(int Hq, int Hkv, int Nq, bool causal, bool mask) {
+    return !causal && !mask && static_cast<long long>(Hq / Hkv) * Nq <= kDecMaxRows;
+}
+
+struct SplitPlan {
+    bool decode;     // decode kernel (32-key chunks) instead of the tile kernel (128-key blocks)
+    int n_splits;    // key ranges
+    int split_keys;  // keys per range
+    size_t bytes;    // workspace
+};
+
+// The plan of a split-KV call.  Decode-shaped calls (ignoring an additive mask,
+// which the caller may add without re-planning) minimise a wave-count cost; the
+// others use choose_splits.  A call with a mask on a decode shape runs the
+// tile kernel with at most the planned number of ranges, so the workspace fits.
+SplitPlan make_plan(int B, int Hq, int Hkv, int Nq, int Nk, int d, bool causal, int requested, int sms) {
+    SplitPlan pl{};
+    const long long rows = static_cast<long long>(B) * Hq * Nq;
+    if (decode_shape(Hq, Hkv, Nq, causal, false)) {
+        const int chunks = (Nk + kDecChunk - 1) / kDecChunk;
+        int n;
+        if (requested > 0) {
+            n = requested;
+        } else {
+            // one CTA per SM streams about its share of HBM bandwidth, so the time is
+            // (waves of CTAs over the SMs) x (chunks per range + a fixed cost of about
+            // kDecRangeCost chunks for the pipeline fill and the merge); ranges keep
+            // at least one chunk per consumer warp
+            const long long pairs = static_cast<long long>(B) * Hkv;
+            const int most = chunks / kDecWarps > 1 ? chunks / kDecWarps : 1;
+            long long best_cost = -1;
+            n = 1;
+            for (int t = 1; t <= most && t <= kMaxSplits; ++t) {
+                const int per_t = (chunks + t - 1) / t;
+                if ((chunks + per_t - 1) / per_t != t) continue;
+                const long long waves = (pairs * t + sms - 1) / sms;
+                const long long cost = waves * (per_t + kDecRangeCost);
+                if (best_cost < 0 || cost < best_cost) { best_cost = cost; n = t; }
+            }
+        }
+        if (n > chunks) n = chunks;
+        if (n < 1) n = 1;
+        const int per = (chunks + n - 1) / n;
+        pl.decode = true;
+        pl.n_splits = (chunks + per - 1) / per;
+        pl.split_keys = per * kDecChunk;
+        pl.bytes = splitkv_bytes(rows, d, pl.n_splits);
+        return pl;
+    }
+    const long long n_qtiles = (static_cast<long long>(Nq) + 2 * kBM - 1) / (2 * kBM);
+    const int chosen = choose_splits(static_cast<long long>(B) * Hq * n_qtiles, Nk, sms, requested);
+    const int n_blocks = (Nk + kBN - 1) / kBN;
+    const int per = (n_blocks + chosen - 1) / chosen;
+    pl.decode = false;
+    pl.n_splits = (n_blocks + per - 1) / per;
+    pl.split_keys = per * kBN;
+    pl.bytes = pl.n_splits > 1 ? splitkv_bytes(rows, d, pl.n_splits) : 0;
+    return pl;
 }
 
 
@@ -289,8 +369,44 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, f
     p.ws_o = nullptr;
     p.ws_lse = nullptr;
     if (split_kv) {
-        const int n_splits = choose_splits(static_cast<long long>(B) * Hq * p.n_qtiles, Nk, sms, n_splits_req);
+        const SplitPlan pl = make_plan(B, Hq, Hkv, Nq, Nk, d, is_causal != 0, n_splits_req, sms);
+        if (pl.decode && additive_mask == nullptr) {
+            if (workspace == nullptr || workspace_bytes < pl.bytes) return ATTN_ERR_INVALID_ARG;
+            DecParams dp;
+            dp.B = B; dp.Hq = Hq; dp.Hkv = Hkv; dp.Nq = Nq; dp.Nk = Nk; dp.group = Hq / Hkv;
+            dp.rows = dp.group * Nq;
+            dp.scale_log2 = p.scale_log2;
+            dp.key_lens = key_lens;
+            dp.q = static_cast<const uint16_t*>(q);
+            dp.n_splits = pl.n_splits;
+            dp.split_keys = pl.split_keys;
+            dp.ws_o = static_cast<float*>(workspace);
+            dp.ws_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                                 round_up(static_cast<size_t>(pl.n_splits) * rows * d * sizeof(float),
+                                                          kWsAlign));
+            dp.timeout_ns = p.timeout_ns;
+            dp.epoch = p.epoch;
+            CUtensorMap dk, dv;
+            if ((st = encode_map(&dk, k, d, Nk, static_cast<long long>(B) * Hkv, kDecChunk)) != ATTN_OK) return st;
+            if ((st = encode_map(&dv, v, d, Nk, static_cast<long long>(B) * Hkv, kDecChunk)) != ATTN_OK) return st;
+            cudaStream_t s = static_cast<cudaStream_t>(stream);
+            const unsigned grid = static_cast<unsigned>(static_cast<long long>(B) * Hkv * pl.n_splits);
+            cudaError_t e;
+            e = d == 128 ? launch_decode<128>(dk, dv, dp, grid, s) : launch_decode<64>(dk, dv, dp, grid, s);
+            if (e != cudaSuccess) return cuda_fail(e);
+            const unsigned cg = static_cast<unsigned>((rows + 7) / 8);
+            if (d == 128)
+                attn_splitkv_combine_kernel<128><<<cg, 256, 0, s>>>(dp.ws_o, dp.ws_lse, static_cast<__nv_bfloat16*>(out),
+                                                                    lse, rows, pl.n_splits);
+            else
+                attn_splitkv_combine_kernel<64><<<cg, 256, 0, s>>>(dp.ws_o, dp.ws_lse, static_cast<__nv_bfloat16*>(out),
+                                                                   lse, rows, pl.n_splits);
+            if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e);
+            return ATTN_OK;
+        }
+        // tile kernel: at most the planned number of ranges, in 128-key blocks
         const int n_blocks = (Nk + kBN - 1) / kBN;
+        const int n_splits = pl.n_splits < n_blocks ? pl.n_splits : n_blocks;
         const int per = (n_blocks + n_splits - 1) / n_splits;
         p.n_splits = (n_blocks + per - 1) / per;
         if (p.n_splits > 1) {
@@ -356,9 +472,11 @@ attn_status_t attn_fwd_mod(const void* q, const void* k, const void* v, void* ou
                     false, 1, nullptr, 0, mod, stream);
 }
 
-attn_status_t attn_splitkv_plan(int B, int Hq, int Nq, int Nk, int d, int n_splits, int sm_count,
-                                int* n_splits_out, size_t* workspace_bytes) {
-    if (B <= 0 || Hq <= 0 || Nq <= 0 || Nk <= 0 || d <= 0 || n_splits < 0 || sm_count < 0) return ATTN_ERR_INVALID_ARG;
+attn_status_t attn_splitkv_plan(int B, int Hq, int Hkv, int Nq, int Nk, int d, int is_causal, int n_splits,
+                                int sm_count, int* n_splits_out, size_t* workspace_bytes) {
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nk <= 0 || d <= 0 || n_splits < 0 || sm_count < 0)
+        return ATTN_ERR_INVALID_ARG;
+    if (Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
     int sms = sm_count;
     if (sms == 0) {
@@ -367,14 +485,9 @@ attn_status_t attn_splitkv_plan(int B, int Hq, int Nq, int Nk, int d, int n_spli
         if (st != ATTN_OK) return st;
         sms = g_dev[dev].sm_count > 0 ? g_dev[dev].sm_count : 1;
     }
-    const long long n_qtiles = (static_cast<long long>(Nq) + 2 * kBM - 1) / (2 * kBM);
-    const int chosen = choose_splits(static_cast<long long>(B) * Hq * n_qtiles, Nk, sms, n_splits);
-    const int n_blocks = (Nk + kBN - 1) / kBN;
-    const int per = (n_blocks + chosen - 1) / chosen;
-    const int used = (n_blocks + per - 1) / per;
-    if (n_splits_out != nullptr) *n_splits_out = used;
-    if (workspace_bytes != nullptr)
-        *workspace_bytes = used > 1 ? splitkv_bytes(static_cast<long long>(B) * Hq * Nq, d, used) : 0;
+    const SplitPlan pl = make_plan(B, Hq, Hkv, Nq, Nk, d, is_causal != 0, n_splits, sms);
+    if (n_splits_out != nullptr) *n_splits_out = pl.n_splits;
+    if (workspace_bytes != nullptr) *workspace_bytes = pl.bytes;
     return ATTN_OK;
 }
 
@@ -565,8 +678,8 @@ extern "C" attn_status_t attn_fwd_splitkv_noalloc(const void* q, const void* k, 
     if (st != ATTN_OK) return st;
     int used = 1;
     size_t need = 0;
-    if ((st = attn_splitkv_plan(B, Hq, Nq, Nk, d, n_splits, g_dev[dev].sm_count > 0 ? g_dev[dev].sm_count : 1,
-                                &used, &need)) != ATTN_OK)
+    if ((st = attn_splitkv_plan(B, Hq, Hkv, Nq, Nk, d, is_causal, n_splits,
+                                g_dev[dev].sm_count > 0 ? g_dev[dev].sm_count : 1, &used, &need)) != ATTN_OK)
         return st;
     if (need > static_cast<size_t>(ATTN_NOALLOC_SCRATCH_BYTES)) return ATTN_ERR_SCRATCH;
     void* scratch = nullptr;

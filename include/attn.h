@@ -145,17 +145,23 @@ attn_status_t attn_fwd_mod(const void *q, const void *k, const void *v, void *ou
  * workspace it then needs.  Host-only arithmetic (no CUDA call) when
  * sm_count > 0; sm_count == 0 queries the current device's SM count.
  *   n_splits: 0 = choose automatically; k > 0 = at most k ranges.
- *   n_splits_out (host, may be NULL): key ranges actually used (1 = no split,
- *     the launch then writes out directly and needs no workspace).
- *   workspace_bytes (host, may be NULL): bytes of device workspace needed.
- * The keys are cut into n_splits_out ranges of equal length (a multiple of
- * 128 keys; the last may be shorter).  The automatic choice minimises
- * (waves of units over the SMs) x (key blocks per range + 2).
- * Errors: ATTN_ERR_INVALID_ARG for non-positive sizes or negative counts,
- * ATTN_ERR_UNSUPPORTED for d not in {64, 128}.
+ *   n_splits_out (host, may be NULL): key ranges planned.
+ *   workspace_bytes (host, may be NULL): bytes of device workspace needed
+ *     (0 when the call writes out directly).
+ * Decoding shapes -- (Hq / Hkv) * Nq <= 16 query rows per K/V head and not
+ * causal -- run on the decode kernel: ranges of 32-key chunks; the automatic
+ * count is the first minimiser of ceil(B * Hkv * n / SMs) * (chunks per range
+ * + 15) over counts n that the equal cut realises exactly, with at least 6
+ * chunks per range; its partial results always go through the workspace.  Other shapes run on the tile kernel:
+ * ranges of 128-key blocks, the automatic choice minimising (waves of units
+ * over the SMs) x (key blocks per range + 2), and one range writes out
+ * directly.  The plan does not depend on an additive mask: with a mask, a
+ * decoding shape runs the tile kernel with at most the planned ranges.
+ * Errors: ATTN_ERR_INVALID_ARG for non-positive sizes, Hq % Hkv != 0 or
+ * negative counts, ATTN_ERR_UNSUPPORTED for d not in {64, 128}.
  */
-attn_status_t attn_splitkv_plan(int B, int Hq, int Nq, int Nk, int d, int n_splits, int sm_count,
-                                int *n_splits_out, size_t *workspace_bytes);
+attn_status_t attn_splitkv_plan(int B, int Hq, int Hkv, int Nq, int Nk, int d, int is_causal, int n_splits,
+                                int sm_count, int *n_splits_out, size_t *workspace_bytes);
 
 /*
  * attn_fwd_splitkv -- attn_fwd with the keys of every (batch, head) cut into
@@ -172,13 +178,15 @@ attn_status_t attn_splitkv_plan(int B, int Hq, int Nq, int Nk, int d, int n_spli
  * Arguments as attn_fwd, plus:
  *   n_splits: 0 = automatic (attn_splitkv_plan), k > 0 = at most k ranges.
  *   workspace: device, 256-byte aligned, at least the bytes attn_splitkv_plan
- *     reports for the same sizes (may be NULL when that is 0).  The library
+ *     reports for the same sizes, is_causal and n_splits (may be NULL when
+ *     that is 0).  The library
  *     writes it before reading it (nothing needs to start at zero); its
  *     contents after the call are unspecified.  Two calls in flight at once
  *     must not share a workspace.
- * Two kernels run on `stream`: the attention kernel (partials to the
- * workspace) and the merge (out, lse); with one range only the first, writing
- * out directly.
+ * Two kernels run on `stream`: the attention kernel -- the decode kernel
+ * (CUDA cores; every query row of a K/V head shares each K/V chunk, read from
+ * HBM once) or the tile kernel -- with partials to the workspace, then the
+ * merge (out, lse); a tile-kernel call with one range writes out directly.
  * Errors: as attn_fwd; ATTN_ERR_INVALID_ARG also for n_splits < 0 or a
  * missing / short workspace, ATTN_ERR_ALIGNMENT for a misaligned workspace.
  */

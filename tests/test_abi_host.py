@@ -102,7 +102,8 @@ def _ws_bytes(rows, d, s):
     (1, 1, 1, 100, 128, 8, 1),    # a single key block never splits
 ])
 def test_splitkv_plan_requested(B, Hq, Nq, Nk, d, req, used):
-    st, n, nbytes = ea.attn_splitkv_plan(B, Hq, Nq, Nk, d, req, 148)
+    """Tile-kernel plans (causal shapes never take the decode kernel)."""
+    st, n, nbytes = ea.attn_splitkv_plan(B, Hq, Nq, Nk, d, req, 148, is_causal=True)
     assert st == ea.ATTN_OK
     assert n == used
     assert nbytes == (_ws_bytes(B * Hq * Nq, d, n) if n > 1 else 0)
@@ -125,8 +126,51 @@ def test_splitkv_plan_auto_minimises_stated_cost(B, Hq, Nq, Nk):
         cost = -(-(units * s) // sms) * (per + 2)
         if best_cost is None or cost < best_cost:
             best, best_cost = s, cost
-    st, n, _ = ea.attn_splitkv_plan(B, Hq, Nq, Nk, 128, 0, sms)
+    st, n, _ = ea.attn_splitkv_plan(B, Hq, Nq, Nk, 128, 0, sms, is_causal=True)
     assert st == ea.ATTN_OK and n == best
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Nq,Nk,d,req,used", [
+    (4, 16, 4, 1, 5000, 128, 6, 6),
+    (1, 1, 1, 1, 100, 128, 8, 4),       # 4 chunks of 32 keys: at most 4 ranges
+])
+def test_splitkv_plan_decode_requested(B, Hq, Hkv, Nq, Nk, d, req, used):
+    st, n, nbytes = ea.attn_splitkv_plan(B, Hq, Nq, Nk, d, req, 148, Hkv=Hkv)
+    assert st == ea.ATTN_OK
+    assert n == used
+    assert nbytes == _ws_bytes(B * Hq * Nq, d, n)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Nq,Nk,d", [
+    (8, 32, 8, 1, 16384, 128), (1, 32, 8, 1, 131072, 128), (2, 8, 2, 3, 3000, 64), (64, 16, 16, 1, 4096, 64),
+    (3, 24, 3, 2, 77777, 128)])
+def test_splitkv_plan_decode_auto_minimises_stated_cost(B, Hq, Hkv, Nq, Nk, d):
+    """Decode-kernel plans: the first minimiser of
+    ceil(B * Hkv * n / SMs) * (chunks per range + 15) over the counts the equal
+    cut realises, at least 6 chunks per range (the header's model); always a
+    workspace."""
+    sms = 148
+    chunks = -(-Nk // 32)
+    most = max(chunks // 6, 1)
+    best, best_cost = 1, None
+    for t in range(1, min(most, 128) + 1):
+        per = -(-chunks // t)
+        if -(-chunks // per) != t:
+            continue
+        cost = -(-(B * Hkv * t) // sms) * (per + 15)
+        if best_cost is None or cost < best_cost:
+            best, best_cost = t, cost
+    st, n, nbytes = ea.attn_splitkv_plan(B, Hq, Nq, Nk, d, 0, sms, Hkv=Hkv)
+    assert st == ea.ATTN_OK and n == best
+    assert nbytes == _ws_bytes(B * Hq * Nq, d, n)
+
+
+def test_splitkv_plan_decode_rows_limit():
+    """More than 16 query rows per K/V head, or causal, falls back to the tile plan."""
+    tile = ea.attn_splitkv_plan(1, 32, 17, 4096, 128, 0, 148, Hkv=32, is_causal=True)
+    assert ea.attn_splitkv_plan(1, 32, 17, 4096, 128, 0, 148, Hkv=32) == tile
+    assert ea.attn_splitkv_plan(1, 32, 1, 4096, 128, 0, 148, Hkv=1) == \
+        ea.attn_splitkv_plan(1, 32, 1, 4096, 128, 0, 148, Hkv=1, is_causal=True)
 
 
 def test_splitkv_plan_rejects_bad_sizes():
@@ -134,6 +178,7 @@ def test_splitkv_plan_rejects_bad_sizes():
     assert ea.attn_splitkv_plan(1, 1, 1, 1, 64, -1, 148)[0] == ea.ATTN_ERR_INVALID_ARG
     assert ea.attn_splitkv_plan(1, 1, 1, 1, 64, 0, -5)[0] == ea.ATTN_ERR_INVALID_ARG
     assert ea.attn_splitkv_plan(1, 1, 1, 1, 96, 0, 148)[0] == ea.ATTN_ERR_UNSUPPORTED
+    assert ea.attn_splitkv_plan(1, 3, 1, 1, 64, 0, 148, Hkv=2)[0] == ea.ATTN_ERR_INVALID_ARG
 
 
 @pytest.mark.parametrize("args,status", [

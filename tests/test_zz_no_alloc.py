@@ -35,7 +35,7 @@ def _noalloc(qd, kd, vd, B, Hq, Hkv, Nq, Nk, d, n_splits, key_lens=None, causal=
 
 
 def _with_workspace(qd, kd, vd, B, Hq, Hkv, Nq, Nk, d, n_splits, key_lens=None, causal=False):
-    st, _, nbytes = ea.attn_splitkv_plan(B, Hq, Nq, Nk, d, n_splits, 0)
+    st, _, nbytes = ea.attn_splitkv_plan(B, Hq, Nq, Nk, d, n_splits, 0, Hkv=Hkv)
     assert st == ea.ATTN_OK
     ws = torch.empty((max(nbytes, 1),), dtype=torch.uint8, device=DEV)
     out = torch.empty_like(qd)
@@ -87,7 +87,7 @@ def test_noalloc_key_lens_twice_and_no_new_device_memory():
 def test_noalloc_rejects_plans_beyond_the_fixed_buffer():
     # 4096 rows x 8 ranges x (128 + 1) fp32 values = 16.9 MB > 16 MiB; real buffers
     B, Hq, Hkv, Nq, Nk, d = 1, 8, 8, 512, 8192, 128
-    st, used, nbytes = ea.attn_splitkv_plan(B, Hq, Nq, Nk, d, 8, 0)
+    st, used, nbytes = ea.attn_splitkv_plan(B, Hq, Nq, Nk, d, 8, 0, Hkv=Hkv)
     assert st == ea.ATTN_OK and used == 8 and nbytes > ea.NOALLOC_SCRATCH_BYTES
     _, _, _, qd, kd, vd = _inputs(B, Hq, Hkv, Nq, Nk, d, seed=23)
     out = torch.zeros_like(qd)
