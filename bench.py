@@ -34,8 +34,21 @@ if ROOT not in sys.path:
 
 METRIC = "fwd attention TFLOP/s (B8 H32 N4096 d128 bf16) and % of B200 BF16 peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCES = ["exact_attention_157_b200/csrc/fwd_kernel_pp.cuh", "exact_attention_157_b200/csrc/fwd_common.cuh",
-                  "exact_attention_157_b200/csrc/sm100_ptx.cuh", "exact_attention_157_b200/csrc/attn_api.cu"]
+# device code of each workload's dominant kernel: a recorded ncu traffic figure is
+# valid only for the sources it was captured on
+_CSRC = "exact_attention_157_b200/csrc/"
+_COMMON = [_CSRC + "fwd_common.cuh", _CSRC + "sm100_ptx.cuh"]
+KERNEL_SOURCES = {"tile": [_CSRC + "fwd_kernel_pp.cuh"] + _COMMON,
+                  "decode": [_CSRC + "decode_kernel.cuh"] + _COMMON,
+                  "bwd": [_CSRC + "bwd_kernels.cuh"] + _COMMON}
+
+
+def kernel_family(w) -> str:
+    if w.backward:
+        return "bwd"
+    if w.split_kv and w.Hq // w.Hkv * w.Nq <= 16 and not w.is_causal:
+        return "decode"
+    return "tile"
 
 
 # --------------------------------------------------------------- helpers
@@ -51,25 +64,25 @@ def load_peaks():
         return dict(FALLBACK_PEAKS, source="fallback")
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(family: str = "tile") -> str:
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in KERNEL_SOURCES[family]:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload: str):
+def recorded_traffic(w):
     """DRAM bytes per launch from the committed ncu summary of this kernel and
     workload, if it was taken on the current kernel sources; else None."""
-    path = os.path.join(ROOT, "profiles", f"attn_fwd_{workload}.md")
+    path = os.path.join(ROOT, "profiles", f"attn_{'bwd' if w.backward else 'fwd'}_{w.name}.md")
     try:
         text = open(path).read()
     except OSError:
         return None
     m_b = re.search(r"^traffic_bytes_per_launch:\s*([0-9.eE+]+)", text, re.M)
     m_h = re.search(r"^kernel_source_sha:\s*([0-9a-f]+)", text, re.M)
-    if not m_b or not m_h or m_h.group(1) != kernel_source_hash():
+    if not m_b or not m_h or m_h.group(1) != kernel_source_hash(kernel_family(w)):
         return None
     return float(m_b.group(1))
 
@@ -442,7 +455,7 @@ def run_ours(args, w):
         roof = {"bound": "hbm", "achieved": per_launch_bytes / t_launch / 1e9, "peak": peaks["hbm_gbs"],
                 "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = recorded_traffic(w.name)
+    roof["traffic"] = recorded_traffic(w)
     roof["peak_source"] = peaks["source"] + " (burst)"
     roof["frac_of_roofline_time"] = max(compute_floor, hbm_floor) / t_launch
 
@@ -475,7 +488,7 @@ def run_ours(args, w):
                 "d2h_bytes_per_step": out_bytes, "ms_per_step": e2e_ms},
         "gpu_launches": launches,
         "clocks": clocks.summary(),
-        "kernel_source_sha": kernel_source_hash(),
+        "kernel_source_sha": kernel_source_hash(kernel_family(w)),
     }
     if world > 1:
         import torch.distributed as dist

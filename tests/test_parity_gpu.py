@@ -262,3 +262,31 @@ def test_out_of_range_key_lens_are_reported():
     st, info = ea.attn_check_device_status(ea._stream_handle(None))
     assert st == ea.ATTN_ERR_DEVICE, hex(info)
     assert torch.isfinite(out).all()  # clamped to Nk, memory-safe
+
+
+# ------------------------------------------------------- short key sequences
+@pytest.mark.parametrize("Nq,Nk", [(196, 196), (4096, 77), (17, 256), (300, 33), (1, 1)])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_short_keys_vs_oracle(Nq, Nk, d, causal):
+    """Short key sequences (the ViT and text cross-attention shapes), with key lengths."""
+    B, Hq, Hkv = 2, 4, 2
+    q, k, v = make_qkv(B, Hq, Hkv, Nq, Nk, d, seed=Nq + 5 * Nk + d + causal)
+    lens = torch.tensor([Nk, max(Nk // 3, 0)], dtype=torch.int32)
+    out, lse = run_gpu(q, k, v, is_causal=causal, key_lens=lens)
+    ro, rl = oracle.attention(q, k, v, is_causal=causal, key_lens=lens.tolist())
+    assert_close(out, lse, ro, rl)
+
+
+def test_short_keys_masked_keys_bit_exact():
+    B, H, Nq, Nk, d = 3, 2, 200, 200, 64
+    q, k, v = make_qkv(B, H, H, Nq, Nk, d, seed=61)
+    lens = torch.tensor([200, 77, 0], dtype=torch.int32)
+    out1, lse1 = run_gpu(q, k, v, key_lens=lens)
+    k2, v2 = k.clone(), v.clone()
+    for b, n in enumerate(lens.tolist()):
+        k2[b, :, n:] = 1e4 * torch.randn(H, Nk - n, d).to(torch.bfloat16)
+        v2[b, :, n:] = 1e4 * torch.randn(H, Nk - n, d).to(torch.bfloat16)
+    out2, lse2 = run_gpu(q, k2, v2, key_lens=lens)
+    assert torch.equal(out1, out2) and torch.equal(lse1, lse2)
+    assert torch.all(out1[2] == 0) and torch.all(torch.isneginf(lse1[2]))
