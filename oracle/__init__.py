@@ -17,6 +17,10 @@ Contents
 ``attention_loops``      pure-Python loops for tiny inputs (brute force).
 ``attention_bwd``        the gradients dQ, dK, dV of the definition for a given dO, in
                          plain C, fp64 (``attn_oracle_bwd.c``).
+``e4m3_decode``,         FP8 inputs: the E4M3 code -> value map written from the format
+``dequantize_blocks``,   (1 sign, 4 exponent bits with bias 7, 3 mantissa bits, subnormals,
+``attention_fp8``        no infinities, S.1111.111 = NaN) and per-128-row block scales;
+                         the result is the definition on the dequantized values.
 
 Sources: "FlashAttention technical analysis" (jsqmd.com/news/722897) section 2.1
 (the three steps), section 2.2 (tiling plus online softmax with running max and
@@ -254,6 +258,38 @@ def attention(q, k, v, *, scale: float | None = None, is_causal: bool = False,
     if rc != 0:
         raise ValueError(f"oracle_attention_fwd rejected its arguments (status {rc})")
     return out, lse
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """Value of each FP8 E4M3 code (uint8): sign bit 7, exponent bits 6..3 with
+    bias 7, mantissa bits 2..0; exponent 0 is subnormal (m / 8 * 2^-6); the
+    all-ones exponent and mantissa (0x7F, 0xFF) is NaN; there are no infinities.
+    The format behind the FP8 tensor-core inputs of "FlashAttention technical
+    analysis" (jsqmd.com/news/722897) sections 4.2 and 6.3."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = c & 0x7
+    val = np.where(e == 0, (m / 8.0) * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 7.0))
+    val = sign * val
+    return np.where((c & 0x7F) == 0x7F, np.nan, val)
+
+
+def dequantize_blocks(codes, scales, block: int = 128) -> np.ndarray:
+    """codes [..., N, d] (E4M3), scales [..., ceil(N / block)]: row i of every
+    head is multiplied by its block's scale, scales[..., i // block] ("each
+    block keeps its own scale factor", jsqmd.com/news/722897 section 6.3)."""
+    x = e4m3_decode(codes)
+    s = np.asarray(scales, dtype=np.float64)
+    n = x.shape[-2]
+    idx = np.arange(n) // block
+    return x * s[..., idx][..., None]
+
+
+def attention_fp8(q8, k8, v8, q_scale, k_scale, v_scale, **kw):
+    """The definition on the dequantized FP8 inputs (fp64): (O, LSE)."""
+    return attention(dequantize_blocks(q8, q_scale), dequantize_blocks(k8, k_scale),
+                     dequantize_blocks(v8, v_scale), **kw)
 
 
 def _masked_scores(q, k, scale, is_causal, key_lens, mask):

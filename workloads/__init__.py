@@ -100,6 +100,33 @@ WORKLOADS = {
 }
 
 
+def quantize_e4m3_blocks(x: torch.Tensor, block: int = 128):
+    """Per-128-row-block FP8 E4M3 codes of x [..., N, d] (fp32): scale = amax of
+    the block / 448 (the largest finite E4M3 value), codes = round-to-nearest of
+    x / scale by torch's float8_e4m3fn conversion.  Returns (codes uint8, scales
+    fp32 [..., ceil(N / block)])."""
+    n = x.shape[-2]
+    nb = (n + block - 1) // block
+    pad = nb * block - n
+    xp = torch.nn.functional.pad(x, (0, 0, 0, pad))
+    xb = xp.reshape(*x.shape[:-2], nb, block, x.shape[-1])
+    amax = xb.abs().amax(dim=(-1, -2))
+    scales = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax)).to(torch.float32)
+    y = (xb / scales[..., None, None]).clamp(-448.0, 448.0).reshape(*xp.shape)[..., :n, :]
+    return y.to(torch.float8_e4m3fn).view(torch.uint8).contiguous(), scales.contiguous()
+
+
+def make_fp8_inputs(B, Hq, Hkv, Nq, Nk, d, seed):
+    """FP8 Q, K, V (codes and per-128-row scales) from the same N(0, 1) draws as
+    make_qkv (fp32 before rounding), on the CPU."""
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn((B, Hq, Nq, d), generator=g)
+    k = torch.randn((B, Hkv, Nk, d), generator=g)
+    v = torch.randn((B, Hkv, Nk, d), generator=g)
+    (q8, qs), (k8, ks), (v8, vs) = (quantize_e4m3_blocks(t) for t in (q, k, v))
+    return q8, k8, v8, qs, ks, vs
+
+
 def make_qkv(B, Hq, Hkv, Nq, Nk, d, seed, device="cpu"):
     """bf16 Q [B,Hq,Nq,d], K/V [B,Hkv,Nk,d], i.i.d. N(0,1) rounded to bf16."""
     g = torch.Generator(device=device)
