@@ -193,9 +193,11 @@ def workload_flops(w):
 
 
 # ---------------------------------------------------------- CPU baseline
-def oracle_sample(w, q, k, v, kl, target_s: float, max_rows=None):
+def oracle_sample(w, q, k, v, kl, target_s: float, max_rows=None, scales=None):
     """Runs the fp64 oracle on a bounded sample of the workload: whole query
     rows of the first (batch, head) pairs, as many as fit in ~target_s.
+    FP8 workloads pass E4M3 codes as q, k, v and their block scales in
+    ``scales``; the sampled heads are dequantized first.
     Returns (flops, seconds, description, threads)."""
     import numpy as np
     import oracle
@@ -205,8 +207,13 @@ def oracle_sample(w, q, k, v, kl, target_s: float, max_rows=None):
 
     def head_inputs(b, h):
         hk = h // group
-        return (q[b:b + 1, h:h + 1].cpu().double().numpy(), k[b:b + 1, hk:hk + 1].cpu().double().numpy(),
-                v[b:b + 1, hk:hk + 1].cpu().double().numpy(), None if kl_list is None else [kl_list[b]])
+        cut = lambda t, i: t[b:b + 1, i:i + 1].cpu()  # noqa: E731
+        if scales is None:
+            qh, kh, vh = (cut(t, i).double().numpy() for t, i in ((q, h), (k, hk), (v, hk)))
+        else:
+            qh, kh, vh = (oracle.dequantize_blocks(cut(t, i).numpy(), cut(sc, i).numpy())
+                          for t, sc, i in ((q, scales[0], h), (k, scales[1], hk), (v, scales[2], hk)))
+        return qh, kh, vh, None if kl_list is None else [kl_list[b]]
 
     per_row = None if w.mask2d is None else mask2d_keys_per_row(w)
     var = dict(softcap=w.softcap, mask2d=w.mask2d)
@@ -258,7 +265,8 @@ def oracle_sample(w, q, k, v, kl, target_s: float, max_rows=None):
     dt = time.perf_counter() - t0
     n_rows = sum(len(r) for _, _, r in plan)
     desc = (f"{n_rows} query rows over {len(plan)} (batch, head) pairs of the {w.name} workload "
-            f"({n_rows / (w.B * w.Hq * w.Nq):.2e} of it), fp64, all keys of each row")
+            f"({n_rows / (w.B * w.Hq * w.Nq):.2e} of it), fp64{' on the dequantized FP8 inputs' if scales else ''}, "
+            f"all keys of each row")
     return total, dt, desc, threads
 
 
@@ -316,12 +324,19 @@ def run_ours(args, w):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
-    q, k, v, kl = make_inputs(w, device=dev, seed=w.seed + 7 * rank)
-    out = torch.empty_like(q)
+    scales = None
+    if w.fp8:
+        from workloads import make_fp8_inputs
+        q, k, v, *scales = make_fp8_inputs(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, seed=w.seed + 7 * rank, device=dev)
+        kl = None
+        out = torch.empty((w.B, w.Hq, w.Nq, w.d), dtype=torch.bfloat16, device=dev)
+    else:
+        q, k, v, kl = make_inputs(w, device=dev, seed=w.seed + 7 * rank)
+        out = torch.empty_like(q)
     lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
     flops = workload_flops(w)
-    in_bytes = q.numel() * 2 + k.numel() * 2 + v.numel() * 2 + (0 if kl is None else kl.numel() * 4)
+    in_bytes = sum(t.numel() * t.element_size() for t in [q, k, v] + (scales or []) + ([] if kl is None else [kl]))
     out_bytes = out.numel() * 2 + lse.numel() * 4
     if w.backward:
         # the forward results and an upstream gradient are inputs of the timed backward step
@@ -350,6 +365,9 @@ def run_ours(args, w):
         per_step_launches = 2 if nbytes > 0 else 1  # attention kernel + merge
 
     def call():
+        if w.fp8:
+            ea.attention_fp8(q, k, v, *scales, is_causal=w.is_causal, out=out, lse=lse, stream=stream)
+            return
         if w.backward:
             ea.attention_backward(q, k, v, out, lse, dout, is_causal=w.is_causal, key_lens=kl, workspace=bws,
                                   stream=stream, dq=dq, dk=dk, dv=dv)
@@ -415,6 +433,18 @@ def run_ours(args, w):
                 call()
                 for dst, src in zip(host_out, (dq, dk, dv)):
                     dst.copy_(src, non_blocking=True)
+    elif w.fp8:
+        host_in = [t.cpu().pin_memory() for t in [q, k, v] + scales]
+        outh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        lseh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+
+        def e2e_step():
+            with torch.cuda.stream(stream):
+                for dst, src in zip([q, k, v] + scales, host_in):
+                    dst.copy_(src, non_blocking=True)
+                call()
+                outh.copy_(out, non_blocking=True)
+                lseh.copy_(lse, non_blocking=True)
     else:
         qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
         klh = None if kl is None else kl.cpu().pin_memory()
@@ -445,18 +475,22 @@ def run_ours(args, w):
     per_launch_bytes = w.qkvo_bytes() + w.lse_bytes()
     if w.backward:  # read Q, K, V, O, dO, LSE; write dQ, dK, dV
         per_launch_bytes = 2 * w.qkvo_bytes() + w.lse_bytes()
+    peak_tc, peak_note = peaks["bf16_tflops"], " (burst)"
+    if w.fp8:  # E4M3 codes and block scales in, bf16 O and fp32 LSE out
+        per_launch_bytes = in_bytes + out.numel() * 2 + w.lse_bytes()
+        peak_tc, peak_note = 2.0 * peaks["bf16_tflops"], " bf16 (burst) x 2, the nominal FP8 / BF16 dense ratio"
     t_launch = ms_per_step * 1e-3
-    compute_floor = per_launch_flops / (peaks["bf16_tflops"] * 1e12)
+    compute_floor = per_launch_flops / (peak_tc * 1e12)
     hbm_floor = per_launch_bytes / (peaks["hbm_gbs"] * 1e9)
     if compute_floor >= hbm_floor:
-        roof = {"bound": "tensor", "achieved": per_launch_flops / t_launch / 1e12, "peak": peaks["bf16_tflops"],
+        roof = {"bound": "tensor", "achieved": per_launch_flops / t_launch / 1e12, "peak": peak_tc,
                 "unit": "TFLOP/s"}
     else:
         roof = {"bound": "hbm", "achieved": per_launch_bytes / t_launch / 1e9, "peak": peaks["hbm_gbs"],
                 "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = recorded_traffic(w)
-    roof["peak_source"] = peaks["source"] + " (burst)"
+    roof["peak_source"] = peaks["source"] + peak_note
     roof["frac_of_roofline_time"] = max(compute_floor, hbm_floor) / t_launch
 
     cpu = None
@@ -464,19 +498,20 @@ def run_ours(args, w):
         if w.backward:
             f, dt, desc, threads = oracle_sample_bwd(w, q, k, v, dout, kl, target_s=args.cpu_seconds)
         else:
-            f, dt, desc, threads = oracle_sample(w, q, k, v, kl, target_s=args.cpu_seconds)
+            f, dt, desc, threads = oracle_sample(w, q, k, v, kl, target_s=args.cpu_seconds, scales=scales)
         cpu = {"value": f / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc,
                "seconds": dt}
 
     result = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "vs_baseline": None, "dtype": "e4m3" if w.fp8 else "bf16", "data": "synthetic",
         "config": {"workload": f"{w.name}: B{w.B} Hq{w.Hq} Hkv{w.Hkv} Nq{w.Nq} Nk{w.Nk} d{w.d}"
-                               f"{' causal' if w.is_causal else ''}",
+                               f"{' causal' if w.is_causal else ''}{' fp8 e4m3' if w.fp8 else ''}",
                    "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Nq": w.Nq, "Nk": w.Nk, "d": w.d,
                    "is_causal": w.is_causal, "key_lens": w.key_lens,
-                   "entry_point": ("attn_bwd" if w.backward else "attn_fwd_splitkv" if w.split_kv else
+                   "entry_point": ("attn_fwd_fp8" if w.fp8 else "attn_bwd" if w.backward else
+                                   "attn_fwd_splitkv" if w.split_kv else
                                    "attn_fwd_mod" if (w.softcap or w.mask2d) else "attn_fwd"),
                    "softcap": w.softcap, "mask2d": w.mask2d,
                    "flops_per_step": flops, "parallelism": f"independent batch per GPU x{world}",
@@ -504,7 +539,13 @@ def run_reference(args, w):
         return  # rank 0 alone runs the CPU oracle
     import torch
     from workloads import make_inputs
-    q, k, v, kl = make_inputs(w, device="cpu")
+    scales = None
+    if w.fp8:
+        from workloads import make_fp8_inputs
+        q, k, v, *scales = make_fp8_inputs(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, seed=w.seed)
+        kl = None
+    else:
+        q, k, v, kl = make_inputs(w, device="cpu")
     do = None
     if w.backward:
         from workloads import make_qkv
@@ -516,7 +557,7 @@ def run_reference(args, w):
         if w.backward:
             f, dt, desc, threads = oracle_sample_bwd(w, q, k, v, do, kl, target_s=per_step)
         else:
-            f, dt, desc, threads = oracle_sample(w, q, k, v, kl, target_s=per_step)
+            f, dt, desc, threads = oracle_sample(w, q, k, v, kl, target_s=per_step, scales=scales)
         if i >= warmup:
             times.append(dt)
             flops_total += f

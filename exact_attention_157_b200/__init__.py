@@ -38,7 +38,7 @@ ATTN_ERR_SCRATCH = 7
 NOALLOC_SCRATCH_BYTES = 16 << 20  # ATTN_NOALLOC_SCRATCH_BYTES
 
 # Every symbol include/attn.h declares.
-EXPORTED = ("attn_fwd", "attn_fwd_mod", "attn_bwd_plan", "attn_bwd", "attn_splitkv_plan", "attn_fwd_splitkv", "attn_fwd_splitkv_noalloc",
+EXPORTED = ("attn_fwd", "attn_fwd_mod", "attn_fwd_fp8", "attn_bwd_plan", "attn_bwd", "attn_splitkv_plan", "attn_fwd_splitkv", "attn_fwd_splitkv_noalloc",
             "attn_check_device_status", "attn_set_wait_timeout_ns", "attn_selftest_timeout",
             "attn_status_string", "attn_last_cuda_error", "attn_version")
 
@@ -89,6 +89,8 @@ def lib() -> ctypes.CDLL:
             L.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, vp, vp, vp]
             L.attn_fwd_mod.restype = i
             L.attn_fwd_mod.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, ctypes.POINTER(AttnScoreMod), vp]
+            L.attn_fwd_fp8.restype = i
+            L.attn_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, vp]
             L.attn_bwd_plan.restype = i
             L.attn_bwd_plan.argtypes = [i, i, i, ctypes.POINTER(ctypes.c_size_t)]
             L.attn_bwd.restype = i
@@ -149,6 +151,13 @@ def attn_fwd_mod(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, is_causal, key
     return int(lib().attn_fwd_mod(q, k, v, out, lse, int(B), int(Hq), int(Hkv), int(Nq), int(Nk), int(d),
                                   float(scale), int(bool(is_causal)), key_lens,
                                   None if mod is None else ctypes.byref(mod), stream))
+
+
+def attn_fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, is_causal,
+                 key_lens=None, stream=None) -> int:
+    """The C FP8 entry point with raw device pointers (ints); returns the status code."""
+    return int(lib().attn_fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, out, lse, int(B), int(Hq), int(Hkv),
+                                  int(Nq), int(Nk), int(d), float(scale), int(bool(is_causal)), key_lens, stream))
 
 
 def attn_bwd_plan(B, Hq, Nq):
@@ -315,6 +324,56 @@ def attention(q, k, v, *, scale: float | None = None, is_causal: bool = False, k
                           workspace.numel() * workspace.element_size(), _stream_handle(stream))
     if st != ATTN_OK:
         raise AttnError(st, "attn_fwd_splitkv")
+    return out, lse
+
+
+def attention_fp8(q8, k8, v8, q_scale, k_scale, v_scale, *, scale: float | None = None, is_causal: bool = False,
+                  key_lens=None, out=None, lse=None, return_lse: bool = True, stream=None):
+    """attn_fwd_fp8 on CUDA tensors: q8 [B, Hq, Nq, 128], k8/v8 [B, Hkv, Nk, 128]
+    (uint8 or float8_e4m3fn, contiguous), scales fp32 [B, H, ceil(N / 128)].
+    Returns (out bf16 [B, Hq, Nq, 128], lse or None)."""
+    import torch
+
+    def codes(name, t):
+        if not isinstance(t, torch.Tensor) or t.device.type != "cuda" or t.dim() != 4 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous 4-D CUDA tensor")
+        if t.dtype == torch.float8_e4m3fn:
+            return t.view(torch.uint8)
+        if t.dtype != torch.uint8:
+            raise TypeError(f"{name} must hold E4M3 codes (uint8 or float8_e4m3fn)")
+        return t
+
+    q8, k8, v8 = codes("q8", q8), codes("k8", k8), codes("v8", v8)
+    B, Hq, Nq, d = q8.shape
+    Bk, Hkv, Nk, dk = k8.shape
+    if Bk != B or dk != d or tuple(v8.shape) != tuple(k8.shape):
+        raise ValueError("q8, k8, v8 shapes disagree")
+    for name, t, h, n in (("q_scale", q_scale, Hq, Nq), ("k_scale", k_scale, Hkv, Nk), ("v_scale", v_scale, Hkv, Nk)):
+        if (not isinstance(t, torch.Tensor) or t.dtype != torch.float32 or t.device != q8.device
+                or not t.is_contiguous() or tuple(t.shape) != (B, h, (n + 127) // 128)):
+            raise ValueError(f"{name} must be a contiguous fp32 CUDA tensor of shape {(B, h, (n + 127) // 128)}")
+    if out is None:
+        out = torch.empty((B, Hq, Nq, d), dtype=torch.bfloat16, device=q8.device)
+    else:
+        _check_bf16_cuda("out", out, 4)
+        if tuple(out.shape) != (B, Hq, Nq, d):
+            raise ValueError("out has the wrong shape")
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q8.device)
+    if lse is not None and (lse.dtype != torch.float32 or not lse.is_contiguous()
+                            or tuple(lse.shape) != (B, Hq, Nq)):
+        raise ValueError("lse must be a contiguous fp32 [B, Hq, Nq] tensor")
+    kl_ptr = None
+    if key_lens is not None:
+        if key_lens.dtype != torch.int32 or key_lens.device != q8.device or key_lens.numel() != B:
+            raise ValueError("key_lens must be an int32 CUDA tensor with B entries")
+        key_lens = key_lens.contiguous()
+        kl_ptr = key_lens.data_ptr()
+    st = attn_fwd_fp8(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), q_scale.data_ptr(), k_scale.data_ptr(),
+                      v_scale.data_ptr(), out.data_ptr(), None if lse is None else lse.data_ptr(), B, Hq, Hkv, Nq,
+                      Nk, d, 0.0 if scale is None else float(scale), is_causal, kl_ptr, _stream_handle(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd_fp8")
     return out, lse
 
 

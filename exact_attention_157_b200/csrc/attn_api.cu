@@ -54,17 +54,20 @@ attn_status_t cuda_fail(cudaError_t e) {
 // 8 K/V slots (128 KB).
 constexpr int kSlots128 = 5, kQStages128 = 1;
 constexpr int kSlots64 = 8, kQStages64 = 2;
+// FP8 (d = 128): 16 KB tiles, so two Q buffers and 8 K/V slots
+constexpr int kSlotsF8 = 8, kQStagesF8 = 2;
+using SmemF8 = SmemPP<128, kSlotsF8, kQStagesF8, 1>;
 
 template <int D, int NSLOT, int QS, bool M>
 cudaError_t set_pp_attrs() {
     constexpr int kSmem = SmemPP<D, NSLOT, QS>::kAlloc;
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_pp_kernel<D, NSLOT, QS, M, false, false>,
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_pp_kernel<D, NSLOT, QS, M, false, false, false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(attn_fwd_pp_kernel<D, NSLOT, QS, M, true, false>,
+    e = cudaFuncSetAttribute(attn_fwd_pp_kernel<D, NSLOT, QS, M, true, false, false>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess || M) return e;
-    return cudaFuncSetAttribute(attn_fwd_pp_kernel<D, NSLOT, QS, false, false, true>,
+    return cudaFuncSetAttribute(attn_fwd_pp_kernel<D, NSLOT, QS, false, false, true, false>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
 }
 
@@ -122,6 +125,9 @@ attn_status_t device_setup(int* dev_out) {
     if ((e = set_pp_attrs<128, kSlots128, kQStages128, true>()) != cudaSuccess) return cuda_fail(e);
     if ((e = set_pp_attrs<64, kSlots64, kQStages64, false>()) != cudaSuccess) return cuda_fail(e);
     if ((e = set_pp_attrs<64, kSlots64, kQStages64, true>()) != cudaSuccess) return cuda_fail(e);
+    if ((e = cudaFuncSetAttribute(attn_fwd_pp_kernel<128, kSlotsF8, kQStagesF8, false, false, false, true>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, SmemF8::kAlloc)) != cudaSuccess)
+        return cuda_fail(e);
     if ((e = set_bwd_attrs<128>()) != cudaSuccess) return cuda_fail(e);
     if ((e = set_decode_attrs<128>()) != cudaSuccess) return cuda_fail(e);
     if ((e = set_decode_attrs<64>()) != cudaSuccess) return cuda_fail(e);
@@ -134,12 +140,13 @@ attn_status_t device_setup(int* dev_out) {
 // 3-D map over a [heads, rows, d] bf16 tensor, box = 64 columns x 128 rows x 1,
 // 128-byte swizzle (the layout the UMMA shared-memory descriptors expect).
 attn_status_t encode_map(CUtensorMap* map, const void* base, int d, int rows, long long heads,
-                         unsigned box_rows = 128u) {
+                         unsigned box_rows = 128u, bool fp8 = false) {
+    const cuuint64_t eb = fp8 ? 1u : 2u;  // bytes per element; a box row is 128 bytes either way
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(heads)};
-    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2u, static_cast<cuuint64_t>(rows) * d * 2u};
-    cuuint32_t box[3] = {64u, box_rows, 1u};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * eb, static_cast<cuuint64_t>(rows) * d * eb};
+    cuuint32_t box[3] = {fp8 ? 128u : 64u, box_rows, 1u};
     cuuint32_t estr[3] = {1u, 1u, 1u};
-    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+    CUresult r = g_encode(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
@@ -154,11 +161,12 @@ cudaError_t launch_pp(const CUtensorMap& tq, const CUtensorMap& tk, const CUtens
                       const FwdParams& p, unsigned grid, cudaStream_t stream) {
     constexpr int kSmem = SmemPP<D, NSLOT, QS>::kAlloc;
     if (p.n_splits > 1)
-        attn_fwd_pp_kernel<D, NSLOT, QS, M, true, false><<<grid, kPPThreads, kSmem, stream>>>(tq, tk, tv, to, p);
+        attn_fwd_pp_kernel<D, NSLOT, QS, M, true, false, false><<<grid, kPPThreads, kSmem, stream>>>(tq, tk, tv, to, p);
     else if (!M && (p.softcap_on || p.m2_kind != 0))
-        attn_fwd_pp_kernel<D, NSLOT, QS, false, false, true><<<grid, kPPThreads, kSmem, stream>>>(tq, tk, tv, to, p);
+        attn_fwd_pp_kernel<D, NSLOT, QS, false, false, true, false><<<grid, kPPThreads, kSmem, stream>>>(tq, tk, tv, to,
+                                                                                                       p);
     else
-        attn_fwd_pp_kernel<D, NSLOT, QS, M, false, false><<<grid, kPPThreads, kSmem, stream>>>(tq, tk, tv, to, p);
+        attn_fwd_pp_kernel<D, NSLOT, QS, M, false, false, false><<<grid, kPPThreads, kSmem, stream>>>(tq, tk, tv, to, p);
     return cudaGetLastError();
 }
 
@@ -331,6 +339,8 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, f
     p.m2_w = 1;
     p.m2_size = 1;
     p.m2_shift = 0;
+    p.q_scale = p.k_scale = p.v_scale = nullptr;
+    p.nqb = p.nkb = 0;
     if (use_mod) {
         if (mod->softcap > 0.0f) {
             // the kernel turns each raw score into the base-2 logit cap*log2(e)*tanh(scale*s/cap),
@@ -549,6 +559,63 @@ int attn_last_cuda_error(void) { return g_last_cuda_error.load(); }
 int attn_version(void) { return kVersion; }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------
+// FP8 forward.
+extern "C" attn_status_t attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_scale,
+                                      const float* k_scale, const float* v_scale, void* out, float* lse,
+                                      int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                                      float scale, int is_causal, const int32_t* key_lens, void* stream) {
+    if (q8 == nullptr || k8 == nullptr || v8 == nullptr || q_scale == nullptr || k_scale == nullptr ||
+        v_scale == nullptr || out == nullptr)
+        return ATTN_ERR_INVALID_ARG;
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nk <= 0 || d <= 0 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+    if (!(std::isfinite(scale)) || scale < 0.0f) return ATTN_ERR_INVALID_ARG;
+    if (d != 128) return ATTN_ERR_UNSUPPORTED;
+    if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8) || !aligned16(out) ||
+        (reinterpret_cast<uintptr_t>(q_scale) & 3u) || (reinterpret_cast<uintptr_t>(k_scale) & 3u) ||
+        (reinterpret_cast<uintptr_t>(v_scale) & 3u) || (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) ||
+        (key_lens != nullptr && (reinterpret_cast<uintptr_t>(key_lens) & 3u)))
+        return ATTN_ERR_ALIGNMENT;
+    int dev = 0;
+    attn_status_t st = device_setup(&dev);
+    if (st != ATTN_OK) return st;
+    const float scale_eff = scale == 0.0f ? static_cast<float>(1.0 / std::sqrt(static_cast<double>(d))) : scale;
+    FwdParams p{};
+    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Nq = Nq; p.Nk = Nk;
+    p.group = Hq / Hkv;
+    p.scale_log2 = static_cast<float>(static_cast<double>(scale_eff) * 1.4426950408889634);
+    p.is_causal = is_causal ? 1 : 0;
+    p.key_lens = key_lens;
+    p.lse = lse;
+    p.out = out;
+    p.n_splits = 1;
+    p.split_keys = (Nk + kBN - 1) / kBN * kBN;
+    p.m2_w = p.m2_size = 1;
+    p.q_scale = q_scale;
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
+    p.nqb = (Nq + kBM - 1) / kBM;
+    p.nkb = (Nk + kBN - 1) / kBN;
+    p.timeout_ns = g_timeout_ns.load();
+    p.epoch = next_epoch();
+    CUtensorMap tq, tk, tv;
+    if ((st = encode_map(&tq, q8, d, Nq, static_cast<long long>(B) * Hq, 128u, true)) != ATTN_OK) return st;
+    if ((st = encode_map(&tk, k8, d, Nk, static_cast<long long>(B) * Hkv, 128u, true)) != ATTN_OK) return st;
+    if ((st = encode_map(&tv, v8, d, Nk, static_cast<long long>(B) * Hkv, 128u, true)) != ATTN_OK) return st;
+    p.n_qtiles = static_cast<int>((static_cast<long long>(Nq) + 2 * kBM - 1) / (2 * kBM));
+    const long long n_units = static_cast<long long>(B) * Hq * p.n_qtiles;
+    if (n_units > (1LL << 30)) return ATTN_ERR_INVALID_ARG;
+    const int sms = g_dev[dev].sm_count > 0 ? g_dev[dev].sm_count : 1;
+    p.unit_run = (is_causal && n_units >= 2LL * sms) ? 2 : 1;
+    const long long want = (n_units + p.unit_run - 1) / p.unit_run;
+    const unsigned g = static_cast<unsigned>(want < sms ? want : sms);
+    attn_fwd_pp_kernel<128, kSlotsF8, kQStagesF8, false, false, false, true>
+        <<<g, kPPThreads, SmemF8::kAlloc, static_cast<cudaStream_t>(stream)>>>(tq, tk, tv, tq, p);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e);
+    return ATTN_OK;
+}
 
 // ------------------------------------------------------------------------
 // Backward pass.

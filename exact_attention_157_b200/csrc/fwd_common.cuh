@@ -11,6 +11,11 @@ constexpr int kBM = 128;          // query rows per tile (= TMEM lanes)
 constexpr int kBN = 128;          // keys per block
 constexpr int kTmemCols = 512;
 constexpr float kLazyTau = 8.0f;  // rescale only when the max grows by > 2^8
+// FP8 probabilities: a tighter threshold (stale-max factor at most 2^2) frees six
+// binades of the E4M3 range, used to store P * 2^6; the largest stored value is
+// then 2^8 <= 448 and normal E4M3 values reach down to 2^-12 of the row max.
+constexpr float kLazyTauF8 = 2.0f;
+constexpr float kPShiftF8 = 6.0f;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -44,6 +49,11 @@ struct FwdParams {
     float sc_in;   // 2 * scale * log2(e) / cap: base-2 exponent of e^(2x / cap) per raw score
     float sc_out;  // cap * log2(e)
     int m2_kind, m2_w, m2_size, m2_shift;
+    // FP8 instantiation: per-128-row block scales of Q [B*Hq][nqb] and K, V [B*Hkv][nkb]
+    const float* q_scale;
+    const float* k_scale;
+    const float* v_scale;
+    int nqb, nkb;
     unsigned long long timeout_ns;
     unsigned int epoch;  // launch id for the launch-wide abort (never 0)
 };

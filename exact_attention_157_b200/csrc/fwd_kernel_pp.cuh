@@ -54,11 +54,11 @@ constexpr int kRegsSoftmax = 200;
 constexpr int kRegsControl = 104;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl <= kPPThreads * 168, "register split");
 
-template <int D, int NSLOT, int QS>
+template <int D, int NSLOT, int QS, int EB = 2>  // EB: bytes per Q/K/V element (2: bf16, 1: FP8)
 struct SmemPP {
-    static constexpr int kChunks = D / 64;
+    static constexpr int kChunks = D * EB / 128;              // 128-byte column chunks of a row
     static constexpr int kChunkBytes = 128 * 128;
-    static constexpr int kTileBytes = kChunks * kChunkBytes;  // 128 rows x D bf16
+    static constexpr int kTileBytes = kChunks * kChunkBytes;  // 128 rows x D elements
     static constexpr int kQBuf = 2 * kTileBytes;              // Q_A then Q_B of one unit
     static constexpr int kQ = 0;                              // QS buffers
     static constexpr int kRing = QS * kQBuf;
@@ -186,12 +186,13 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int s, int kv_le
     return x;
 }
 
-template <int D, int NSLOT, int QS, bool HAS_MASK, bool SPLIT, bool MOD>
+template <int D, int NSLOT, int QS, bool HAS_MASK, bool SPLIT, bool MOD, bool FP8>
 __global__ void __launch_bounds__(kPPThreads, 1)
 attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                    const FwdParams p) {
-    using L = SmemPP<D, NSLOT, QS>;
+    using L = SmemPP<D, NSLOT, QS, FP8 ? 1 : 2>;
+    constexpr int kElemsPerChunk = FP8 ? 128 : 64;  // TMA box columns
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw_base = smem_u32(smem_raw);
     const uint32_t sbase = (raw_base + 1023u) & ~1023u;
@@ -278,7 +279,7 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     #pragma unroll
                     for (int c = 0; c < L::kChunks; ++c)
                         tma_load_3d(sbase + L::kQ + qb * L::kQBuf + t * L::kTileBytes + c * L::kChunkBytes, &tm_q,
-                                    bar(L::QFULL + qb), c * 64, x.q0 + t * kBM, x.bh);
+                                    bar(L::QFULL + qb), c * kElemsPerChunk, x.q0 + t * kBM, x.bh);
                 }
                 ++q_loads[qb];
                 for (int i = 0; i < 2 * n_max; ++i, ++i_glob) {  // K_0, V_0, K_1, V_1, ...
@@ -292,7 +293,7 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     #pragma unroll
                     for (int c = 0; c < L::kChunks; ++c)
                         tma_load_3d(sbase + L::kRing + s * L::kTileBytes + c * L::kChunkBytes, map, bar(L::FULL + s),
-                                    c * 64, (x.j_lo + (i >> 1)) * kBN, x.bhk);
+                                    c * kElemsPerChunk, (x.j_lo + (i >> 1)) * kBN, x.bhk);
                     uses[s] = use + 1;
                 }
             }
@@ -309,8 +310,12 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         // The whole warp runs this loop (warp-uniform control flow and operands);
         // one elected lane issues each tcgen05 instruction.
         {
-            constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kBN, false);
-            constexpr uint32_t kIdescO = idesc_bf16_f32(kBM, D, true);
+            constexpr uint32_t kIdescS = FP8 ? idesc_e4m3_f32(kBM, kBN, false) : idesc_bf16_f32(kBM, kBN, false);
+            constexpr uint32_t kIdescO = FP8 ? idesc_e4m3_f32(kBM, D, true) : idesc_bf16_f32(kBM, D, true);
+            // K steps of one MMA: 16 bf16 or 32 FP8 elements, 32 bytes either way
+            constexpr int kSSteps = FP8 ? D / 32 : D / 16;
+            constexpr int kPvKeys = FP8 ? 32 : 16;          // keys per PV step
+            constexpr int kPvSteps = (kBN / 2) / kPvKeys;   // per half of P
             int q_loads[QS];
             #pragma unroll
             for (int q = 0; q < QS; ++q) q_loads[q] = 0;
@@ -335,10 +340,14 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     const uint32_t q_addr = qbuf + t * L::kTileBytes;
                     const uint32_t k_addr = sbase + L::kRing + slot_of(2 * j) * L::kTileBytes;
                     #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
+                    for (int kk = 0; kk < kSSteps; ++kk) {
                         const uint32_t off = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
-                        mma_ss_warp(tmem + t * 128, smem_desc_sw128(q_addr + off, 16, 1024),
-                               smem_desc_sw128(k_addr + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+                        if constexpr (FP8)
+                            mma_ss_f8_warp(tmem + t * 128, smem_desc_sw128(q_addr + off, 16, 1024),
+                                           smem_desc_sw128(k_addr + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+                        else
+                            mma_ss_warp(tmem + t * 128, smem_desc_sw128(q_addr + off, 16, 1024),
+                                        smem_desc_sw128(k_addr + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
                     }
                     mma_commit_warp(bar(L::SFULL + t));
                 };
@@ -348,10 +357,13 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     const uint32_t o_tmem = tmem + L::kColO + t * D;
                     const uint32_t p_tmem = tmem + t * 128;
                     #pragma unroll
-                    for (int k4 = 0; k4 < kBN / 32; ++k4) {
-                        const int kk = half * (kBN / 32) + k4;
-                        mma_ts_warp(o_tmem, p_tmem + kk * 8, smem_desc_sw128(v_addr + kk * 2048, L::kChunkBytes, 1024),
-                               kIdescO, (j > 0 || kk > 0) ? 1u : 0u);
+                    for (int k4 = 0; k4 < kPvSteps; ++k4) {
+                        const int kk = half * kPvSteps + k4;
+                        const uint64_t vd = smem_desc_sw128(v_addr + kk * kPvKeys * 128, L::kChunkBytes, 1024);
+                        if constexpr (FP8)
+                            mma_ts_f8_warp(o_tmem, p_tmem + kk * 8, vd, kIdescO, (j > 0 || kk > 0) ? 1u : 0u);
+                        else
+                            mma_ts_warp(o_tmem, p_tmem + kk * 8, vd, kIdescO, (j > 0 || kk > 0) ? 1u : 0u);
                     }
                 };
                 ok = mbar_wait_warp(bar(L::QFULL + qb), q_loads[qb] & 1, limit, abort_flag, p.epoch, kRoleMma, 20) &&
@@ -435,6 +447,17 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             if constexpr (MOD) {
                 if (p.m2_kind != 0) rq = rect_2d(p, q_idx);
             }
+            // FP8: this tile's Q block scale and the largest V block scale of the head
+            // (P is stored as 2^6 * P * sv_block / sv_max so that one O accumulator
+            // serves every key block; O is multiplied by 2^-6 sv_max at the end)
+            float sq_t = 1.0f, sv_max = 1.0f;
+            if constexpr (FP8) {
+                if (q0_t < p.Nq) sq_t = __ldg(p.q_scale + static_cast<long long>(x.bh) * p.nqb + q0_t / kBM);
+                const float* vsr = p.v_scale + static_cast<long long>(x.bhk) * p.nkb;
+                sv_max = 0.0f;
+                for (int i = 0; i < p.nkb; ++i) sv_max = fmaxf(sv_max, __ldg(vsr + i));
+                if (!(sv_max > 0.0f)) sv_max = 1.0f;
+            }
             const float* mask_row = nullptr;
             if constexpr (HAS_MASK) {
                 if (q_idx < p.Nq)
@@ -455,6 +478,17 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 float* s = reinterpret_cast<float*>(sr);
                 const int j0 = (x.j_lo + j) * kBN;
                 const bool boundary = (j0 + kBN > kv_len) || (p.is_causal && j0 + kBN - 1 > q0_t);
+                // score scale of this block (FP8: times the Q and K block scales) and, for
+                // FP8, log2 of this block's V scale relative to the head's largest
+                float cl = c_log2, lr = 0.0f, inv_r = 1.0f;
+                if constexpr (FP8) {
+                    const long long kb = static_cast<long long>(x.bhk) * p.nkb + (x.j_lo + j);
+                    const float svb = __ldg(p.v_scale + kb);
+                    cl = c_log2 * sq_t * __ldg(p.k_scale + kb);
+                    lr = svb > 0.0f ? __log2f(svb / sv_max) + kPShiftF8 : -INFINITY;
+                    inv_r = svb > 0.0f ? sv_max / svb * exp2f(-kPShiftF8) : 0.0f;
+                }
+                const uint64_t cl2 = pack_f32x2(cl, cl);
 
                 // keys c >= lim of this block are masked (padding / past the diagonal)
                 int lim = kv_len - j0;
@@ -510,7 +544,7 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     } else {
                         #pragma unroll
                         for (int c = 0; c < kN / 2; ++c) {
-                            const uint64_t xv = ffma2(pack_f32x2(sh[2 * c], sh[2 * c + 1]), c2, ns2);
+                            const uint64_t xv = ffma2(pack_f32x2(sh[2 * c], sh[2 * c + 1]), cl2, ns2);
                             sh[2 * c] = ex2_approx(lo_f32(xv));
                             sh[2 * c + 1] = ex2_approx(hi_f32(xv));
                         }
@@ -543,7 +577,7 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         mx = fmaxf(mx, s[c]);
                     }
                 } else {
-                    mx = row_max() * c_log2;
+                    mx = row_max() * cl;
                 }
 
                 // Lazy correction, decided per row: a row moves its reference max only when
@@ -553,7 +587,7 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 // sum_{i<j} P_i V_i here (S_t(j) was issued after PV_t(j-1)); the rescale
                 // of O_t itself is done after the first half of P_t is stored (fewer live
                 // registers) and before the P0 arrive that lets PV_t(j) start.
-                const bool need = mx > m_used + kLazyTau;
+                const bool need = mx > m_used + (FP8 ? kLazyTauF8 : kLazyTau);
                 const bool warp_rescale = __any_sync(0xffffffffu, need) && j > 0;
                 float alpha = 1.0f;
                 if (need) {
@@ -562,10 +596,10 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     m_used = mx;
                 }
                 const float shift = (m_used == -INFINITY) ? 0.0f : m_used;
-                const uint64_t nshift2 = pack_f32x2(-shift, -shift);
+                const uint64_t nshift2 = pack_f32x2(lr - shift, lr - shift);
 
                 uint64_t acc0 = 0, acc1 = 0, acc2 = 0, acc3 = 0;  // packed partial sums
-                uint32_t pk[kBN / 4];
+                uint32_t pk[FP8 ? kBN / 8 : kBN / 4];
                 // row-sum terms and bf16 pairs of keys [64h, 64h + 64)
                 auto pack_half = [&](auto half_c) {
                     float* sh = s + decltype(half_c)::value * (kBN / 2);
@@ -578,7 +612,12 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                             case 2: acc2 = fadd2(acc2, e); break;
                             default: acc3 = fadd2(acc3, e); break;
                         }
-                        pk[c] = pack_bf16x2(sh[2 * c], sh[2 * c + 1]);
+                        if constexpr (FP8) {
+                            if ((c & 1) == 0)
+                                pk[c >> 1] = pack_e4m3x4(sh[2 * c], sh[2 * c + 1], sh[2 * c + 2], sh[2 * c + 3]);
+                        } else {
+                            pk[c] = pack_bf16x2(sh[2 * c], sh[2 * c + 1]);
+                        }
                     }
                 };
                 exp_keys(std::integral_constant<int, 0>{}, nshift2);
@@ -589,7 +628,10 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 // rescaled (if needed) before P0 releases the first PV.
                 auto store_half = [&](auto half_c) {
                     constexpr int h = decltype(half_c)::value;
-                    tmem_st32(s_tmem + h * 32, pk);
+                    if constexpr (FP8)
+                        tmem_st16(s_tmem + h * 16, pk);  // 4 E4M3 per column: 64 keys in 16 columns
+                    else
+                        tmem_st32(s_tmem + h * 32, pk);
                     if (h == 0 && warp_rescale) {
                         #pragma unroll
                         for (int c = 0; c < D / 32; ++c) {
@@ -610,7 +652,7 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 pack_half(std::integral_constant<int, 1>{});
                 store_half(std::integral_constant<int, 1>{});
                 const uint64_t acc = fadd2(fadd2(acc0, acc2), fadd2(acc1, acc3));
-                l_sum += lo_f32(acc) + hi_f32(acc);
+                l_sum += (lo_f32(acc) + hi_f32(acc)) * inv_r;
             }
 
             // ------------------------------------------------------------ epilogue
@@ -681,6 +723,41 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 }
                 if (do_epilogue && q_idx < p.Nq)
                     p.ws_lse[rs] = l_sum > 0.0f ? (m_used + __log2f(l_sum)) * kLn2 : -INFINITY;
+                named_barrier_sync(1 + t, 128);
+                if ((threadIdx.x & 127) == 0) release_q(qb);
+            } else if constexpr (FP8) {
+                // FP8: O = 2^-6 sv_max * acc / l, bf16, row by row (the FP8 Q buffer is too
+                // small to stage a bf16 tile)
+                const float scl = inv_l * sv_max * exp2f(-kPShiftF8);
+                uint16_t* orow = static_cast<uint16_t*>(p.out) + (static_cast<long long>(x.bh) * p.Nq + q_idx) * D;
+                #pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t o[32];
+                    if (n_blocks > 0 && do_epilogue) {
+                        tmem_ld32(o_tmem + c * 32, o);
+                        tmem_wait_ld();
+                    } else {
+                        #pragma unroll
+                        for (int v = 0; v < 32; ++v) o[v] = 0u;
+                    }
+                    if (c == D / 32 - 1) {
+                        tc_fence_before();
+                        mbar_arrive(bar(L::OEMPTY + t));
+                    }
+                    if (do_epilogue && q_idx < p.Nq) {
+                        uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+                        #pragma unroll
+                        for (int v = 0; v < 4; ++v)
+                            dst[v] = make_uint4(
+                                pack_bf16x2(__uint_as_float(o[8 * v]) * scl, __uint_as_float(o[8 * v + 1]) * scl),
+                                pack_bf16x2(__uint_as_float(o[8 * v + 2]) * scl, __uint_as_float(o[8 * v + 3]) * scl),
+                                pack_bf16x2(__uint_as_float(o[8 * v + 4]) * scl, __uint_as_float(o[8 * v + 5]) * scl),
+                                pack_bf16x2(__uint_as_float(o[8 * v + 6]) * scl, __uint_as_float(o[8 * v + 7]) * scl));
+                    }
+                }
+                if (do_epilogue && q_idx < p.Nq && p.lse != nullptr)
+                    p.lse[static_cast<long long>(x.bh) * p.Nq + q_idx] =
+                        l_sum > 0.0f ? (m_used + __log2f(l_sum)) * kLn2 : -INFINITY;
                 named_barrier_sync(1 + t, 128);
                 if ((threadIdx.x & 127) == 0) release_q(qb);
             } else {

@@ -235,6 +235,40 @@ attn_status_t attn_fwd_splitkv_noalloc(const void *q, const void *k, const void 
                                        int n_splits, void *stream);
 
 /*
+ * attn_fwd_fp8 -- attn_fwd on FP8 E4M3 inputs with one fp32 scale factor per
+ * 128-row block of every head; the output stays bf16.
+ *
+ * "FlashAttention technical analysis" (jsqmd.com/news/722897), sections 4.2
+ * and 6.3: Q, K and V enter the tensor cores as FP8, each block of rows with
+ * its own scale factor, and the softmax and the accumulators stay in higher
+ * precision.  The value computed is attn_fwd's on the dequantized inputs
+ *   Q[b,h,i,:] = q_scale[b,h,i/128] * e4m3(q8[b,h,i,:])   (likewise K, V),
+ * i.e. softmax(scale * Q K^T) V with per-row LSE.  Both products run on FP8
+ * tensor cores with fp32 accumulation; the block scales of Q and K scale each
+ * score block, and the probabilities enter the second product as E4M3 after
+ * being multiplied by v_scale(block) / max(v_scale of the head), the largest
+ * V scale being applied to the output once.  Rounding P to E4M3 (3 mantissa
+ * bits) bounds the error of an output element by about 2^-4 times
+ * sum_j P_ij |V_jc|, plus subnormal and bf16 output rounding.
+ *
+ * Layout, all device, contiguous:
+ *   q8   uint8 E4M3 [B, Hq, Nq, d]      k8, v8   uint8 E4M3 [B, Hkv, Nk, d]
+ *   q_scale fp32 [B, Hq, ceil(Nq/128)]   k_scale, v_scale fp32 [B, Hkv, ceil(Nk/128)]
+ *   out  bf16 [B, Hq, Nq, d]             lse  fp32 [B, Hq, Nq] or NULL
+ * Every scale must be positive and finite; the codes 0x7F and 0xFF (NaN) must
+ * not occur.  The kernel does not check either (a violation gives undefined
+ * values, never a fault).  q8, k8, v8 and out 16-byte aligned, scales and lse
+ * 4-byte aligned.  d must be 128.  scale, is_causal, key_lens: as attn_fwd;
+ * additive masks and split-KV are not offered on this path.
+ * Errors: as attn_fwd; ATTN_ERR_UNSUPPORTED for d != 128.
+ */
+attn_status_t attn_fwd_fp8(const void *q8, const void *k8, const void *v8,
+                           const float *q_scale, const float *k_scale, const float *v_scale,
+                           void *out, float *lse,
+                           int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                           float scale, int is_causal, const int32_t *key_lens, void *stream);
+
+/*
  * attn_bwd_plan -- device workspace bytes attn_bwd needs (host-only).  The
  * workspace holds two fp32 values per query row (D = rowsum(dO * O) and the
  * base-2 LSE), rows padded to a multiple of 128 per head.

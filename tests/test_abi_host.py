@@ -241,3 +241,23 @@ def test_bwd_validation_is_host_side(args, status):
               scale=0.0, is_causal=0, key_lens=None, workspace=A, workspace_bytes=1 << 20)
     kw.update(args)
     assert ea.attn_bwd(**kw) == status
+
+
+# ------------------------------------------------------------------- FP8
+@pytest.mark.parametrize("args,status", [
+    (dict(q8=0), ea.ATTN_ERR_INVALID_ARG),
+    (dict(v_scale=0), ea.ATTN_ERR_INVALID_ARG),
+    (dict(out=0), ea.ATTN_ERR_INVALID_ARG),
+    (dict(Hq=3, Hkv=2), ea.ATTN_ERR_INVALID_ARG),
+    (dict(Nk=0), ea.ATTN_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), ea.ATTN_ERR_INVALID_ARG),
+    (dict(d=64), ea.ATTN_ERR_UNSUPPORTED),
+    (dict(k8=A + 8), ea.ATTN_ERR_ALIGNMENT),
+    (dict(q_scale=A + 2), ea.ATTN_ERR_ALIGNMENT),
+    (dict(lse=A + 1), ea.ATTN_ERR_ALIGNMENT),
+])
+def test_fp8_validation_is_host_side(args, status):
+    kw = dict(q8=A, k8=A, v8=A, q_scale=A, k_scale=A, v_scale=A, out=A, lse=None, B=1, Hq=2, Hkv=2,
+              Nq=64, Nk=64, d=128, scale=0.0, is_causal=0)
+    kw.update(args)
+    assert ea.attn_fwd_fp8(**kw) == status

@@ -55,6 +55,7 @@ class Workload:
     softcap: float = 0.0    # > 0: soft-capped scores (attn_fwd_mod)
     mask2d: tuple | None = None  # ("neighborhood", W, R) or ("window", W, w, shift) (attn_fwd_mod)
     backward: bool = False  # the step is the backward pass (attn_bwd) of this shape
+    fp8: bool = False       # FP8 E4M3 inputs with per-128-row block scales (attn_fwd_fp8)
 
     @property
     def scale(self) -> float:
@@ -94,6 +95,8 @@ WORKLOADS = {
         Workload("long_bwd", 8, 32, 32, 4096, 4096, 128, seed=1008, backward=True),
         Workload("long_causal_bwd", 8, 32, 32, 4096, 4096, 128, is_causal=True, seed=1009, backward=True),
         Workload("prefill_gqa_bwd", 1, 32, 2, 16384, 16384, 128, is_causal=True, seed=1010, backward=True),
+        Workload("long_fp8", 8, 32, 32, 4096, 4096, 128, seed=1014, fp8=True),
+        Workload("long_causal_fp8", 8, 32, 32, 4096, 4096, 128, is_causal=True, seed=1015, fp8=True),
         Workload("vit3136_softcap", 8, 12, 12, 3136, 3136, 64, seed=1006, softcap=30.0),
         Workload("vit3136_neighborhood", 8, 12, 12, 3136, 3136, 64, seed=1007, mask2d=("neighborhood", 56, 5)),
     ]
@@ -116,13 +119,13 @@ def quantize_e4m3_blocks(x: torch.Tensor, block: int = 128):
     return y.to(torch.float8_e4m3fn).view(torch.uint8).contiguous(), scales.contiguous()
 
 
-def make_fp8_inputs(B, Hq, Hkv, Nq, Nk, d, seed):
-    """FP8 Q, K, V (codes and per-128-row scales) from the same N(0, 1) draws as
-    make_qkv (fp32 before rounding), on the CPU."""
-    g = torch.Generator().manual_seed(seed)
-    q = torch.randn((B, Hq, Nq, d), generator=g)
-    k = torch.randn((B, Hkv, Nk, d), generator=g)
-    v = torch.randn((B, Hkv, Nk, d), generator=g)
+def make_fp8_inputs(B, Hq, Hkv, Nq, Nk, d, seed, device="cpu"):
+    """FP8 Q, K, V (codes and per-128-row scales) from N(0, 1) fp32 draws of a
+    generator on ``device`` seeded with ``seed``."""
+    g = torch.Generator(device=device).manual_seed(int(seed))
+    q = torch.randn((B, Hq, Nq, d), generator=g, device=device)
+    k = torch.randn((B, Hkv, Nk, d), generator=g, device=device)
+    v = torch.randn((B, Hkv, Nk, d), generator=g, device=device)
     (q8, qs), (k8, ks), (v8, vs) = (quantize_e4m3_blocks(t) for t in (q, k, v))
     return q8, k8, v8, qs, ks, vs
 
