@@ -56,11 +56,11 @@ constexpr int kSlots128 = 5, kQStages128 = 1;
 constexpr int kSlots64 = 8, kQStages64 = 2;
 // FP8 (d = 128): 16 KB tiles, so two Q buffers and 8 K/V slots
 constexpr int kSlotsF8 = 8, kQStagesF8 = 2;
-using SmemF8 = SmemPP<128, kSlotsF8, kQStagesF8, 1>;
+using SmemF8 = SmemPPFor<128, kSlotsF8, kQStagesF8, true>;
 
 template <int D, int NSLOT, int QS, bool M>
 cudaError_t set_pp_attrs() {
-    constexpr int kSmem = SmemPP<D, NSLOT, QS>::kAlloc;
+    constexpr int kSmem = SmemPPFor<D, NSLOT, QS, false>::kAlloc;
     cudaError_t e = cudaFuncSetAttribute(attn_fwd_pp_kernel<D, NSLOT, QS, M, false, false, false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;
@@ -159,7 +159,7 @@ attn_status_t encode_map(CUtensorMap* map, const void* base, int d, int rows, lo
 template <int D, int NSLOT, int QS, bool M>
 cudaError_t launch_pp(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
                       const FwdParams& p, unsigned grid, cudaStream_t stream) {
-    constexpr int kSmem = SmemPP<D, NSLOT, QS>::kAlloc;
+    constexpr int kSmem = SmemPPFor<D, NSLOT, QS, false>::kAlloc;
     if (p.n_splits > 1)
         attn_fwd_pp_kernel<D, NSLOT, QS, M, true, false, false><<<grid, kPPThreads, kSmem, stream>>>(tq, tk, tv, to, p);
     else if (!M && (p.softcap_on || p.m2_kind != 0))

@@ -54,7 +54,8 @@ constexpr int kRegsSoftmax = 200;
 constexpr int kRegsControl = 104;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl <= kPPThreads * 168, "register split");
 
-template <int D, int NSLOT, int QS, int EB = 2>  // EB: bytes per Q/K/V element (2: bf16, 1: FP8)
+// EB: bytes per Q/K/V element (2: bf16, 1: FP8); PSMEM: P of both tiles in shared memory
+template <int D, int NSLOT, int QS, int EB = 2, bool PSMEM = false>
 struct SmemPP {
     static constexpr int kChunks = D * EB / 128;              // 128-byte column chunks of a row
     static constexpr int kChunkBytes = 128 * 128;
@@ -62,7 +63,9 @@ struct SmemPP {
     static constexpr int kQBuf = 2 * kTileBytes;              // Q_A then Q_B of one unit
     static constexpr int kQ = 0;                              // QS buffers
     static constexpr int kRing = QS * kQBuf;
-    static constexpr int kBars = kRing + NSLOT * kTileBytes;
+    static constexpr int kPS = kRing + NSLOT * kTileBytes;   // P_A, P_B: 128 rows x 128 one-byte keys
+    static constexpr int kPBytes = 128 * 128;
+    static constexpr int kBars = kPS + (PSMEM ? 2 * kPBytes : 0);
     // barrier indices
     static constexpr int QFULL = 0;                   // QS: Q buffer loaded
     static constexpr int QEMPTY = QS;                 // QS: Q buffer free (2 arrivals: both tiles' stores)
@@ -74,14 +77,21 @@ struct SmemPP {
     static constexpr int OFINAL = SFULL + 6;          // 2: last PV_t of a unit complete
     static constexpr int OEMPTY = SFULL + 8;          // 2: O_t read out by the epilogue (128 arrivals)
     static constexpr int MMAFIN = SFULL + 10;
-    static constexpr int kNumBars = MMAFIN + 1;
+    static constexpr int SFREE = SFULL + 11;          // 2: S_t(j) read into registers (128 arrivals)
+    static constexpr int PVDONE = SFULL + 13;         // 2: PV_t(j) complete (P_t buffer and O_t free)
+    static constexpr int kNumBars = PVDONE + 2;
     static constexpr int kMisc = kBars + 8 * kNumBars;
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;
     static constexpr int kColO = 256;
+    static constexpr int kColP = kColO + 2 * D;  // d = 64: P_A, P_B (64 columns each) after O
     static_assert(kColO + 2 * D <= kTmemCols, "TMEM budget");
     static_assert(kAlloc <= 232448, "shared memory budget");
 };
+
+// The layout of one kernel instantiation; the host sizes the launch with the same alias.
+template <int D, int NSLOT, int QS, bool FP8>
+using SmemPPFor = SmemPP<D, NSLOT, QS, FP8 ? 1 : 2, FP8>;
 
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
     float d;
@@ -108,6 +118,35 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
 
 __device__ __forceinline__ float lo_f32(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v)); }
 __device__ __forceinline__ float hi_f32(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
+
+// FP8 path: one pair of exponentials in every ATTN_F8_EXP_EMU is taken on the FMA
+// pipe instead of the special-function unit (0: none).  With FP8 products the
+// softmax warps, not the tensor cores, set the pace; one pair in four measured
+// best (one in two or three was slower: the extra FMA-pipe instructions then
+// cost more issue slots than the special-function unit frees).
+#ifndef ATTN_F8_EXP_EMU
+#define ATTN_F8_EXP_EMU 4
+#endif
+
+// 2^x for two fp32 values with FMA-pipe arithmetic only: x = n + f, n the nearest
+// integer (added to the exponent field) and 2^f for |f| <= 1/2 from a cubic whose
+// coefficients were fitted by the Remez exchange for least maximum relative error
+// (7.5e-5 on the interval).  x is clamped at -125 so that the result stays normal.
+__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t xv) {
+    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: x + kRound holds round(x) in its low bits
+    const float x0 = fmaxf(lo_f32(xv), -125.0f), x1 = fmaxf(hi_f32(xv), -125.0f);
+    const uint64_t x = pack_f32x2(x0, x1);
+    const uint64_t t = fadd2(x, pack_f32x2(kRound, kRound));
+    const uint64_t n = fadd2(t, pack_f32x2(-kRound, -kRound));
+    const uint64_t f = ffma2(n, pack_f32x2(-1.0f, -1.0f), x);
+    uint64_t q = ffma2(f, pack_f32x2(0.0551716685295105f, 0.0551716685295105f),
+                       pack_f32x2(0.2426111251115799f, 0.2426111251115799f));
+    q = ffma2(q, f, pack_f32x2(0.6932609677314758f, 0.6932609677314758f));
+    q = ffma2(q, f, pack_f32x2(0.9999280571937561f, 0.9999280571937561f));
+    const uint32_t r0 = static_cast<uint32_t>(q) + (static_cast<uint32_t>(t) << 23);
+    const uint32_t r1 = static_cast<uint32_t>(q >> 32) + (static_cast<uint32_t>(t >> 32) << 23);
+    return (static_cast<uint64_t>(r1) << 32) | r0;
+}
 
 // Everything about one work unit that every role derives identically.
 struct Unit {
@@ -191,8 +230,22 @@ __global__ void __launch_bounds__(kPPThreads, 1)
 attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                    const FwdParams p) {
-    using L = SmemPP<D, NSLOT, QS, FP8 ? 1 : 2>;
+    using L = SmemPPFor<D, NSLOT, QS, FP8>;
     constexpr int kElemsPerChunk = FP8 ? 128 : 64;  // TMA box columns
+    // Decoupled S and P: where P_t has a buffer of its own (FP8: shared memory; d = 64:
+    // spare tensor-memory columns), S_t(j+1) is issued as soon as the softmax has read
+    // S_t(j) into registers, so that it runs during softmax_t(j).  Otherwise (bf16,
+    // d = 128, tensor memory full) P_t(j) overwrites S_t(j) and S_t(j+1) waits for PV_t(j).
+    // (The additive-mask variant keeps the aliased form: it would spill registers.)
+    constexpr bool kDec = FP8 || (D == 64 && !HAS_MASK);
+    static_assert(!kDec || FP8 || L::kColP + 2 * 64 <= kTmemCols, "P columns");
+    // A launch whose dynamic shared memory does not hold this layout touches nothing.
+    uint32_t dyn_smem;
+    asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn_smem));
+    if (dyn_smem < static_cast<uint32_t>(L::kAlloc)) {
+        if (threadIdx.x == 0) record_error(kErrDevice, kRoleSoftmax, 34);
+        return;
+    }
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw_base = smem_u32(smem_raw);
     const uint32_t sbase = (raw_base + 1023u) & ~1023u;
@@ -214,7 +267,7 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         }
         for (int s = 0; s < NSLOT; ++s) {
             mbar_init(bar(L::FULL + s), 1);
-            mbar_init(bar(L::EMPTY + s), 1);
+            mbar_init(bar(L::EMPTY + s), kDec ? 2 : 1);  // decoupled: one MMA warp per tile releases
         }
         for (int t = 0; t < 2; ++t) {
             mbar_init(bar(L::SFULL + t), 1);
@@ -222,8 +275,10 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             mbar_init(bar(L::P1 + t), 128);
             mbar_init(bar(L::OFINAL + t), 1);
             mbar_init(bar(L::OEMPTY + t), 128);
+            mbar_init(bar(L::SFREE + t), 128);
+            mbar_init(bar(L::PVDONE + t), 1);
         }
-        mbar_init(bar(L::MMAFIN), 1);
+        mbar_init(bar(L::MMAFIN), kDec ? 2 : 1);
         *abort_flag = launch_aborted(p.epoch) ? 1 : 0;
         fence_mbar_init();
     }
@@ -248,7 +303,7 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
     if (warp >= 8) {
       asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" :: "n"(kRegsControl));
-      if (warp >= 10) {
+      if (warp == 11 || (warp == 10 && !kDec)) {
         // idle warps
       } else if (warp == 8) {
         // ============================== TMA producer ==============================
@@ -308,8 +363,10 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       } else {
         // =============================== MMA issuer ===============================
         // The whole warp runs this loop (warp-uniform control flow and operands);
-        // one elected lane issues each tcgen05 instruction.
+        // one elected lane issues each tcgen05 instruction.  Decoupled S and P:
+        // warp 9 serves tile A and warp 10 tile B, each with waits of its own.
         {
+            const int mt = kDec ? warp - 9 : 0;
             constexpr uint32_t kIdescS = FP8 ? idesc_e4m3_f32(kBM, kBN, false) : idesc_bf16_f32(kBM, kBN, false);
             constexpr uint32_t kIdescO = FP8 ? idesc_e4m3_f32(kBM, D, true) : idesc_bf16_f32(kBM, D, true);
             // K steps of one MMA: 16 bf16 or 32 FP8 elements, 32 bytes either way
@@ -321,6 +378,7 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             for (int q = 0; q < QS; ++q) q_loads[q] = 0;
             int i_glob = 0;      // K/V loads consumed so far
             int gp[2] = {0, 0};  // P_t blocks consumed so far (P0 / P1 phase)
+            int gf[2] = {0, 0};  // SFREE_t phases waited for (decoupled S and P)
             bool ok = true;
             int it = 0;
             int kv_next = unit_key_len(p, unit_seq(cta, 0, G, p.unit_run), n_units);
@@ -336,34 +394,39 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     return mbar_wait_warp(bar(L::FULL + slot_of(i)), ((i_glob + i) / NSLOT) & 1, limit, abort_flag,
                                      p.epoch, kRoleMma, site);
                 };
-                auto issue_s = [&](int t, int j) {
-                    const uint32_t q_addr = qbuf + t * L::kTileBytes;
-                    const uint32_t k_addr = sbase + L::kRing + slot_of(2 * j) * L::kTileBytes;
+                // S_t(j) = Q_t K_j^T in batches of four K steps (32 bytes each), then the
+                // SFULL_t commit and an optional second commit (0: none)
+                auto issue_s = [&](int t, int j, uint32_t bar_b = 0u) {
+                    const uint64_t qd = smem_desc_sw128(qbuf + t * L::kTileBytes, 16, 1024);
+                    const uint64_t kd = smem_desc_sw128(sbase + L::kRing + slot_of(2 * j) * L::kTileBytes, 16, 1024);
+                    static_assert(kSSteps == 4 || kSSteps == 8, "S steps");
                     #pragma unroll
-                    for (int kk = 0; kk < kSSteps; ++kk) {
-                        const uint32_t off = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
-                        if constexpr (FP8)
-                            mma_ss_f8_warp(tmem + t * 128, smem_desc_sw128(q_addr + off, 16, 1024),
-                                           smem_desc_sw128(k_addr + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
-                        else
-                            mma_ss_warp(tmem + t * 128, smem_desc_sw128(q_addr + off, 16, 1024),
-                                        smem_desc_sw128(k_addr + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+                    for (int g = 0; g < kSSteps / 4; ++g) {
+                        const uint64_t o = static_cast<uint64_t>(g * (L::kChunkBytes >> 4));  // descriptor units
+                        const bool last = g == kSSteps / 4 - 1;
+                        mma4_ss_warp<FP8>(tmem + t * 128, qd + o, qd + o + 2, qd + o + 4, qd + o + 6, kd + o, kd + o + 2,
+                                          kd + o + 4, kd + o + 6, kIdescS, g > 0 ? 1u : 0u,
+                                          last ? bar(L::SFULL + t) : 0u, last ? bar_b : 0u);
                     }
-                    mma_commit_warp(bar(L::SFULL + t));
                 };
-                // O_t += P_t(j)[:, keys 64 half .. +63] V_j[those keys, :]
-                auto issue_pv = [&](int t, int j, int half) {
+                // O_t += P_t(j)[:, keys of this half] V_j[those keys, :], then up to two commits
+                auto issue_pv = [&](int t, int j, int half, uint32_t bar_a = 0u, uint32_t bar_b = 0u) {
                     const uint32_t v_addr = sbase + L::kRing + slot_of(2 * j + 1) * L::kTileBytes;
                     const uint32_t o_tmem = tmem + L::kColO + t * D;
-                    const uint32_t p_tmem = tmem + t * 128;
-                    #pragma unroll
-                    for (int k4 = 0; k4 < kPvSteps; ++k4) {
-                        const int kk = half * kPvSteps + k4;
-                        const uint64_t vd = smem_desc_sw128(v_addr + kk * kPvKeys * 128, L::kChunkBytes, 1024);
-                        if constexpr (FP8)
-                            mma_ts_f8_warp(o_tmem, p_tmem + kk * 8, vd, kIdescO, (j > 0 || kk > 0) ? 1u : 0u);
-                        else
-                            mma_ts_warp(o_tmem, p_tmem + kk * 8, vd, kIdescO, (j > 0 || kk > 0) ? 1u : 0u);
+                    const int kk0 = half * kPvSteps;
+                    const uint64_t vd = smem_desc_sw128(v_addr + kk0 * kPvKeys * 128, L::kChunkBytes, 1024);
+                    constexpr uint64_t kVStep = kPvKeys * 128 / 16;  // one step of keys, descriptor units
+                    const uint32_t acc0 = (j > 0 || kk0 > 0) ? 1u : 0u;
+                    if constexpr (FP8) {
+                        // P_t in shared memory, 128-byte K-major rows (SW128), 32 keys per step
+                        static_assert(kPvSteps == 2, "PV steps");
+                        const uint64_t pd = smem_desc_sw128(sbase + L::kPS + t * L::kPBytes + kk0 * 32, 16, 1024);
+                        mma2_ss_warp<true>(o_tmem, pd, pd + 2, vd, vd + kVStep, kIdescO, acc0, bar_a, bar_b);
+                    } else {
+                        static_assert(kPvSteps == 4, "PV steps");
+                        const uint32_t pt = (kDec ? tmem + L::kColP + t * 64 : tmem + t * 128) + kk0 * 8;
+                        mma4_ts_warp(o_tmem, pt, pt + 8, pt + 16, pt + 24, vd, vd + kVStep, vd + 2 * kVStep,
+                                     vd + 3 * kVStep, kIdescO, acc0, bar_a, bar_b);
                     }
                 };
                 ok = mbar_wait_warp(bar(L::QFULL + qb), q_loads[qb] & 1, limit, abort_flag, p.epoch, kRoleMma, 20) &&
@@ -371,6 +434,57 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 ++q_loads[qb];
                 if (!ok) break;
                 tc_fence_after();
+                if constexpr (kDec) {
+                    // One tile: S_t(j+1) as soon as the softmax has read S_t(j) (SFREE),
+                    // then PV_t(j) by halves as P_t(j) is stored (P0, P1).  Every K/V load
+                    // of the unit is released once by each of the two warps: after the
+                    // products that read it, or, for blocks this tile does not use, once
+                    // the load has landed (so that the arrival cannot count towards the
+                    // slot's previous use).
+                    const int t = mt;
+                    const int nt = x.n_t[t];
+                    auto release_unused = [&](int i, unsigned site) -> bool {
+                        if (!wait_full(i, site)) return false;
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar(L::EMPTY + slot_of(i)));
+                        return true;
+                    };
+                    if (nt > 0) {
+                        issue_s(t, 0, bar(L::EMPTY + slot_of(0)));  // and K_0 released
+                    } else {
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar(L::EMPTY + slot_of(0)));
+                    }
+                    for (int j = 0; ok && j < nt; ++j) {
+                        if (j + 1 < nt) {
+                            if (!mbar_wait_warp(bar(L::SFREE + t), gf[t] & 1, limit, abort_flag, p.epoch, kRoleMma, 28) ||
+                                !wait_full(2 * j + 2, 29))
+                                { ok = false; break; }
+                            ++gf[t];
+                            tc_fence_after();
+                            issue_s(t, j + 1, bar(L::EMPTY + slot_of(2 * j + 2)));  // and K_{j+1} released
+                        }
+                        if (!mbar_wait_warp(bar(L::P0 + t), gp[t] & 1, limit, abort_flag, p.epoch, kRoleMma, 22))
+                            { ok = false; break; }
+                        if (j == 0 && it > 0 &&
+                            !mbar_wait_warp(bar(L::OEMPTY + t), (it - 1) & 1, limit, abort_flag, p.epoch, kRoleMma, 23))
+                            { ok = false; break; }
+                        if (!wait_full(2 * j + 1, 24)) { ok = false; break; }
+                        tc_fence_after();
+                        issue_pv(t, j, 0);
+                        if (!mbar_wait_warp(bar(L::P1 + t), gp[t] & 1, limit, abort_flag, p.epoch, kRoleMma, 27))
+                            { ok = false; break; }
+                        ++gp[t];
+                        tc_fence_after();
+                        // then PVDONE_t (OFINAL_t after the last block) and V_j released
+                        issue_pv(t, j, 1, bar((j + 1 < nt ? L::PVDONE : L::OFINAL) + t), bar(L::EMPTY + slot_of(2 * j + 1)));
+                    }
+                    // loads of the unit past this tile's last block, in load order
+                    for (int j = nt; ok && j < n_max; ++j) {
+                        if (j > 0 && !release_unused(2 * j, 36)) { ok = false; break; }
+                        if (!release_unused(2 * j + 1, 37)) { ok = false; break; }
+                    }
+                } else {
                 for (int t = 0; t < 2; ++t)
                     if (x.n_t[t] > 0) issue_s(t, 0);
                 mma_commit_warp(bar(L::EMPTY + slot_of(0)));  // K_0 released once both S(0) complete
@@ -395,23 +509,24 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                             { ok = false; break; }
                         ++gp[t];
                         tc_fence_after();
-                        issue_pv(t, j, 1);
-                        if (j + 1 < x.n_t[t]) {
+                        const bool last_t = j + 1 >= x.n_t[t];
+                        issue_pv(t, j, 1, last_t ? bar(L::OFINAL + t) : 0u);
+                        if (!last_t) {
                             if (!k_next_ready) {
                                 if (!wait_full(2 * j + 2, 25)) { ok = false; break; }
                                 k_next_ready = true;
                                 tc_fence_after();
                             }
                             issue_s(t, j + 1);
-                        } else {
-                            mma_commit_warp(bar(L::OFINAL + t));
                         }
                     }
                     if (!ok) break;
-                    mma_commit_warp(bar(L::EMPTY + slot_of(2 * j + 1)));  // V_j: both PV(j) issued above
-                    // K_{j+1}: the tile with n_t = n_max uses every block, so k_next_ready
-                    // holds exactly when j + 1 < n_max (each load is released once).
-                    if (k_next_ready) mma_commit_warp(bar(L::EMPTY + slot_of(2 * j + 2)));
+                    // V_j (both PV(j) issued above) and K_{j+1}: the tile with n_t = n_max uses
+                    // every block, so k_next_ready holds exactly when j + 1 < n_max (each load
+                    // is released once).
+                    mma_commit2_warp(bar(L::EMPTY + slot_of(2 * j + 1)),
+                                     k_next_ready ? bar(L::EMPTY + slot_of(2 * j + 2)) : 0u);
+                }
                 }
                 i_glob += 2 * n_max;
             }
@@ -430,6 +545,7 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         const float c_log2 = p.scale_log2;
         const uint64_t c2 = pack_f32x2(c_log2, c_log2);
         int gs = 0;       // S_t blocks consumed so far (SFULL phase)
+        int gpd = 0;      // PVDONE_t phases waited for (decoupled S and P)
         int n_final = 0;  // units with a PV for this tile so far (OFINAL phase)
         bool ok = true;
         int it = 0;
@@ -465,7 +581,23 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                                static_cast<long long>(q_idx) * p.msq;
             }
 
+            // FP8: the K and V block scales of the next key block, loaded one block ahead
+            const long long kb0 = static_cast<long long>(x.bhk) * p.nkb + x.j_lo;
+            float ks_next = 1.0f, vs_next = 1.0f;
+            if constexpr (FP8) {
+                if (n_blocks > 0) {
+                    ks_next = __ldg(p.k_scale + kb0);
+                    vs_next = __ldg(p.v_scale + kb0);
+                }
+            }
             for (int j = 0; j < n_blocks; ++j) {
+                const float ksb = ks_next, svb = vs_next;
+                if constexpr (FP8) {
+                    if (j + 1 < n_blocks) {
+                        ks_next = __ldg(p.k_scale + kb0 + j + 1);
+                        vs_next = __ldg(p.v_scale + kb0 + j + 1);
+                    }
+                }
                 bool got = mbar_wait(bar(L::SFULL + t), gs & 1, limit, abort_flag, p.epoch, kRoleSoftmax, 30);
                 if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
                 ++gs;
@@ -475,6 +607,13 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 for (int c = 0; c < kBN / 32; ++c)
                     tmem_ld32(s_tmem + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
                 tmem_wait_ld();
+                if constexpr (kDec) {
+                    // S_t(j) is in registers: the MMA warp may overwrite it with S_t(j+1)
+                    if (j + 1 < n_blocks) {
+                        tc_fence_before();
+                        mbar_arrive(bar(L::SFREE + t));
+                    }
+                }
                 float* s = reinterpret_cast<float*>(sr);
                 const int j0 = (x.j_lo + j) * kBN;
                 const bool boundary = (j0 + kBN > kv_len) || (p.is_causal && j0 + kBN - 1 > q0_t);
@@ -482,9 +621,7 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 // FP8, log2 of this block's V scale relative to the head's largest
                 float cl = c_log2, lr = 0.0f, inv_r = 1.0f;
                 if constexpr (FP8) {
-                    const long long kb = static_cast<long long>(x.bhk) * p.nkb + (x.j_lo + j);
-                    const float svb = __ldg(p.v_scale + kb);
-                    cl = c_log2 * sq_t * __ldg(p.k_scale + kb);
+                    cl = c_log2 * sq_t * ksb;
                     lr = svb > 0.0f ? __log2f(svb / sv_max) + kPShiftF8 : -INFINITY;
                     inv_r = svb > 0.0f ? sv_max / svb * exp2f(-kPShiftF8) : 0.0f;
                 }
@@ -542,11 +679,18 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         #pragma unroll
                         for (int c = 0; c < kN; ++c) sh[c] = ex2_approx(sh[c] - sft);
                     } else {
+                        constexpr int kEmu = FP8 ? ATTN_F8_EXP_EMU : 0;
                         #pragma unroll
                         for (int c = 0; c < kN / 2; ++c) {
                             const uint64_t xv = ffma2(pack_f32x2(sh[2 * c], sh[2 * c + 1]), cl2, ns2);
-                            sh[2 * c] = ex2_approx(lo_f32(xv));
-                            sh[2 * c + 1] = ex2_approx(hi_f32(xv));
+                            if (kEmu > 0 && c % (kEmu > 0 ? kEmu : 1) == kEmu - 1) {
+                                const uint64_t r = exp2_poly_x2(xv);
+                                sh[2 * c] = lo_f32(r);
+                                sh[2 * c + 1] = hi_f32(r);
+                            } else {
+                                sh[2 * c] = ex2_approx(lo_f32(xv));
+                                sh[2 * c + 1] = ex2_approx(hi_f32(xv));
+                            }
                         }
                     }
                 };
@@ -626,12 +770,31 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 // Keys 0..63, then 64..127: each half is stored and signalled on its own
                 // (P0, P1), so PV over the first half runs during the second half.  O_t is
                 // rescaled (if needed) before P0 releases the first PV.
-                auto store_half = [&](auto half_c) {
+                auto store_half = [&](auto half_c) -> bool {
                     constexpr int h = decltype(half_c)::value;
-                    if constexpr (FP8)
-                        tmem_st16(s_tmem + h * 16, pk);  // 4 E4M3 per column: 64 keys in 16 columns
-                    else
+                    if constexpr (kDec) {
+                        // PV_t(j-1) must be complete before P_t and O_t are touched
+                        if (h == 0 && j > 0) {
+                            const bool got_pv = mbar_wait(bar(L::PVDONE + t), gpd & 1, limit, abort_flag, p.epoch,
+                                                          kRoleSoftmax, 33);
+                            ++gpd;
+                            if (!__all_sync(0xffffffffu, got_pv)) return false;
+                            tc_fence_after();
+                        }
+                    }
+                    if constexpr (FP8) {
+                        // 64 keys = 64 bytes of this row, four 16-byte units at swizzled positions
+                        const uint32_t prow = sbase + L::kPS + t * L::kPBytes + row * 128;
+                        #pragma unroll
+                        for (int c4 = 0; c4 < 4; ++c4)
+                            st_shared_v4(prow + (((h * 4 + c4) ^ (row & 7)) << 4), pk[4 * c4], pk[4 * c4 + 1],
+                                         pk[4 * c4 + 2], pk[4 * c4 + 3]);
+                        fence_proxy_async_smem();
+                    } else if constexpr (kDec) {
+                        tmem_st32(lane_tmem + L::kColP + t * 64 + h * 32, pk);
+                    } else {
                         tmem_st32(s_tmem + h * 32, pk);
+                    }
                     if (h == 0 && warp_rescale) {
                         #pragma unroll
                         for (int c = 0; c < D / 32; ++c) {
@@ -646,8 +809,9 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     tmem_wait_st();
                     tc_fence_before();
                     mbar_arrive(bar((h == 0 ? L::P0 : L::P1) + t));
+                    return true;
                 };
-                store_half(std::integral_constant<int, 0>{});
+                if (!store_half(std::integral_constant<int, 0>{})) { ok = false; break; }
                 exp_keys(std::integral_constant<int, 1>{}, nshift2);
                 pack_half(std::integral_constant<int, 1>{});
                 store_half(std::integral_constant<int, 1>{});

@@ -70,6 +70,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking probe of a phase (acquire on success).
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok != 0;
+}
+
 // Launch-wide abort: the first role of a launch whose wait expires stores the
 // launch's epoch here, and every other wait of the same launch gives up at its
 // next poll.  A later launch carries a new epoch and is not affected.
@@ -171,6 +181,10 @@ __device__ __forceinline__ void bulk_wait_group0() {
 }
 
 // Make this thread's generic-proxy shared-memory writes visible to the async proxy.
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" :: "r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -259,6 +273,107 @@ __device__ __forceinline__ void mma_ts_f8_warp(uint32_t d_tmem, uint32_t a_tmem,
                  "setp.ne.b32 p, %4, 0;\n\t"
                  "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}"
                  :: "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
+
+// Batches of MMAs into one accumulator under one elected lane, followed by up
+// to two commits (a barrier address of 0 means none): one elect and one
+// predicate set-up for the whole batch.  The first MMA accumulates iff acc0 != 0,
+// the others always.  A operands: shared-memory descriptors (SS) or tensor-memory
+// addresses (TS); kind::f16 (bf16) or kind::f8f6f4 (E4M3).
+template <bool F8>
+__device__ __forceinline__ void mma4_ss_warp(uint32_t d, uint64_t a0, uint64_t a1, uint64_t a2, uint64_t a3,
+                                             uint64_t b0, uint64_t b1, uint64_t b2, uint64_t b3, uint32_t idesc,
+                                             uint32_t acc0, uint32_t bar_a = 0u, uint32_t bar_b = 0u) {
+    if constexpr (F8) {
+        asm volatile("{\n\t.reg .pred p, e, t, ca, cb;\n\t"
+                 "elect.sync _|e, 0xffffffff;\n\t"
+                 "setp.ne.b32 p, %10, 0;\n\t"
+                 "setp.eq.b32 t, %9, %9;\n\t"
+                 "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %5, %9, p;\n\t"
+                 "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %2, %6, %9, t;\n\t"
+                 "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %3, %7, %9, t;\n\t"
+                 "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %4, %8, %9, t;\n\t"
+                 "setp.ne.b32 ca, %11, 0;\n\tand.pred ca, ca, e;\n\t"
+                 "@ca tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%11];\n\t"
+                 "setp.ne.b32 cb, %12, 0;\n\tand.pred cb, cb, e;\n\t"
+                 "@cb tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%12];\n\t}"
+                     :: "r"(d), "l"(a0), "l"(a1), "l"(a2), "l"(a3), "l"(b0), "l"(b1), "l"(b2), "l"(b3), "r"(idesc), "r"(acc0), "r"(bar_a), "r"(bar_b) : "memory");
+    } else {
+        asm volatile("{\n\t.reg .pred p, e, t, ca, cb;\n\t"
+                 "elect.sync _|e, 0xffffffff;\n\t"
+                 "setp.ne.b32 p, %10, 0;\n\t"
+                 "setp.eq.b32 t, %9, %9;\n\t"
+                 "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %5, %9, p;\n\t"
+                 "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %2, %6, %9, t;\n\t"
+                 "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %7, %9, t;\n\t"
+                 "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %4, %8, %9, t;\n\t"
+                 "setp.ne.b32 ca, %11, 0;\n\tand.pred ca, ca, e;\n\t"
+                 "@ca tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%11];\n\t"
+                 "setp.ne.b32 cb, %12, 0;\n\tand.pred cb, cb, e;\n\t"
+                 "@cb tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%12];\n\t}"
+                     :: "r"(d), "l"(a0), "l"(a1), "l"(a2), "l"(a3), "l"(b0), "l"(b1), "l"(b2), "l"(b3), "r"(idesc), "r"(acc0), "r"(bar_a), "r"(bar_b) : "memory");
+    }
+}
+
+template <bool F8>
+__device__ __forceinline__ void mma2_ss_warp(uint32_t d, uint64_t a0, uint64_t a1, uint64_t b0, uint64_t b1,
+                                             uint32_t idesc, uint32_t acc0, uint32_t bar_a = 0u,
+                                             uint32_t bar_b = 0u) {
+    if constexpr (F8) {
+        asm volatile("{\n\t.reg .pred p, e, t, ca, cb;\n\t"
+                 "elect.sync _|e, 0xffffffff;\n\t"
+                 "setp.ne.b32 p, %6, 0;\n\t"
+                 "setp.eq.b32 t, %5, %5;\n\t"
+                 "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %3, %5, p;\n\t"
+                 "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %2, %4, %5, t;\n\t"
+                 "setp.ne.b32 ca, %7, 0;\n\tand.pred ca, ca, e;\n\t"
+                 "@ca tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%7];\n\t"
+                 "setp.ne.b32 cb, %8, 0;\n\tand.pred cb, cb, e;\n\t"
+                 "@cb tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%8];\n\t}"
+                     :: "r"(d), "l"(a0), "l"(a1), "l"(b0), "l"(b1), "r"(idesc), "r"(acc0), "r"(bar_a), "r"(bar_b) : "memory");
+    } else {
+        asm volatile("{\n\t.reg .pred p, e, t, ca, cb;\n\t"
+                 "elect.sync _|e, 0xffffffff;\n\t"
+                 "setp.ne.b32 p, %6, 0;\n\t"
+                 "setp.eq.b32 t, %5, %5;\n\t"
+                 "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %3, %5, p;\n\t"
+                 "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %2, %4, %5, t;\n\t"
+                 "setp.ne.b32 ca, %7, 0;\n\tand.pred ca, ca, e;\n\t"
+                 "@ca tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%7];\n\t"
+                 "setp.ne.b32 cb, %8, 0;\n\tand.pred cb, cb, e;\n\t"
+                 "@cb tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%8];\n\t}"
+                     :: "r"(d), "l"(a0), "l"(a1), "l"(b0), "l"(b1), "r"(idesc), "r"(acc0), "r"(bar_a), "r"(bar_b) : "memory");
+    }
+}
+
+// kind::f16, A from tensor memory (P as bf16 pairs)
+__device__ __forceinline__ void mma4_ts_warp(uint32_t d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                             uint64_t b0, uint64_t b1, uint64_t b2, uint64_t b3, uint32_t idesc,
+                                             uint32_t acc0, uint32_t bar_a = 0u, uint32_t bar_b = 0u) {
+    asm volatile("{\n\t.reg .pred p, e, t, ca, cb;\n\t"
+                 "elect.sync _|e, 0xffffffff;\n\t"
+                 "setp.ne.b32 p, %10, 0;\n\t"
+                 "setp.eq.b32 t, %9, %9;\n\t"
+                 "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %5, %9, p;\n\t"
+                 "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%2], %6, %9, t;\n\t"
+                 "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%3], %7, %9, t;\n\t"
+                 "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%4], %8, %9, t;\n\t"
+                 "setp.ne.b32 ca, %11, 0;\n\tand.pred ca, ca, e;\n\t"
+                 "@ca tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%11];\n\t"
+                 "setp.ne.b32 cb, %12, 0;\n\tand.pred cb, cb, e;\n\t"
+                 "@cb tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%12];\n\t}"
+                 :: "r"(d), "r"(a0), "r"(a1), "r"(a2), "r"(a3), "l"(b0), "l"(b1), "l"(b2), "l"(b3), "r"(idesc), "r"(acc0), "r"(bar_a), "r"(bar_b) : "memory");
+}
+
+// Up to two commits under one elected lane (0: none).
+__device__ __forceinline__ void mma_commit2_warp(uint32_t bar_a, uint32_t bar_b) {
+    asm volatile("{\n\t.reg .pred e, ca, cb;\n\t"
+                 "elect.sync _|e, 0xffffffff;\n\t"
+                 "setp.ne.b32 ca, %0, 0;\n\tand.pred ca, ca, e;\n\t"
+                 "@ca tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t"
+                 "setp.ne.b32 cb, %1, 0;\n\tand.pred cb, cb, e;\n\t"
+                 "@cb tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%1];\n\t}"
+                 :: "r"(bar_a), "r"(bar_b) : "memory");
 }
 
 __device__ __forceinline__ void mma_commit_warp(uint32_t bar) {
