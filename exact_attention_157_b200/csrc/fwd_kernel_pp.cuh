@@ -18,22 +18,37 @@
 //   warp 8      TMA producer: Q_A, Q_B of each unit into one of QS Q buffers,
 //               K_0, V_0, K_1, V_1, ... of every unit into one ring of NSLOT
 //               slots (128-byte swizzle, no multicast), in consumption order
-//   warp 9      TMEM owner and MMA issuer (warp-uniform, one elected lane issues), per unit
-//                 S_A(0) S_B(0) | PV_A(0) S_A(1) PV_B(0) S_B(1) | PV_A(1) ...
-//               so that while the softmax of one tile runs, the tensor cores
-//               work on the other tile (two MMAs of cover each way)
-//   warps 10-11 idle (they complete the third warpgroup that setmaxnreg needs)
+//   warp 9      TMEM owner and MMA issuer (warp-uniform; one elected lane issues
+//               each batch of MMAs and commits)
+//   warp 10     aliased form: idle; decoupled form: MMA issuer of tile B
+//   warp 11     idle (completes the third warpgroup that setmaxnreg needs)
 //
 // TMEM: S_A cols [0,128), S_B [128,256), O_A [256,256+D), O_B [256+D,256+2D).
-// P_t (bf16 pairs, 64 cols) overwrites the first half of S_t once the softmax
-// has read S_t; S_t(j+1) is issued after PV_t(j) by the same thread, and
-// tcgen05.mma operations of one thread execute in issue order.  Because S_t(j)
-// is issued after PV_t(j-1), S_t(j) complete implies O_t = sum_{i<j} P_i V_i,
-// so the softmax may rescale O_t right away, without another barrier.
+//
+// Aliased form (bf16, d = 128: tensor memory is full).  P_t (bf16 pairs, 64
+// cols) overwrites the first half of S_t once the softmax has read S_t, so
+// S_t(j+1) is issued after PV_t(j) by the same thread (tcgen05.mma operations
+// of one thread execute in issue order):
+//     S_A(0) S_B(0) | PV_A(0) S_A(1) PV_B(0) S_B(1) | PV_A(1) ...
+// While the softmax of one tile runs, the tensor cores work on the other.
+// Because S_t(j) is issued after PV_t(j-1), S_t(j) complete implies
+// O_t = sum_{i<j} P_i V_i, so the softmax may rescale O_t right away.
+//
+// Decoupled form (FP8, and bf16 with d = 64).  P_t has a buffer of its own:
+// FP8 in shared memory (128 rows x 128 one-byte keys, read by an SS-form MMA),
+// bf16 d = 64 in the spare TMEM columns [384 + 64 t, 448 + 64 t).  The softmax
+// arrives on SFREE_t as soon as S_t(j) is in registers, and the MMA warp of the
+// tile issues S_t(j+1) at once, so it runs during softmax_t(j); PV_t(j) follows
+// as P_t(j) is stored.  Before it stores P_t(j) or rescales O_t, the softmax
+// waits for PVDONE_t (PV_t(j-1) complete).  Each K/V slot is released by both
+// MMA warps (the EMPTY barriers count two); a tile past its last key block
+// releases a load only once it has landed, so that the arrival cannot count
+// towards the slot's previous use.
+//
 // Across units, PV_t(0) of the next unit waits until the epilogue has read O_t
 // out of TMEM (OEMPTY), and the epilogue stages O_t through the unit's own
 // (dead) Q_t buffer, which the producer refills only after the TMA store has
-// read it (QEMPTY).
+// read it (QEMPTY).  (FP8 writes its bf16 rows directly.)
 //
 // Online softmax in base 2 with the scale folded into the FMA and lazy
 // rescaling ("FlashAttention technical analysis", jsqmd.com/news/722897,

@@ -97,8 +97,12 @@ WORKLOADS = {
         Workload("prefill_gqa_bwd", 1, 32, 2, 16384, 16384, 128, is_causal=True, seed=1010, backward=True),
         Workload("long_fp8", 8, 32, 32, 4096, 4096, 128, seed=1014, fp8=True),
         Workload("long_causal_fp8", 8, 32, 32, 4096, 4096, 128, is_causal=True, seed=1015, fp8=True),
-        # a quarter of long_fp8 (inputs and output still larger than L2), for full ncu captures
+        # quarters of long_fp8, long, long_bwd and decode_gqa (inputs still larger than
+        # L2, under 1 GB on the device), for full ncu captures
         Workload("long_fp8_small", 2, 32, 32, 4096, 4096, 128, seed=1016, fp8=True),
+        Workload("long_small", 2, 32, 32, 4096, 4096, 128, seed=1017),
+        Workload("long_bwd_small", 2, 32, 32, 4096, 4096, 128, seed=1018, backward=True),
+        Workload("decode_gqa_small", 2, 32, 8, 1, 16384, 128, seed=1019, split_kv=True),
         Workload("vit3136_softcap", 8, 12, 12, 3136, 3136, 64, seed=1006, softcap=30.0),
         Workload("vit3136_neighborhood", 8, 12, 12, 3136, 3136, 64, seed=1007, mask2d=("neighborhood", 56, 5)),
     ]
