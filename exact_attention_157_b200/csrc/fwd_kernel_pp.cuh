@@ -419,9 +419,8 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     for (int g = 0; g < kSSteps / 4; ++g) {
                         const uint64_t o = static_cast<uint64_t>(g * (L::kChunkBytes >> 4));  // descriptor units
                         const bool last = g == kSSteps / 4 - 1;
-                        mma4_ss_warp<FP8>(tmem + t * 128, qd + o, qd + o + 2, qd + o + 4, qd + o + 6, kd + o, kd + o + 2,
-                                          kd + o + 4, kd + o + 6, kIdescS, g > 0 ? 1u : 0u,
-                                          last ? bar(L::SFULL + t) : 0u, last ? bar_b : 0u);
+                        mma_ss_batch_warp<FP8, 4, 2, 2>(tmem + t * 128, qd + o, kd + o, kIdescS, g > 0 ? 1u : 0u,
+                                                        last ? bar(L::SFULL + t) : 0u, last ? bar_b : 0u);
                     }
                 };
                 // O_t += P_t(j)[:, keys of this half] V_j[those keys, :], then up to two commits
@@ -436,12 +435,12 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         // P_t in shared memory, 128-byte K-major rows (SW128), 32 keys per step
                         static_assert(kPvSteps == 2, "PV steps");
                         const uint64_t pd = smem_desc_sw128(sbase + L::kPS + t * L::kPBytes + kk0 * 32, 16, 1024);
-                        mma2_ss_warp<true>(o_tmem, pd, pd + 2, vd, vd + kVStep, kIdescO, acc0, bar_a, bar_b);
+                        mma_ss_batch_warp<true, 2, 2, static_cast<int>(kVStep)>(o_tmem, pd, vd, kIdescO, acc0, bar_a,
+                                                                                bar_b);
                     } else {
                         static_assert(kPvSteps == 4, "PV steps");
                         const uint32_t pt = (kDec ? tmem + L::kColP + t * 64 : tmem + t * 128) + kk0 * 8;
-                        mma4_ts_warp(o_tmem, pt, pt + 8, pt + 16, pt + 24, vd, vd + kVStep, vd + 2 * kVStep,
-                                     vd + 3 * kVStep, kIdescO, acc0, bar_a, bar_b);
+                        mma_ts4_batch_warp<8, static_cast<int>(kVStep)>(o_tmem, pt, vd, kIdescO, acc0, bar_a, bar_b);
                     }
                 };
                 ok = mbar_wait_warp(bar(L::QFULL + qb), q_loads[qb] & 1, limit, abort_flag, p.epoch, kRoleMma, 20) &&

@@ -275,94 +275,109 @@ __device__ __forceinline__ void mma_ts_f8_warp(uint32_t d_tmem, uint32_t a_tmem,
                  :: "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
 }
 
-// Batches of MMAs into one accumulator under one elected lane, followed by up
+// Batches of N MMAs into one accumulator under one elected lane, followed by up
 // to two commits (a barrier address of 0 means none): one elect and one
-// predicate set-up for the whole batch.  The first MMA accumulates iff acc0 != 0,
-// the others always.  A operands: shared-memory descriptors (SS) or tensor-memory
-// addresses (TS); kind::f16 (bf16) or kind::f8f6f4 (E4M3).
-template <bool F8>
-__device__ __forceinline__ void mma4_ss_warp(uint32_t d, uint64_t a0, uint64_t a1, uint64_t a2, uint64_t a3,
-                                             uint64_t b0, uint64_t b1, uint64_t b2, uint64_t b3, uint32_t idesc,
-                                             uint32_t acc0, uint32_t bar_a = 0u, uint32_t bar_b = 0u) {
-    if constexpr (F8) {
+// predicate set-up for the whole batch.  MMA i reads A at a0 + i * kAStep and B
+// at b0 + i * kBStep (descriptor units of 16 bytes, or TMEM columns for a TS-form
+// A); the first accumulates iff acc0 != 0, the others always.  kind::f16 (bf16)
+// or kind::f8f6f4 (E4M3).
+template <bool F8, int N, int kAStep, int kBStep>
+__device__ __forceinline__ void mma_ss_batch_warp(uint32_t d, uint64_t a0, uint64_t b0, uint32_t idesc,
+                                                  uint32_t acc0, uint32_t bar_a = 0u, uint32_t bar_b = 0u) {
+    static_assert(N == 2 || N == 4, "batch size");
+    if constexpr (F8 && N == 4) {
         asm volatile("{\n\t.reg .pred p, e, t, ca, cb;\n\t"
-                 "elect.sync _|e, 0xffffffff;\n\t"
-                 "setp.ne.b32 p, %10, 0;\n\t"
-                 "setp.eq.b32 t, %9, %9;\n\t"
-                 "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %5, %9, p;\n\t"
-                 "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %2, %6, %9, t;\n\t"
-                 "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %3, %7, %9, t;\n\t"
-                 "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %4, %8, %9, t;\n\t"
-                 "setp.ne.b32 ca, %11, 0;\n\tand.pred ca, ca, e;\n\t"
-                 "@ca tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%11];\n\t"
-                 "setp.ne.b32 cb, %12, 0;\n\tand.pred cb, cb, e;\n\t"
-                 "@cb tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%12];\n\t}"
-                     :: "r"(d), "l"(a0), "l"(a1), "l"(a2), "l"(a3), "l"(b0), "l"(b1), "l"(b2), "l"(b3), "r"(idesc), "r"(acc0), "r"(bar_a), "r"(bar_b) : "memory");
+                     ".reg .b64 a;\n\t.reg .b64 b;\n\t"
+                     "elect.sync _|e, 0xffffffff;\n\t"
+                     "setp.ne.b32 p, %4, 0;\n\t"
+                     "setp.eq.b32 t, %3, %3;\n\t"
+                     "mov.b64 a, %1;\n\tmov.b64 b, %2;\n\t"
+                     "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a, b, %3, p;\n\t"
+                     "add.s64 a, a, %7;\n\tadd.s64 b, b, %8;\n\t"
+                     "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a, b, %3, t;\n\t"
+                     "add.s64 a, a, %7;\n\tadd.s64 b, b, %8;\n\t"
+                     "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a, b, %3, t;\n\t"
+                     "add.s64 a, a, %7;\n\tadd.s64 b, b, %8;\n\t"
+                     "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a, b, %3, t;\n\t"
+                     "setp.ne.b32 ca, %5, 0;\n\tand.pred ca, ca, e;\n\t"
+                     "@ca tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%5];\n\t"
+                     "setp.ne.b32 cb, %6, 0;\n\tand.pred cb, cb, e;\n\t"
+                     "@cb tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%6];\n\t}"
+                     :: "r"(d), "l"(a0), "l"(b0), "r"(idesc), "r"(acc0), "r"(bar_a), "r"(bar_b), "n"(kAStep), "n"(kBStep) : "memory");
+    } else if constexpr (F8) {
+        asm volatile("{\n\t.reg .pred p, e, t, ca, cb;\n\t"
+                     ".reg .b64 a;\n\t.reg .b64 b;\n\t"
+                     "elect.sync _|e, 0xffffffff;\n\t"
+                     "setp.ne.b32 p, %4, 0;\n\t"
+                     "setp.eq.b32 t, %3, %3;\n\t"
+                     "mov.b64 a, %1;\n\tmov.b64 b, %2;\n\t"
+                     "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a, b, %3, p;\n\t"
+                     "add.s64 a, a, %7;\n\tadd.s64 b, b, %8;\n\t"
+                     "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a, b, %3, t;\n\t"
+                     "setp.ne.b32 ca, %5, 0;\n\tand.pred ca, ca, e;\n\t"
+                     "@ca tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%5];\n\t"
+                     "setp.ne.b32 cb, %6, 0;\n\tand.pred cb, cb, e;\n\t"
+                     "@cb tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%6];\n\t}"
+                     :: "r"(d), "l"(a0), "l"(b0), "r"(idesc), "r"(acc0), "r"(bar_a), "r"(bar_b), "n"(kAStep), "n"(kBStep) : "memory");
+    } else if constexpr (N == 4) {
+        asm volatile("{\n\t.reg .pred p, e, t, ca, cb;\n\t"
+                     ".reg .b64 a;\n\t.reg .b64 b;\n\t"
+                     "elect.sync _|e, 0xffffffff;\n\t"
+                     "setp.ne.b32 p, %4, 0;\n\t"
+                     "setp.eq.b32 t, %3, %3;\n\t"
+                     "mov.b64 a, %1;\n\tmov.b64 b, %2;\n\t"
+                     "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, p;\n\t"
+                     "add.s64 a, a, %7;\n\tadd.s64 b, b, %8;\n\t"
+                     "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, t;\n\t"
+                     "add.s64 a, a, %7;\n\tadd.s64 b, b, %8;\n\t"
+                     "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, t;\n\t"
+                     "add.s64 a, a, %7;\n\tadd.s64 b, b, %8;\n\t"
+                     "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, t;\n\t"
+                     "setp.ne.b32 ca, %5, 0;\n\tand.pred ca, ca, e;\n\t"
+                     "@ca tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%5];\n\t"
+                     "setp.ne.b32 cb, %6, 0;\n\tand.pred cb, cb, e;\n\t"
+                     "@cb tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%6];\n\t}"
+                     :: "r"(d), "l"(a0), "l"(b0), "r"(idesc), "r"(acc0), "r"(bar_a), "r"(bar_b), "n"(kAStep), "n"(kBStep) : "memory");
     } else {
         asm volatile("{\n\t.reg .pred p, e, t, ca, cb;\n\t"
-                 "elect.sync _|e, 0xffffffff;\n\t"
-                 "setp.ne.b32 p, %10, 0;\n\t"
-                 "setp.eq.b32 t, %9, %9;\n\t"
-                 "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %5, %9, p;\n\t"
-                 "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %2, %6, %9, t;\n\t"
-                 "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %7, %9, t;\n\t"
-                 "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %4, %8, %9, t;\n\t"
-                 "setp.ne.b32 ca, %11, 0;\n\tand.pred ca, ca, e;\n\t"
-                 "@ca tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%11];\n\t"
-                 "setp.ne.b32 cb, %12, 0;\n\tand.pred cb, cb, e;\n\t"
-                 "@cb tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%12];\n\t}"
-                     :: "r"(d), "l"(a0), "l"(a1), "l"(a2), "l"(a3), "l"(b0), "l"(b1), "l"(b2), "l"(b3), "r"(idesc), "r"(acc0), "r"(bar_a), "r"(bar_b) : "memory");
+                     ".reg .b64 a;\n\t.reg .b64 b;\n\t"
+                     "elect.sync _|e, 0xffffffff;\n\t"
+                     "setp.ne.b32 p, %4, 0;\n\t"
+                     "setp.eq.b32 t, %3, %3;\n\t"
+                     "mov.b64 a, %1;\n\tmov.b64 b, %2;\n\t"
+                     "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, p;\n\t"
+                     "add.s64 a, a, %7;\n\tadd.s64 b, b, %8;\n\t"
+                     "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, t;\n\t"
+                     "setp.ne.b32 ca, %5, 0;\n\tand.pred ca, ca, e;\n\t"
+                     "@ca tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%5];\n\t"
+                     "setp.ne.b32 cb, %6, 0;\n\tand.pred cb, cb, e;\n\t"
+                     "@cb tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%6];\n\t}"
+                     :: "r"(d), "l"(a0), "l"(b0), "r"(idesc), "r"(acc0), "r"(bar_a), "r"(bar_b), "n"(kAStep), "n"(kBStep) : "memory");
     }
 }
 
-template <bool F8>
-__device__ __forceinline__ void mma2_ss_warp(uint32_t d, uint64_t a0, uint64_t a1, uint64_t b0, uint64_t b1,
-                                             uint32_t idesc, uint32_t acc0, uint32_t bar_a = 0u,
-                                             uint32_t bar_b = 0u) {
-    if constexpr (F8) {
-        asm volatile("{\n\t.reg .pred p, e, t, ca, cb;\n\t"
-                 "elect.sync _|e, 0xffffffff;\n\t"
-                 "setp.ne.b32 p, %6, 0;\n\t"
-                 "setp.eq.b32 t, %5, %5;\n\t"
-                 "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %3, %5, p;\n\t"
-                 "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %2, %4, %5, t;\n\t"
-                 "setp.ne.b32 ca, %7, 0;\n\tand.pred ca, ca, e;\n\t"
-                 "@ca tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%7];\n\t"
-                 "setp.ne.b32 cb, %8, 0;\n\tand.pred cb, cb, e;\n\t"
-                 "@cb tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%8];\n\t}"
-                     :: "r"(d), "l"(a0), "l"(a1), "l"(b0), "l"(b1), "r"(idesc), "r"(acc0), "r"(bar_a), "r"(bar_b) : "memory");
-    } else {
-        asm volatile("{\n\t.reg .pred p, e, t, ca, cb;\n\t"
-                 "elect.sync _|e, 0xffffffff;\n\t"
-                 "setp.ne.b32 p, %6, 0;\n\t"
-                 "setp.eq.b32 t, %5, %5;\n\t"
-                 "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %3, %5, p;\n\t"
-                 "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %2, %4, %5, t;\n\t"
-                 "setp.ne.b32 ca, %7, 0;\n\tand.pred ca, ca, e;\n\t"
-                 "@ca tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%7];\n\t"
-                 "setp.ne.b32 cb, %8, 0;\n\tand.pred cb, cb, e;\n\t"
-                 "@cb tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%8];\n\t}"
-                     :: "r"(d), "l"(a0), "l"(a1), "l"(b0), "l"(b1), "r"(idesc), "r"(acc0), "r"(bar_a), "r"(bar_b) : "memory");
-    }
-}
-
-// kind::f16, A from tensor memory (P as bf16 pairs)
-__device__ __forceinline__ void mma4_ts_warp(uint32_t d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                             uint64_t b0, uint64_t b1, uint64_t b2, uint64_t b3, uint32_t idesc,
-                                             uint32_t acc0, uint32_t bar_a = 0u, uint32_t bar_b = 0u) {
+// kind::f16 with A (P as bf16 pairs) in tensor memory, four MMAs
+template <int kAStep, int kBStep>
+__device__ __forceinline__ void mma_ts4_batch_warp(uint32_t d, uint32_t a0, uint64_t b0, uint32_t idesc,
+                                                   uint32_t acc0, uint32_t bar_a = 0u, uint32_t bar_b = 0u) {
     asm volatile("{\n\t.reg .pred p, e, t, ca, cb;\n\t"
-                 "elect.sync _|e, 0xffffffff;\n\t"
-                 "setp.ne.b32 p, %10, 0;\n\t"
-                 "setp.eq.b32 t, %9, %9;\n\t"
-                 "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %5, %9, p;\n\t"
-                 "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%2], %6, %9, t;\n\t"
-                 "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%3], %7, %9, t;\n\t"
-                 "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%4], %8, %9, t;\n\t"
-                 "setp.ne.b32 ca, %11, 0;\n\tand.pred ca, ca, e;\n\t"
-                 "@ca tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%11];\n\t"
-                 "setp.ne.b32 cb, %12, 0;\n\tand.pred cb, cb, e;\n\t"
-                 "@cb tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%12];\n\t}"
-                 :: "r"(d), "r"(a0), "r"(a1), "r"(a2), "r"(a3), "l"(b0), "l"(b1), "l"(b2), "l"(b3), "r"(idesc), "r"(acc0), "r"(bar_a), "r"(bar_b) : "memory");
+                     ".reg .b32 a;\n\t.reg .b64 b;\n\t"
+                     "elect.sync _|e, 0xffffffff;\n\t"
+                     "setp.ne.b32 p, %4, 0;\n\t"
+                     "setp.eq.b32 t, %3, %3;\n\t"
+                     "mov.b32 a, %1;\n\tmov.b64 b, %2;\n\t"
+                     "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, p;\n\t"
+                     "add.u32 a, a, %7;\n\tadd.s64 b, b, %8;\n\t"
+                     "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, t;\n\t"
+                     "add.u32 a, a, %7;\n\tadd.s64 b, b, %8;\n\t"
+                     "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, t;\n\t"
+                     "add.u32 a, a, %7;\n\tadd.s64 b, b, %8;\n\t"
+                     "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, t;\n\t"
+                     "setp.ne.b32 ca, %5, 0;\n\tand.pred ca, ca, e;\n\t"
+                     "@ca tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%5];\n\t"
+                     "setp.ne.b32 cb, %6, 0;\n\tand.pred cb, cb, e;\n\t"
+                     "@cb tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%6];\n\t}"
+                 :: "r"(d), "r"(a0), "l"(b0), "r"(idesc), "r"(acc0), "r"(bar_a), "r"(bar_b), "n"(kAStep), "n"(kBStep) : "memory");
 }
 
 // Up to two commits under one elected lane (0: none).
