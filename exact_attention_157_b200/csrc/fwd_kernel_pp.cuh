@@ -69,8 +69,9 @@ constexpr int kRegsSoftmax = 200;
 constexpr int kRegsControl = 104;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl <= kPPThreads * 168, "register split");
 
-// EB: bytes per Q/K/V element (2: bf16, 1: FP8); PSMEM: P of both tiles in shared memory
-template <int D, int NSLOT, int QS, int EB = 2, bool PSMEM = false>
+// EB: bytes per Q/K/V element (2: bf16, 1: FP8); PSMEM: P of both tiles in shared memory;
+// OSTAGE: a staging buffer for the bf16 O tiles of its own (else O is staged in the dead Q buffer)
+template <int D, int NSLOT, int QS, int EB = 2, bool PSMEM = false, bool OSTAGE = false>
 struct SmemPP {
     static constexpr int kChunks = D * EB / 128;              // 128-byte column chunks of a row
     static constexpr int kChunkBytes = 128 * 128;
@@ -80,7 +81,8 @@ struct SmemPP {
     static constexpr int kRing = QS * kQBuf;
     static constexpr int kPS = kRing + NSLOT * kTileBytes;   // P_A, P_B: 128 rows x 128 one-byte keys
     static constexpr int kPBytes = 128 * 128;
-    static constexpr int kBars = kPS + (PSMEM ? 2 * kPBytes : 0);
+    static constexpr int kOS = kPS + (PSMEM ? 2 * kPBytes : 0);  // O_A, O_B staging (OSTAGE)
+    static constexpr int kBars = kOS + (OSTAGE ? 2 * kTileBytes : 0);
     // barrier indices
     static constexpr int QFULL = 0;                   // QS: Q buffer loaded
     static constexpr int QEMPTY = QS;                 // QS: Q buffer free (2 arrivals: both tiles' stores)
@@ -106,7 +108,7 @@ struct SmemPP {
 
 // The layout of one kernel instantiation; the host sizes the launch with the same alias.
 template <int D, int NSLOT, int QS, bool FP8>
-using SmemPPFor = SmemPP<D, NSLOT, QS, FP8 ? 1 : 2, FP8>;
+using SmemPPFor = SmemPP<D, NSLOT, QS, FP8 ? 1 : 2, FP8, !FP8 && D == 64>;
 
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
     float d;
@@ -870,8 +872,13 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 ++n_final;
                 tc_fence_after();
             }
+            // Q_t has been read by every S_t of the unit (OFINAL_t).  Unless O is staged
+            // in it (bf16, d = 128), the producer may refill the Q buffer now.
+            constexpr bool kOStage = !SPLIT && !FP8 && D == 64;  // bf16 O staged in a buffer of its own
+            if constexpr (SPLIT || FP8 || kOStage) {
+                if ((threadIdx.x & 127) == 0) release_q(qb);
+            }
             const bool do_epilogue = __all_sync(0xffffffffu, ok && !*abort_flag) && q0_t < p.Nq;
-            uint8_t* stage = smem + L::kQ + qb * L::kQBuf + t * L::kTileBytes;  // Q_t is dead after OFINAL_t
             const float inv_l = l_sum > 0.0f ? 1.0f / l_sum : 0.0f;
             if constexpr (SPLIT) {
                 // Split-KV: this key range's O (normalised by its own row sum) and LSE go
@@ -901,11 +908,9 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 }
                 if (do_epilogue && q_idx < p.Nq)
                     p.ws_lse[rs] = l_sum > 0.0f ? (m_used + __log2f(l_sum)) * kLn2 : -INFINITY;
-                named_barrier_sync(1 + t, 128);
-                if ((threadIdx.x & 127) == 0) release_q(qb);
             } else if constexpr (FP8) {
-                // FP8: O = 2^-6 sv_max * acc / l, bf16, row by row (the FP8 Q buffer is too
-                // small to stage a bf16 tile)
+                // O = 2^-6 sv_max acc / l, bf16, each thread writing its own row straight
+                // from registers (the FP8 Q buffer is too small to stage bf16 tiles)
                 const float scl = inv_l * sv_max * exp2f(-kPShiftF8);
                 uint16_t* orow = static_cast<uint16_t*>(p.out) + (static_cast<long long>(x.bh) * p.Nq + q_idx) * D;
                 #pragma unroll
@@ -919,6 +924,7 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         for (int v = 0; v < 32; ++v) o[v] = 0u;
                     }
                     if (c == D / 32 - 1) {
+                        // O_t has been read out of TMEM: the next unit's PV_t(0) may overwrite it.
                         tc_fence_before();
                         mbar_arrive(bar(L::OEMPTY + t));
                     }
@@ -936,9 +942,17 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 if (do_epilogue && q_idx < p.Nq && p.lse != nullptr)
                     p.lse[static_cast<long long>(x.bh) * p.Nq + q_idx] =
                         l_sum > 0.0f ? (m_used + __log2f(l_sum)) * kLn2 : -INFINITY;
-                named_barrier_sync(1 + t, 128);
-                if ((threadIdx.x & 127) == 0) release_q(qb);
             } else {
+            // bf16 O through shared memory (128-byte swizzled rows) and one TMA store per
+            // tile.  d = 64: a staging buffer of its own, whose previous store is waited
+            // for here, a unit later; d = 128: the dead Q_t buffer, released once the
+            // store has read it.
+            uint8_t* stage = kOStage ? smem + L::kOS + t * L::kTileBytes
+                                     : smem + L::kQ + qb * L::kQBuf + t * L::kTileBytes;
+            if constexpr (kOStage) {
+                if ((threadIdx.x & 127) == 0) bulk_wait_group_read0();
+                named_barrier_sync(1 + t, 128);
+            }
             #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t o[32];
@@ -983,15 +997,17 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                     for (int c = 0; c < L::kChunks; ++c)
                         tma_store_3d(&tm_o, smem_u32(stage) + c * L::kChunkBytes, c * 64, q0_t, x.bh);
                     bulk_commit_group();
-                    bulk_wait_group_read0();
+                    if constexpr (!kOStage) bulk_wait_group_read0();
                 }
-                release_q(qb);  // the producer may refill this Q buffer
+                if constexpr (!kOStage) release_q(qb);  // the producer may refill this Q buffer
             }
             }  // !SPLIT
         }
     }
 
     // ================================ teardown ================================
+    // (a TMA store still reading the O staging buffer must finish before the CTA exits)
+    if (warp < 8 && (threadIdx.x & 127) == 0) bulk_wait_group_read0();
     tc_fence_before();
     __syncthreads();
     if (warp == 9) {
