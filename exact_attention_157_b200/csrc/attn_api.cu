@@ -158,8 +158,10 @@ attn_status_t encode_map(CUtensorMap* map, const void* base, int d, int rows, lo
 
 template <int D, int NSLOT, int QS, bool M>
 cudaError_t launch_pp(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
-                      const FwdParams& p, unsigned grid, cudaStream_t stream) {
+                      const FwdParams& p_in, unsigned grid, cudaStream_t stream) {
     constexpr int kSmem = SmemPPFor<D, NSLOT, QS, false>::kAlloc;
+    FwdParams p = p_in;
+    set_fast_divs(p);
     if (p.n_splits > 1)
         attn_fwd_pp_kernel<D, NSLOT, QS, M, true, false, false><<<grid, kPPThreads, kSmem, stream>>>(tq, tk, tv, to, p);
     else if (!M && (p.softcap_on || p.m2_kind != 0))
@@ -610,6 +612,7 @@ extern "C" attn_status_t attn_fwd_fp8(const void* q8, const void* k8, const void
     p.unit_run = (is_causal && n_units >= 2LL * sms) ? 2 : 1;
     const long long want = (n_units + p.unit_run - 1) / p.unit_run;
     const unsigned g = static_cast<unsigned>(want < sms ? want : sms);
+    set_fast_divs(p);
     attn_fwd_pp_kernel<128, kSlotsF8, kQStagesF8, false, false, false, true>
         <<<g, kPPThreads, SmemF8::kAlloc, static_cast<cudaStream_t>(stream)>>>(tq, tk, tv, tq, p);
     const cudaError_t e = cudaGetLastError();

@@ -22,6 +22,27 @@ constexpr float kLn2 = 0.6931471805599453f;
 // Roles for error reporting.
 enum : unsigned int { kRoleSoftmax = 1, kRoleProducer = 2, kRoleMma = 3, kRoleSelftest = 9 };
 
+// Division by an invariant d >= 1 without a divide instruction ("Division by
+// Invariant Integers using Multiplication", Granlund and Montgomery, PLDI 1994,
+// Theorem 4.2 with N = 31): with l = ceil(log2 d) and m = floor(2^(31+l) / d) + 1,
+// floor(n / d) = floor(m n / 2^(31+l)) for every 0 <= n < 2^31, and m < 2^32.
+// (32-bit integer division by a run-time value goes through a reciprocal on the
+// special-function unit, which the softmax keeps saturated: at each unit boundary
+// a handful of them cost ~1000 cycles, measured with an instrumented copy.)
+struct FastDiv {
+    uint32_t m, l;
+};
+
+inline FastDiv make_fast_div(uint32_t d) {
+    uint32_t l = 0;
+    while ((1ull << l) < d) ++l;
+    return FastDiv{static_cast<uint32_t>((1ull << (31 + l)) / d + 1ull), l};
+}
+
+__device__ __forceinline__ int fdiv(int n, FastDiv f) {
+    return static_cast<int>((static_cast<uint64_t>(f.m) * static_cast<uint32_t>(n)) >> (31 + f.l));
+}
+
 struct FwdParams {
     int B, Hq, Hkv, Nq, Nk;
     int group;          // Hq / Hkv
@@ -56,7 +77,19 @@ struct FwdParams {
     int nqb, nkb;
     unsigned long long timeout_ns;
     unsigned int epoch;  // launch id for the launch-wide abort (never 0)
+    // divisors of the unit decode and of the 2-D masks (set by set_fast_divs)
+    FastDiv fd_qtiles, fd_per_head, fd_hq, fd_group, fd_w, fd_size;
 };
+
+// Fills the FastDiv fields from the fields they divide by (host, before a launch).
+inline void set_fast_divs(FwdParams& p) {
+    p.fd_qtiles = make_fast_div(static_cast<uint32_t>(p.n_qtiles));
+    p.fd_per_head = make_fast_div(static_cast<uint32_t>(p.n_qtiles * p.n_splits));
+    p.fd_hq = make_fast_div(static_cast<uint32_t>(p.Hq));
+    p.fd_group = make_fast_div(static_cast<uint32_t>(p.group));
+    p.fd_w = make_fast_div(static_cast<uint32_t>(p.m2_w > 0 ? p.m2_w : 1));
+    p.fd_size = make_fast_div(static_cast<uint32_t>(p.m2_size > 0 ? p.m2_size : 1));
+}
 
 // Rectangle of the token grid that query row i may see under a 2-D mask: key
 // rows [r_lo, r_hi] and, within each, columns [c_lo, c_hi] (clipped to the grid).
@@ -66,7 +99,7 @@ struct Rect2D {
 
 __device__ __forceinline__ Rect2D rect_2d(const FwdParams& p, int i) {
     const long long W = p.m2_w;
-    const long long qr = i / W, qc = i - qr * W;
+    const long long qr = fdiv(i, p.fd_w), qc = i - qr * W;
     long long r_lo, r_hi, c_lo, c_hi;
     if (p.m2_kind == 1) {  // |dr| < R and |dc| < R
         r_lo = qr - p.m2_size + 1;
@@ -75,12 +108,12 @@ __device__ __forceinline__ Rect2D rect_2d(const FwdParams& p, int i) {
         c_hi = qc + p.m2_size - 1;
     } else {  // same displaced window
         const long long w = p.m2_size, sh = p.m2_shift;
-        r_lo = ((qr + sh) / w) * w - sh;
+        r_lo = static_cast<long long>(fdiv(static_cast<int>(qr + sh), p.fd_size)) * w - sh;
         r_hi = r_lo + w - 1;
-        c_lo = ((qc + sh) / w) * w - sh;
+        c_lo = static_cast<long long>(fdiv(static_cast<int>(qc + sh), p.fd_size)) * w - sh;
         c_hi = c_lo + w - 1;
     }
-    const long long last_row = (static_cast<long long>(p.Nk) - 1) / W;  // key rows that exist
+    const long long last_row = fdiv(p.Nk - 1, p.fd_w);  // key rows that exist
     Rect2D r;
     r.r_lo = static_cast<int>(r_lo < 0 ? 0 : r_lo);
     r.r_hi = static_cast<int>(r_hi > last_row ? last_row : r_hi);

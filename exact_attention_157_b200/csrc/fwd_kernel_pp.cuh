@@ -184,33 +184,38 @@ __device__ __forceinline__ int unit_seq(int c, int k, int G, int P) {
 // The key length of the batch entry of the unit at sequence position s (a
 // global load, issued one unit ahead by every role so that its latency is off
 // the critical path).
+// FAST: the unit decode divides by multiplication (FastDiv).  Measured on B200: it
+// pays where units are short and many per CTA (d = 64: vit -4 %, unet_cross -8 %
+// time), and costs 2-3 % at d = 128, whose units run 32 key blocks each.
+template <bool FAST>
 __device__ __forceinline__ int unit_key_len(const FwdParams& p, int s, int n_units) {
     if (p.key_lens == nullptr || s >= n_units) return p.Nk;
+    if constexpr (FAST) return __ldg(p.key_lens + fdiv(fdiv(s, p.fd_per_head), p.fd_hq));
     return __ldg(p.key_lens + (s / (p.n_qtiles * p.n_splits)) / p.Hq);
 }
 
 // Units are numbered (head, split, query-unit): the units of one head and key
 // range are adjacent.  Without split-KV (SPLIT = false) there is one range.
-template <bool SPLIT, bool MOD>
+template <bool SPLIT, bool MOD, bool FAST>
 __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int s, int kv_len, bool report) {
     Unit x;
     int pos;
     if constexpr (SPLIT) {
         const int per_head = p.n_qtiles * p.n_splits;
-        x.bh = s / per_head;
+        x.bh = FAST ? fdiv(s, p.fd_per_head) : s / per_head;
         const int r = s - x.bh * per_head;
-        x.split = r / p.n_qtiles;
+        x.split = FAST ? fdiv(r, p.fd_qtiles) : r / p.n_qtiles;
         pos = r - x.split * p.n_qtiles;
     } else {
-        x.bh = s / p.n_qtiles;
+        x.bh = FAST ? fdiv(s, p.fd_qtiles) : s / p.n_qtiles;
         x.split = 0;
         pos = s - x.bh * p.n_qtiles;
     }
     // causal: heavy and light query tiles alternate (n-1, 0, n-2, 1, ...)
     const int qt = !p.is_causal ? pos : (pos & 1) ? (pos >> 1) : p.n_qtiles - 1 - (pos >> 1);
-    x.b = x.bh / p.Hq;
+    x.b = FAST ? fdiv(x.bh, p.fd_hq) : x.bh / p.Hq;
     x.h = x.bh - x.b * p.Hq;
-    x.bhk = x.b * p.Hkv + x.h / p.group;
+    x.bhk = x.b * p.Hkv + (FAST ? fdiv(x.h, p.fd_group) : x.h / p.group);
     x.q0 = qt * 2 * kBM;
     x.tile_b_valid = x.q0 + kBM < p.Nq;
     if (kv_len < 0 || kv_len > p.Nk) {
@@ -334,10 +339,10 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             int i_glob = 0;  // K/V loads issued so far (ring position)
             bool ok = true;
             int it = 0;
-            int kv_next = unit_key_len(p, unit_seq(cta, 0, G, p.unit_run), n_units);
+            int kv_next = unit_key_len<D == 64>(p, unit_seq(cta, 0, G, p.unit_run), n_units);
             for (int u = unit_seq(cta, 0, G, p.unit_run); ok && u < n_units; ++it, u = unit_seq(cta, it, G, p.unit_run)) {
-                const Unit x = decode_unit<SPLIT, MOD>(p, u, kv_next, false);
-                kv_next = unit_key_len(p, unit_seq(cta, it + 1, G, p.unit_run), n_units);
+                const Unit x = decode_unit<SPLIT, MOD, D == 64>(p, u, kv_next, false);
+                kv_next = unit_key_len<D == 64>(p, unit_seq(cta, it + 1, G, p.unit_run), n_units);
                 const int qb = it % QS;
                 const int n_max = x.n_max();
                 if (n_max == 0) continue;  // nothing to load; its epilogue does not use a Q buffer
@@ -398,10 +403,10 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             int gf[2] = {0, 0};  // SFREE_t phases waited for (decoupled S and P)
             bool ok = true;
             int it = 0;
-            int kv_next = unit_key_len(p, unit_seq(cta, 0, G, p.unit_run), n_units);
+            int kv_next = unit_key_len<D == 64>(p, unit_seq(cta, 0, G, p.unit_run), n_units);
             for (int u = unit_seq(cta, 0, G, p.unit_run); ok && u < n_units; ++it, u = unit_seq(cta, it, G, p.unit_run)) {
-                const Unit x = decode_unit<SPLIT, MOD>(p, u, kv_next, false);
-                kv_next = unit_key_len(p, unit_seq(cta, it + 1, G, p.unit_run), n_units);
+                const Unit x = decode_unit<SPLIT, MOD, D == 64>(p, u, kv_next, false);
+                kv_next = unit_key_len<D == 64>(p, unit_seq(cta, it + 1, G, p.unit_run), n_units);
                 const int n_max = x.n_max();
                 if (n_max == 0) continue;
                 const int qb = it % QS;
@@ -565,10 +570,10 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         int n_final = 0;  // units with a PV for this tile so far (OFINAL phase)
         bool ok = true;
         int it = 0;
-        int kv_next = unit_key_len(p, unit_seq(cta, 0, G, p.unit_run), n_units);
+        int kv_next = unit_key_len<D == 64>(p, unit_seq(cta, 0, G, p.unit_run), n_units);
         for (int u = unit_seq(cta, 0, G, p.unit_run); u < n_units; ++it, u = unit_seq(cta, it, G, p.unit_run)) {
-            const Unit x = decode_unit<SPLIT, MOD>(p, u, kv_next, threadIdx.x == 0);
-            kv_next = unit_key_len(p, unit_seq(cta, it + 1, G, p.unit_run), n_units);
+            const Unit x = decode_unit<SPLIT, MOD, D == 64>(p, u, kv_next, threadIdx.x == 0);
+            kv_next = unit_key_len<D == 64>(p, unit_seq(cta, it + 1, G, p.unit_run), n_units);
             const int q0_t = x.q0 + t * kBM;
             const int q_idx = q0_t + row;
             const int n_blocks = ok ? x.n_t[t] : 0;
@@ -658,8 +663,8 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                         // one run of columns per key row the block touches
                         uint32_t mw[kBN / 32] = {0u, 0u, 0u, 0u};
                         const int W = p.m2_w;
-                        int kr = j0 / W;
-                        const int kr_end = (j0 + kBN - 1) / W;
+                        int kr = fdiv(j0, p.fd_w);
+                        const int kr_end = fdiv(j0 + kBN - 1, p.fd_w);
                         if (kr < rq.r_lo) kr = rq.r_lo;
                         for (; kr <= kr_end && kr <= rq.r_hi; ++kr) {
                             int a = kr * W + rq.c_lo - j0, b = kr * W + rq.c_hi - j0;
