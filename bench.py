@@ -568,7 +568,7 @@ def run_reference(args, w):
         "ms_per_step": 1e3 * t / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic", "impl": "reference",
         "config": {"workload": f"{w.name}: B{w.B} Hq{w.Hq} Hkv{w.Hkv} Nq{w.Nq} Nk{w.Nk} d{w.d}"
-                               f"{' causal' if w.is_causal else ''}",
+                               f"{' causal' if w.is_causal else ''}{' fp8 e4m3' if w.fp8 else ''}",
                    "sample_per_step": desc},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
