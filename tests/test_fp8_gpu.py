@@ -168,3 +168,29 @@ def test_full_size_sampled_rows():
 def _deq_rows(codes, scales):
     """Dequantize selected rows whose block scales are given one per row."""
     return oracle.e4m3_decode(codes.numpy()) * np.asarray(scales, dtype=np.float64)[..., None]
+
+
+def test_deterministic():
+    q8, k8, v8, qs, ks, vs = make_fp8_inputs(2, 4, 2, 600, 900, 128, seed=18)
+    o1, l1 = run_fp8(q8, k8, v8, qs, ks, vs, is_causal=True)
+    o2, l2 = run_fp8(q8, k8, v8, qs, ks, vs, is_causal=True)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
+def test_masked_keys_are_bit_exact():
+    """Other codes at masked key positions (past each key length) change no
+    output bit; the block scales are kept, so P's V-scale fold is unchanged."""
+    q8, k8, v8, qs, ks, vs = make_fp8_inputs(3, 2, 2, 300, 384, 128, seed=19)
+    lens = [384, 200, 129]
+    kl = torch.tensor(lens, dtype=torch.int32)
+    o1, l1 = run_fp8(q8, k8, v8, qs, ks, vs, key_lens=kl)
+    g = torch.Generator().manual_seed(20)
+    k2, v2 = k8.clone(), v8.clone()
+    for b, n in enumerate(lens):
+        # random finite E4M3 codes (0x7F and 0xFF, the NaN codes, excluded)
+        for t in (k2, v2):
+            c = torch.randint(0, 0x7F, (2, 384 - n, 128), generator=g, dtype=torch.int64)
+            sign = torch.randint(0, 2, c.shape, generator=g, dtype=torch.int64) << 7
+            t[b, :, n:] = (c | sign).to(torch.uint8)
+    o2, l2 = run_fp8(q8, k2, v2, qs, ks, vs, key_lens=kl)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)

@@ -122,10 +122,12 @@ def test_additive_mask_broadcast_and_causal():
     assert_close(out, lse, ro, rl)
 
 
+@pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("causal", [False, True])
-def test_masked_keys_are_bit_exact(causal):
-    """Finite garbage at masked key positions changes no output bit."""
-    B, H, N, d = 3, 2, 384, 128
+def test_masked_keys_are_bit_exact(causal, d):
+    """Finite garbage at masked key positions changes no output bit (d = 64 runs the
+    decoupled form of the kernel, d = 128 the aliased one)."""
+    B, H, N = 3, 2, 384
     q, k, v = make_qkv(B, H, H, N, N, d, seed=51)
     lens = torch.tensor([384, 200, 129], dtype=torch.int32)
     out1, lse1 = run_gpu(q, k, v, is_causal=causal, key_lens=lens)
@@ -144,8 +146,9 @@ def test_masked_keys_are_bit_exact(causal):
         assert not torch.equal(out3[0, :, -1], out1[0, :, -1])
 
 
-def test_deterministic():
-    q, k, v = make_qkv(2, 4, 4, 1000, 1000, 128, seed=61)
+@pytest.mark.parametrize("d", [64, 128])
+def test_deterministic(d):
+    q, k, v = make_qkv(2, 4, 4, 1000, 1000, d, seed=61)
     a = run_gpu(q, k, v, is_causal=True)
     b = run_gpu(q, k, v, is_causal=True)
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
