@@ -324,17 +324,23 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             my_d = p.delta[r];
         }
         const int key_row = DKDV ? blk * kBN + row : 0;
+        // DKDV: LSE2 and D of each iteration's 128 queries, one value per thread, loaded
+        // before the wait for S^T and dP^T (the loads overlap those products) and shared
+        // through a double buffer (a buffer is rewritten two iterations later, after
+        // every thread has passed the barrier of the iteration between)
+        __shared__ float s_l2[2][kBM], s_dd[2][kBM];
         bool ok = !*abort_flag;
         for (int it = 0; ok && it < n_iter; ++it) {
             const int ib = iter_blk(it);
             // DKDV: LSE2 and D of this iteration's 128 queries (the same addresses in every
             // lane: broadcast loads; rows are padded to 128, so 16-byte aligned)
-            const float* l2row = nullptr;
-            const float* ddrow = nullptr;
+            const int buf = it & 1;
             if constexpr (DKDV) {
+                // rows are padded to a multiple of 128 per head: row < 128 stays in bounds
                 const long long r = static_cast<long long>(b * p.Hq + iter_head(it)) * p.nq_pad + ib * kBM;
-                l2row = p.lse2 + r;
-                ddrow = p.delta + r;
+                s_l2[buf][row] = __ldg(p.lse2 + r + row);
+                s_dd[buf][row] = __ldg(p.delta + r + row);
+                named_barrier_sync(1, kBM);
             }
             const bool got = mbar_wait(bar(L::STFULL_), it & 1, limit, abort_flag, p.epoch, kRoleBwdElem, 2);
             if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
@@ -345,16 +351,6 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tmem_ld32(lane_tmem + L::kColA + c * 32, sv);
                 tmem_ld32(lane_tmem + L::kColB + c * 32, dv);
                 tmem_wait_ld();
-                float l2c[32], ddc[32];
-                if constexpr (DKDV) {
-                    #pragma unroll
-                    for (int v = 0; v < 8; ++v) {
-                        const float4 a = __ldg(reinterpret_cast<const float4*>(l2row + c * 32) + v);
-                        const float4 z = __ldg(reinterpret_cast<const float4*>(ddrow + c * 32) + v);
-                        l2c[4 * v] = a.x; l2c[4 * v + 1] = a.y; l2c[4 * v + 2] = a.z; l2c[4 * v + 3] = a.w;
-                        ddc[4 * v] = z.x; ddc[4 * v + 1] = z.y; ddc[4 * v + 2] = z.z; ddc[4 * v + 3] = z.w;
-                    }
-                }
                 uint32_t pw[16], dw[16];
                 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
@@ -366,8 +362,8 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         bool vis;
                         if constexpr (DKDV) {
                             const int qi = ib * kBM + col;
-                            l2 = l2c[e + u];
-                            dd = ddc[e + u];
+                            l2 = s_l2[buf][col];  // the same address in every lane: a broadcast
+                            dd = s_dd[buf][col];
                             vis = key_row < kv_len && (!p.is_causal || key_row <= qi);
                         } else {
                             const int kj = ib * kBN + col;
