@@ -104,6 +104,7 @@ WORKLOADS = {
         Workload("long_bwd_small", 2, 32, 32, 4096, 4096, 128, seed=1018, backward=True),
         Workload("decode_gqa_small", 2, 32, 8, 1, 16384, 128, seed=1019, split_kv=True),
         Workload("long_causal_small", 2, 32, 32, 4096, 4096, 128, is_causal=True, seed=1020),
+        Workload("long_causal_fp8_small", 2, 32, 32, 4096, 4096, 128, is_causal=True, seed=1022, fp8=True),
         # half of prefill_gqa (one K/V head and its 16 query heads)
         Workload("prefill_gqa_small", 1, 16, 1, 16384, 16384, 128, is_causal=True, seed=1021),
         Workload("vit3136_softcap", 8, 12, 12, 3136, 3136, 64, seed=1006, softcap=30.0),
