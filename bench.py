@@ -3,6 +3,10 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload long] [--impl ours|reference]
 
+--gpus N > 1 without a launcher starts N ranks itself (torch.distributed.run,
+one process per GPU, rendezvous on 127.0.0.1); under torchrun, WORLD_SIZE must
+equal N.
+
 One step = one exact-attention forward pass (every step of the hot path, one
 kernel launch) over the whole workload, inputs resident in HBM.  The default
 workload is B8 H32 N4096 d128 bf16, non-causal (the shape of the pages' B8 H32
@@ -22,7 +26,6 @@ import hashlib
 import json
 import math
 import os
-import re
 import statistics
 import sys
 import threading
@@ -73,18 +76,18 @@ def kernel_source_hash(family: str = "tile") -> str:
 
 
 def recorded_traffic(w):
-    """DRAM bytes per launch from the committed ncu summary of this kernel and
-    workload, if it was taken on the current kernel sources; else None."""
-    path = os.path.join(ROOT, "profiles", f"attn_{'bwd' if w.backward else 'fwd'}_{w.name}.md")
+    """DRAM bytes per launch of this kernel and workload from profiles/traffic.json
+    (written beside the ncu summaries), if they were taken on the current kernel
+    sources; else None."""
+    key = f"attn_{'bwd' if w.backward else 'fwd'}_{w.name}"
     try:
-        text = open(path).read()
-    except OSError:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f).get(key)
+    except (OSError, ValueError):
         return None
-    m_b = re.search(r"^traffic_bytes_per_launch:\s*([0-9.eE+]+)", text, re.M)
-    m_h = re.search(r"^kernel_source_sha:\s*([0-9a-f]+)", text, re.M)
-    if not m_b or not m_h or m_h.group(1) != kernel_source_hash(kernel_family(w)):
+    if not rec or rec.get("kernel_source_sha") != kernel_source_hash(kernel_family(w)):
         return None
-    return float(m_b.group(1))
+    return float(rec["traffic_bytes_per_launch"])
 
 
 class ClockSampler:
@@ -576,8 +579,23 @@ def run_reference(args, w):
     print(json.dumps(result), flush=True)
 
 
+def launch_ranks(n: int, argv) -> int:
+    """Runs this script as n ranks on this node (one process per GPU) under
+    torch.distributed.run, rendezvous on 127.0.0.1, and returns its exit code.
+    Each rank reads RANK / LOCAL_RANK / WORLD_SIZE from the environment."""
+    import socket
+    import subprocess
+    with socket.socket() as sock:
+        sock.bind(("127.0.0.1", 0))
+        port = sock.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr=127.0.0.1", f"--master-port={port}", os.path.abspath(__file__), *argv]
+    return subprocess.run(cmd, cwd=ROOT).returncode
+
+
 def main(argv=None):
     from workloads import WORKLOADS
+    argv = list(sys.argv[1:] if argv is None else argv)
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
@@ -590,6 +608,13 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be at least 1")
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        return launch_ranks(args.gpus, argv)  # one rank per GPU, started here
+    world = dist_env()[0]
+    if world != args.gpus:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}: launch with --nproc-per-node {args.gpus}")
     w = WORKLOADS[args.workload]
     if args.impl == "reference":
         run_reference(args, w)
@@ -598,4 +623,4 @@ def main(argv=None):
 
 
 if __name__ == "__main__":
-    main()
+    sys.exit(main() or 0)

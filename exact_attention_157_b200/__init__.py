@@ -40,7 +40,7 @@ NOALLOC_SCRATCH_BYTES = 16 << 20  # ATTN_NOALLOC_SCRATCH_BYTES
 # Every symbol include/attn.h declares.
 EXPORTED = ("attn_fwd", "attn_fwd_mod", "attn_fwd_fp8", "attn_bwd_plan", "attn_bwd", "attn_splitkv_plan", "attn_fwd_splitkv", "attn_fwd_splitkv_noalloc",
             "attn_check_device_status", "attn_set_wait_timeout_ns", "attn_selftest_timeout",
-            "attn_status_string", "attn_last_cuda_error", "attn_version")
+            "attn_selftest_exp2_poly", "attn_status_string", "attn_last_cuda_error", "attn_version")
 
 MASK2D_KINDS = {None: 0, "neighborhood": 1, "window": 2}
 
@@ -110,6 +110,8 @@ def lib() -> ctypes.CDLL:
             L.attn_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
             L.attn_selftest_timeout.restype = i
             L.attn_selftest_timeout.argtypes = [vp]
+            L.attn_selftest_exp2_poly.restype = i
+            L.attn_selftest_exp2_poly.argtypes = [vp, vp, i, vp]
             L.attn_status_string.restype = ctypes.c_char_p
             L.attn_status_string.argtypes = [i]
             L.attn_last_cuda_error.restype = i
@@ -226,6 +228,19 @@ def attn_set_wait_timeout_ns(ns: int) -> int:
 
 def attn_selftest_timeout(stream=None) -> int:
     return int(lib().attn_selftest_timeout(stream))
+
+
+def exp2_poly(x, stream=None):
+    """2^x by the FP8 path's FMA-pipe polynomial (attn_selftest_exp2_poly) for a
+    contiguous fp32 CUDA tensor; returns a new tensor."""
+    import torch
+    if not (x.is_cuda and x.dtype == torch.float32 and x.is_contiguous()):
+        raise TypeError("x must be a contiguous float32 CUDA tensor")
+    y = torch.empty_like(x)
+    st = int(lib().attn_selftest_exp2_poly(x.data_ptr(), y.data_ptr(), x.numel(), _stream_handle(stream)))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_selftest_exp2_poly")
+    return y
 
 
 # ------------------------------------------------------- torch marshalling

@@ -271,15 +271,13 @@ SplitPlan make_plan(int B, int Hq, int Hkv, int Nq, int Nk, int d, bool causal, 
 }
 
 
-// Shared by attn_fwd (n_splits = 1) and attn_fwd_splitkv.
-attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, float* lse,
-                       int B, int Hq, int Hkv, int Nq, int Nk, int d,
-                       float scale, int is_causal,
-                       const int32_t* key_lens,
-                       const float* additive_mask, const int64_t* mask_strides,
-                       bool split_kv, int n_splits_req, void* workspace, size_t workspace_bytes,
-                       const attn_score_mod_t* mod, void* stream) {
-    // ---- host-side validation (no CUDA call before this passes)
+// Host-side argument checks of the forward entry points (no CUDA call); on
+// success the element strides of the additive mask are in msb, msh, msq.
+attn_status_t validate_fwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                           int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
+                           const int32_t* key_lens, const float* additive_mask, const int64_t* mask_strides,
+                           bool split_kv, int n_splits_req, const void* workspace, const attn_score_mod_t* mod,
+                           long long* msb, long long* msh, long long* msq) {
     if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return ATTN_ERR_INVALID_ARG;
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nk <= 0 || d <= 0) return ATTN_ERR_INVALID_ARG;
     if (Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
@@ -291,20 +289,19 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, f
         (key_lens != nullptr && (reinterpret_cast<uintptr_t>(key_lens) & 3u)) ||
         (additive_mask != nullptr && (reinterpret_cast<uintptr_t>(additive_mask) & 3u)))
         return ATTN_ERR_ALIGNMENT;
-    long long msb = 0, msh = 0, msq = 0;
+    *msb = *msh = *msq = 0;
     if (additive_mask != nullptr) {
         if (mask_strides != nullptr) {
-            msb = mask_strides[0];
-            msh = mask_strides[1];
-            msq = mask_strides[2];
-            if (msb < 0 || msh < 0 || msq < 0) return ATTN_ERR_INVALID_ARG;
+            *msb = mask_strides[0];
+            *msh = mask_strides[1];
+            *msq = mask_strides[2];
+            if (*msb < 0 || *msh < 0 || *msq < 0) return ATTN_ERR_INVALID_ARG;
         } else {
-            msq = Nk;
-            msh = static_cast<long long>(Nq) * Nk;
-            msb = msh * Hq;
+            *msq = Nk;
+            *msh = static_cast<long long>(Nq) * Nk;
+            *msb = *msh * Hq;
         }
     }
-
     if (split_kv && (n_splits_req < 0 || (workspace != nullptr && reinterpret_cast<uintptr_t>(workspace) % kWsAlign)))
         return n_splits_req < 0 ? ATTN_ERR_INVALID_ARG : ATTN_ERR_ALIGNMENT;
     const bool use_mod = mod != nullptr && (mod->softcap != 0.0f || mod->mask2d_kind != ATTN_MASK2D_NONE);
@@ -317,6 +314,23 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, f
             return ATTN_ERR_INVALID_ARG;
     }
     if (use_mod && (additive_mask != nullptr || split_kv)) return ATTN_ERR_UNSUPPORTED;
+    return ATTN_OK;
+}
+
+// Shared by attn_fwd (n_splits = 1) and attn_fwd_splitkv.
+attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, float* lse,
+                       int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                       float scale, int is_causal,
+                       const int32_t* key_lens,
+                       const float* additive_mask, const int64_t* mask_strides,
+                       bool split_kv, int n_splits_req, void* workspace, size_t workspace_bytes,
+                       const attn_score_mod_t* mod, void* stream) {
+    // ---- host-side validation (no CUDA call before this passes)
+    long long msb = 0, msh = 0, msq = 0;
+    attn_status_t vst = validate_fwd(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, key_lens, additive_mask,
+                                     mask_strides, split_kv, n_splits_req, workspace, mod, &msb, &msh, &msq);
+    if (vst != ATTN_OK) return vst;
+    const bool use_mod = mod != nullptr && (mod->softcap != 0.0f || mod->mask2d_kind != ATTN_MASK2D_NONE);
 
     int dev = 0;
     attn_status_t st = device_setup(&dev);
@@ -459,6 +473,17 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, f
     return ATTN_OK;
 }
 
+// y[i] = exp2_poly_x2(x[i]), two elements per thread (the FP8 softmax's
+// FMA-pipe exponential, exposed for its accuracy test).
+__global__ void attn_exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
+    const long long i = 2LL * (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x);
+    if (i >= n) return;
+    const bool two = i + 1 < n;
+    const uint64_t r = exp2_poly_x2(pack_f32x2(x[i], two ? x[i + 1] : x[i]));
+    y[i] = lo_f32(r);
+    if (two) y[i + 1] = hi_f32(r);
+}
+
 }  // namespace
 
 extern "C" {
@@ -537,6 +562,21 @@ attn_status_t attn_selftest_timeout(void* stream) {
     if (st != ATTN_OK) return st;
     attn_selftest_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(g_timeout_ns.load(), next_epoch());
     cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e);
+    return ATTN_OK;
+}
+
+attn_status_t attn_selftest_exp2_poly(const float* x, float* y, int n, void* stream) {
+    if (n < 0 || (n > 0 && (x == nullptr || y == nullptr))) return ATTN_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(x) & 3u) || (reinterpret_cast<uintptr_t>(y) & 3u)) return ATTN_ERR_ALIGNMENT;
+    if (n == 0) return ATTN_OK;
+    int dev = 0;
+    attn_status_t st = device_setup(&dev);
+    if (st != ATTN_OK) return st;
+    const long long pairs = (static_cast<long long>(n) + 1) / 2;
+    const unsigned grid = static_cast<unsigned>((pairs + 255) / 256);
+    attn_exp2_poly_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
+    const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e);
     return ATTN_OK;
 }
@@ -741,10 +781,13 @@ extern "C" attn_status_t attn_fwd_splitkv_noalloc(const void* q, const void* k, 
                                                   float scale, int is_causal, const int32_t* key_lens,
                                                   const float* additive_mask, const int64_t* mask_strides,
                                                   int n_splits, void* stream) {
-    if (B <= 0 || Hq <= 0 || Nq <= 0 || Nk <= 0 || n_splits < 0) return ATTN_ERR_INVALID_ARG;
-    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+    // every argument check runs before the one-time device set-up
+    long long msb = 0, msh = 0, msq = 0;
+    attn_status_t st = validate_fwd(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, key_lens, additive_mask,
+                                    mask_strides, true, n_splits, nullptr, nullptr, &msb, &msh, &msq);
+    if (st != ATTN_OK) return st;
     int dev = 0;
-    attn_status_t st = device_setup(&dev);
+    st = device_setup(&dev);
     if (st != ATTN_OK) return st;
     int used = 1;
     size_t need = 0;

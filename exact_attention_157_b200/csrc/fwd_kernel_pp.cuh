@@ -63,8 +63,9 @@ namespace attn_sm100 {
 
 constexpr int kPPThreads = 384;  // 12 warps = 3 warpgroups
 // Register split (setmaxnreg): launched at 168 per thread (384 x 168 = 64512);
-// the TMA/MMA warpgroup gives back to 88 and the two softmax warpgroups take
-// 208: 2 x 128 x 208 + 128 x 88 = 64512, exactly the launch total.
+// the TMA/MMA warpgroup gives back to kRegsControl and the two softmax
+// warpgroups take kRegsSoftmax: 2 x 128 x 200 + 128 x 104 = 64512, exactly the
+// launch total.
 constexpr int kRegsSoftmax = 200;
 constexpr int kRegsControl = 104;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl <= kPPThreads * 168, "register split");
@@ -148,7 +149,9 @@ __device__ __forceinline__ float hi_f32(uint64_t v) { return __uint_as_float(sta
 // 2^x for two fp32 values with FMA-pipe arithmetic only: x = n + f, n the nearest
 // integer (added to the exponent field) and 2^f for |f| <= 1/2 from a cubic whose
 // coefficients were fitted by the Remez exchange for least maximum relative error
-// (7.5e-5 on the interval).  x is clamped at -125 so that the result stays normal.
+// (7.5e-5 on the interval).  x < -125 (a masked key's -inf among them) gives 0, as
+// ex2.approx does far below the normal range; the arithmetic itself runs on x
+// clamped at -125 so that the result stays normal.
 __device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t xv) {
     constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: x + kRound holds round(x) in its low bits
     const float x0 = fmaxf(lo_f32(xv), -125.0f), x1 = fmaxf(hi_f32(xv), -125.0f);
@@ -160,8 +163,10 @@ __device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t xv) {
                        pack_f32x2(0.2426111251115799f, 0.2426111251115799f));
     q = ffma2(q, f, pack_f32x2(0.6932609677314758f, 0.6932609677314758f));
     q = ffma2(q, f, pack_f32x2(0.9999280571937561f, 0.9999280571937561f));
-    const uint32_t r0 = static_cast<uint32_t>(q) + (static_cast<uint32_t>(t) << 23);
-    const uint32_t r1 = static_cast<uint32_t>(q >> 32) + (static_cast<uint32_t>(t >> 32) << 23);
+    uint32_t r0 = static_cast<uint32_t>(q) + (static_cast<uint32_t>(t) << 23);
+    uint32_t r1 = static_cast<uint32_t>(q >> 32) + (static_cast<uint32_t>(t >> 32) << 23);
+    r0 = lo_f32(xv) < -125.0f ? 0u : r0;
+    r1 = hi_f32(xv) < -125.0f ? 0u : r1;
     return (static_cast<uint64_t>(r1) << 32) | r0;
 }
 

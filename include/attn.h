@@ -224,7 +224,9 @@ attn_status_t attn_fwd_splitkv(const void *q, const void *k, const void *v, void
  * order them on one stream or synchronise between them.
  *
  * Arguments and results as attn_fwd_splitkv without workspace and
- * workspace_bytes.  Errors: as attn_fwd_splitkv, plus ATTN_ERR_SCRATCH.
+ * workspace_bytes.  Errors: as attn_fwd_splitkv, plus ATTN_ERR_SCRATCH.  All
+ * argument checks run before the first-call set-up, so a rejected call does
+ * no set-up.
  */
 #define ATTN_NOALLOC_SCRATCH_BYTES (16u << 20)
 attn_status_t attn_fwd_splitkv_noalloc(const void *q, const void *k, const void *v, void *out, float *lse,
@@ -328,6 +330,18 @@ attn_status_t attn_set_wait_timeout_ns(uint64_t ns);
  * it touches no caller memory.  Asynchronous on `stream`.
  */
 attn_status_t attn_selftest_timeout(void *stream);
+
+/*
+ * attn_selftest_exp2_poly -- y[i] = 2^x[i] by the polynomial exponential that
+ * the FP8 forward pass runs on the FMA pipe for one pair of probabilities in
+ * four (x = n + f with n the nearest integer, 2^f from a cubic fitted for least
+ * maximum relative error on |f| <= 1/2; 0 for x < -125).  Exposed so that its
+ * accuracy can be tested against 2^x; not part of the attention computation.
+ *   x, y: device fp32 [n], 4-byte aligned; n >= 0.  Asynchronous on `stream`.
+ * Errors: ATTN_ERR_INVALID_ARG (n < 0, or a NULL pointer with n > 0),
+ * ATTN_ERR_ALIGNMENT, ATTN_ERR_UNSUPPORTED / ATTN_ERR_CUDA as attn_fwd.
+ */
+attn_status_t attn_selftest_exp2_poly(const float *x, float *y, int n, void *stream);
 
 /* Text for a status code (static storage). */
 const char *attn_status_string(int status);

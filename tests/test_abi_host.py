@@ -261,3 +261,30 @@ def test_fp8_validation_is_host_side(args, status):
               Nq=64, Nk=64, d=128, scale=0.0, is_causal=0)
     kw.update(args)
     assert ea.attn_fwd_fp8(**kw) == status
+
+
+@pytest.mark.parametrize("args,status", [
+    (dict(q=0), ea.ATTN_ERR_INVALID_ARG),
+    (dict(Hkv=0), ea.ATTN_ERR_INVALID_ARG),
+    (dict(Hq=3, Hkv=2), ea.ATTN_ERR_INVALID_ARG),
+    (dict(scale=-1.0), ea.ATTN_ERR_INVALID_ARG),
+    (dict(n_splits=-1), ea.ATTN_ERR_INVALID_ARG),
+    (dict(d=96), ea.ATTN_ERR_UNSUPPORTED),
+    (dict(k=A + 4), ea.ATTN_ERR_ALIGNMENT),
+])
+def test_noalloc_argument_errors_come_before_device_setup(args, status):
+    """attn_fwd_splitkv_noalloc checks every argument before its one-time
+    device set-up: on this GPU-less host any CUDA call would fail with
+    ATTN_ERR_CUDA or ATTN_ERR_UNSUPPORTED instead of the argument error."""
+    kw = dict(q=A, k=A, v=A, out=A, lse=None, B=1, Hq=2, Hkv=2, Nq=8, Nk=8, d=64,
+              scale=0.0, is_causal=0, key_lens=None, additive_mask=None, mask_strides=None, n_splits=0)
+    kw.update(args)
+    assert ea.attn_fwd_splitkv_noalloc(**kw) == status
+
+
+def test_exp2_selftest_argument_errors():
+    lib = ea.lib()
+    assert lib.attn_selftest_exp2_poly(None, None, -1, None) == ea.ATTN_ERR_INVALID_ARG
+    assert lib.attn_selftest_exp2_poly(None, None, 4, None) == ea.ATTN_ERR_INVALID_ARG
+    assert lib.attn_selftest_exp2_poly(A + 2, A, 4, None) == ea.ATTN_ERR_ALIGNMENT
+    assert lib.attn_selftest_exp2_poly(None, None, 0, None) == ea.ATTN_OK  # nothing to do

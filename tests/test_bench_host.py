@@ -25,10 +25,11 @@ def test_split_kv_with_many_rows_per_kv_head_uses_the_tile_kernel():
     assert bench.kernel_family(w) == "tile"
 
 
-def write_profile(root, name, traffic, sha):
+def write_traffic(root, name, traffic, sha):
+    import json
     os.makedirs(os.path.join(root, "profiles"), exist_ok=True)
-    with open(os.path.join(root, "profiles", f"attn_fwd_{name}.md"), "w") as f:
-        f.write(f"# summary\n\ntraffic_bytes_per_launch: {traffic}\nkernel_source_sha: {sha}\n")
+    with open(os.path.join(root, "profiles", "traffic.json"), "w") as f:
+        json.dump({f"attn_fwd_{name}": {"traffic_bytes_per_launch": traffic, "kernel_source_sha": sha}}, f)
 
 
 def test_recorded_traffic_only_for_the_sources_it_was_taken_on(tmp_path, monkeypatch):
@@ -37,11 +38,22 @@ def test_recorded_traffic_only_for_the_sources_it_was_taken_on(tmp_path, monkeyp
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     # the current sources' hash (the temporary root holds no sources)
     monkeypatch.setattr(bench, "kernel_source_hash", lambda family="tile": sha)
-    assert bench.recorded_traffic(w) is None  # no summary
-    write_profile(str(tmp_path), "long", 123456, "0" * 16)
-    assert bench.recorded_traffic(w) is None  # summary of other sources
-    write_profile(str(tmp_path), "long", 123456, sha)
+    assert bench.recorded_traffic(w) is None  # no record
+    write_traffic(str(tmp_path), "long", 123456, "0" * 16)
+    assert bench.recorded_traffic(w) is None  # record of other sources
+    write_traffic(str(tmp_path), "long", 123456, sha)
     assert bench.recorded_traffic(w) == 123456.0
+    write_traffic(str(tmp_path), "vit", 1, sha)
+    assert bench.recorded_traffic(w) is None  # another workload's record
+
+
+def test_committed_traffic_records_are_well_formed():
+    import json
+    recs = json.load(open(os.path.join(os.path.dirname(bench.__file__), "profiles", "traffic.json")))
+    for key, rec in recs.items():
+        assert key.startswith(("attn_fwd_", "attn_bwd_"))
+        assert rec["traffic_bytes_per_launch"] > 0 and len(rec["kernel_source_sha"]) == 16
+        assert os.path.exists(os.path.join(os.path.dirname(bench.__file__), "profiles", rec["summary"]))
 
 
 def test_kernel_source_hash_depends_on_family_sources():

@@ -20,7 +20,7 @@ import exact_attention_157_b200 as ea
 import oracle
 from workloads import make_qkv
 
-from test_parity_gpu import bf16_half_ulp
+from tolerances import bf16_half_ulp
 
 pytestmark = pytest.mark.gpu
 

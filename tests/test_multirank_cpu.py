@@ -52,7 +52,7 @@ def _reference_worker(rank, world, port, results):
     buf = io.StringIO()
     with contextlib.redirect_stdout(buf):
         bench.main(["--impl", "reference", "--workload", "tiny", "--steps", "1", "--warmup", "3",
-                    "--reference-seconds", "2"])
+                    "--reference-seconds", "2", "--gpus", str(world)])
     results[rank] = buf.getvalue()
 
 
@@ -74,3 +74,29 @@ def test_single_rank_helpers_are_identity():
     import bench
     assert bench.max_over_ranks(3.25, 1) == 3.25
     bench.barrier(1)
+
+
+def test_bench_launches_its_own_ranks():
+    """`bench.py --gpus 2` without a launcher starts two ranks itself
+    (torch.distributed.run on 127.0.0.1); here through the reference arm, which
+    needs no GPU: rank 0 prints the one JSON line, with n_gpus = 2."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_PORT")}
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--gpus", "2",
+                        "--workload", "tiny", "--steps", "1", "--warmup", "3", "--reference-seconds", "2"],
+                       cwd=root, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    line = json.loads(lines[0])
+    assert line["n_gpus"] == 2 and line["impl"] == "reference"
+
+
+def test_bench_rejects_a_world_size_that_differs_from_gpus(monkeypatch):
+    import bench
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    with pytest.raises(SystemExit):
+        bench.main(["--impl", "reference", "--workload", "tiny", "--gpus", "4"])

@@ -9,7 +9,8 @@ import exact_attention_157_b200 as ea
 import oracle
 from workloads import make_qkv
 
-from test_parity_gpu import assert_close, run_gpu
+from test_parity_gpu import run_gpu
+from tolerances import assert_close, reference
 
 pytestmark = pytest.mark.gpu
 
@@ -20,8 +21,8 @@ def check(B, Hq, Hkv, Nq, Nk, d, seed, softcap=0.0, mask2d=None, causal=False, k
     if key_lens is not None:
         kw["key_lens"] = torch.tensor(key_lens, dtype=torch.int32)
     out, lse = run_gpu(q, k, v, **kw)
-    ro, rl = oracle.attention(q, k, v, is_causal=causal, softcap=softcap, mask2d=mask2d, key_lens=key_lens)
-    assert_close(out, lse, ro, rl)
+    ro, rl, ra = reference(q, k, v, is_causal=causal, softcap=softcap, mask2d=mask2d, key_lens=key_lens)
+    assert_close(out, lse, ro, rl, rabs=ra)
 
 
 @pytest.mark.parametrize("cap", [30.0, 5.0, 1.0])

@@ -10,7 +10,7 @@ import exact_attention_157_b200 as ea
 import oracle
 from workloads import make_qkv
 
-from test_parity_gpu import assert_close
+from tolerances import assert_close, reference
 
 pytestmark = pytest.mark.gpu
 
@@ -22,20 +22,21 @@ def _inputs(B, Hq, Hkv, Nq, Nk, d, seed):
     return q, k, v, q.to(DEV), k.to(DEV), v.to(DEV)
 
 
-def _noalloc(qd, kd, vd, B, Hq, Hkv, Nq, Nk, d, n_splits, key_lens=None, causal=False):
+def _noalloc(qd, kd, vd, B, Hq, Hkv, Nq, Nk, d, n_splits, key_lens=None, causal=False, mask=None):
     out = torch.empty_like(qd)
     lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=DEV)
     st = ea.attn_fwd_splitkv_noalloc(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), out.data_ptr(), lse.data_ptr(),
                                      B, Hq, Hkv, Nq, Nk, d, 0.0, causal,
                                      key_lens=None if key_lens is None else key_lens.data_ptr(),
+                                     additive_mask=None if mask is None else mask.data_ptr(),
                                      n_splits=n_splits, stream=ea._stream_handle(None))
     assert st == ea.ATTN_OK, ea.status_string(st)
     ea.check_device_status()
     return out, lse
 
 
-def _with_workspace(qd, kd, vd, B, Hq, Hkv, Nq, Nk, d, n_splits, key_lens=None, causal=False):
-    st, _, nbytes = ea.attn_splitkv_plan(B, Hq, Nq, Nk, d, n_splits, 0, Hkv=Hkv)
+def _with_workspace(qd, kd, vd, B, Hq, Hkv, Nq, Nk, d, n_splits, key_lens=None, causal=False, mask=None):
+    st, _, nbytes = ea.attn_splitkv_plan(B, Hq, Nq, Nk, d, n_splits, 0, Hkv=Hkv, is_causal=causal)
     assert st == ea.ATTN_OK
     ws = torch.empty((max(nbytes, 1),), dtype=torch.uint8, device=DEV)
     out = torch.empty_like(qd)
@@ -43,6 +44,7 @@ def _with_workspace(qd, kd, vd, B, Hq, Hkv, Nq, Nk, d, n_splits, key_lens=None, 
     st = ea.attn_fwd_splitkv(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), out.data_ptr(), lse.data_ptr(),
                              B, Hq, Hkv, Nq, Nk, d, 0.0, causal,
                              key_lens=None if key_lens is None else key_lens.data_ptr(),
+                             additive_mask=None if mask is None else mask.data_ptr(),
                              n_splits=n_splits, workspace=ws.data_ptr(), workspace_bytes=nbytes,
                              stream=ea._stream_handle(None))
     assert st == ea.ATTN_OK, ea.status_string(st)
@@ -58,12 +60,39 @@ def _with_workspace(qd, kd, vd, B, Hq, Hkv, Nq, Nk, d, n_splits, key_lens=None, 
 def test_noalloc_matches_workspace_entry_point_twice(B, Hq, Hkv, Nq, Nk, d, n_splits):
     q, k, v, qd, kd, vd = _inputs(B, Hq, Hkv, Nq, Nk, d, seed=B * 100 + Nq + Nk + d)
     ref_o, ref_l = _with_workspace(qd, kd, vd, B, Hq, Hkv, Nq, Nk, d, n_splits)
-    ro, rl = oracle.attention(q, k, v)
+    ro, rl, ra = reference(q, k, v)
     for _ in range(2):  # two calls in a row reuse the same scratch
         out, lse = _noalloc(qd, kd, vd, B, Hq, Hkv, Nq, Nk, d, n_splits)
         assert (out.float() - ref_o.float()).abs().max().item() <= 1e-2
         assert (lse - ref_l).abs().max().item() <= 1e-3
-        assert_close(out, lse, ro, rl)
+        assert_close(out, lse, ro, rl, rabs=ra)
+
+
+@pytest.mark.parametrize("case", ["causal", "decode_shape_with_mask"])
+def test_noalloc_causal_and_masked_decode_shape_twice(case):
+    """The two other plan branches: a causal call (tile kernel, key ranges that
+    end at the diagonal), and a decoding shape given an additive mask, which runs
+    the tile kernel with the range count of the decode plan."""
+    if case == "causal":
+        B, Hq, Hkv, Nq, Nk, d, n_splits = 2, 4, 2, 700, 700, 64, 3
+    else:
+        B, Hq, Hkv, Nq, Nk, d, n_splits = 2, 8, 2, 2, 2500, 128, 0
+    q, k, v, qd, kd, vd = _inputs(B, Hq, Hkv, Nq, Nk, d, seed=29 + Nk)
+    mask = None
+    if case != "causal":
+        g = torch.Generator().manual_seed(30)
+        mask = torch.randn(B, Hq, Nq, Nk, generator=g) * 2.0
+        mask[0, 1, 0, 600:] = -float("inf")
+    causal = case == "causal"
+    md = None if mask is None else mask.to(DEV)
+    ref_o, ref_l = _with_workspace(qd, kd, vd, B, Hq, Hkv, Nq, Nk, d, n_splits, causal=causal, mask=md)
+    ro, rl, ra = reference(q, k, v, is_causal=causal, mask=None if mask is None else mask.double().numpy())
+    for _ in range(2):
+        out, lse = _noalloc(qd, kd, vd, B, Hq, Hkv, Nq, Nk, d, n_splits, causal=causal, mask=md)
+        assert (out.float() - ref_o.float()).abs().max().item() <= 1e-2
+        assert (lse - ref_l).abs().max().item() <= 1e-3
+        assert_close(out, lse, ro, rl, rabs=ra)
+        assert_close(ref_o, ref_l, ro, rl, rabs=ra)
 
 
 def test_noalloc_key_lens_twice_and_no_new_device_memory():
