@@ -21,6 +21,8 @@ Contents
 ``dequantize_blocks``,   (1 sign, 4 exponent bits with bias 7, 3 mantissa bits, subnormals,
 ``attention_fp8``        no infinities, S.1111.111 = NaN) and per-128-row block scales;
                          the result is the definition on the dequantized values.
+``e4m3_encode``,         the value -> code map (round to nearest even) and the block
+``quantize_e4m3_blocks`` quantiser (scale = block amax / 448), in fp32 arithmetic.
 
 Sources: "FlashAttention technical analysis" (jsqmd.com/news/722897) section 2.1
 (the three steps), section 2.2 (tiling plus online softmax with running max and
@@ -110,6 +112,14 @@ def _bind_bwd(path):
         dp, dp, dp, dp, dp, dp, dp,
         ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
         ctypes.c_double, ctypes.c_int, ip, ip, ctypes.c_int, ctypes.c_int]
+    lib.oracle_attention_bwd_mod.restype = ctypes.c_int
+    lib.oracle_attention_bwd_mod.argtypes = [
+        dp, dp, dp, dp, dp, dp, dp,
+        ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+        ctypes.c_double, ctypes.c_int, ip,
+        dp, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+        ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+        ip, ctypes.c_int, ctypes.c_int]
     return lib
 
 
@@ -138,11 +148,14 @@ def compile_variant_bwd(src_text: str, out_path: str):
 
 
 def attention_bwd(q, k, v, dout, *, scale: float | None = None, is_causal: bool = False, key_lens=None,
-                  units=None, n_threads: int = 0, lib=None):
+                  units=None, n_threads: int = 0, lib=None, mask=None, softcap: float = 0.0, mask2d=None):
     """Gradients of the definition for the upstream gradient ``dout`` (fp64).
 
     q, dout: [B, Hq, Nq, d]; k, v: [B, Hkv, Nk, d]; key_lens: [B] or None;
     units: optional list of b * Hkv + hkv pairs to compute (others are NaN).
+    mask: additive mask broadcastable to [B, Hq, Nq, Nk]; softcap: cap of the
+    soft-capped score (0: off); mask2d: None, ("neighborhood", W, R) or
+    ("window", W, w[, shift]), as in ``attention``.
     Returns (dQ [B, Hq, Nq, d], dK [B, Hkv, Nk, d], dV [B, Hkv, Nk, d]).
     """
     q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(dout)
@@ -155,10 +168,19 @@ def attention_bwd(q, k, v, dout, *, scale: float | None = None, is_causal: bool 
     dv = np.full(v.shape, np.nan)
     kl = None if key_lens is None else np.ascontiguousarray(np.asarray(key_lens, dtype=np.int32))
     un = None if units is None else np.ascontiguousarray(np.asarray(units, dtype=np.int32))
-    rc = (lib or _load_bwd()).oracle_attention_bwd(
+    mk, sb, sh, sq = None, 0, 0, 0
+    if mask is not None:
+        mk, sb, sh, sq = _mask_view(mask, B, Hq, Nq, Nk)
+    kind, W, size, shift = 0, 1, 1, 0
+    if mask2d is not None:
+        kind = {"neighborhood": 1, "window": 2}[mask2d[0]]
+        W, size = int(mask2d[1]), int(mask2d[2])
+        shift = int(mask2d[3]) if len(mask2d) > 3 else 0
+    rc = (lib or _load_bwd()).oracle_attention_bwd_mod(
         _ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv),
         B, Hq, Hkv, Nq, Nk, d, float(scale), int(bool(is_causal)),
-        _ptr(kl, ctypes.c_int32), _ptr(un, ctypes.c_int32), 0 if un is None else len(un), int(n_threads))
+        _ptr(kl, ctypes.c_int32), _ptr(mk), sb, sh, sq, float(softcap or 0.0), kind, W, size, shift,
+        _ptr(un, ctypes.c_int32), 0 if un is None else len(un), int(n_threads))
     if rc != 0:
         raise ValueError(f"oracle_attention_bwd rejected its arguments (status {rc})")
     return dq, dk, dv
@@ -284,6 +306,56 @@ def dequantize_blocks(codes, scales, block: int = 128) -> np.ndarray:
     n = x.shape[-2]
     idx = np.arange(n) // block
     return x * s[..., idx][..., None]
+
+
+def e4m3_encode(y) -> np.ndarray:
+    """E4M3 code (uint8) of each fp32 value y, |y| <= 448, rounded to the nearest
+    representable value with ties to the even code: written from the format
+    (1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits; exponent field 0
+    holds the subnormals m / 8 * 2^-6; the largest finite value is 1.75 * 2^8 =
+    448).  The sign bit is taken from y's sign bit (-0.0 gives 0x80)."""
+    y = np.asarray(y, dtype=np.float32)
+    if (np.abs(y) > 448.0).any() or np.isnan(y).any():
+        raise ValueError("e4m3_encode: values must be finite and within [-448, 448]")
+    a = np.abs(y).astype(np.float64)  # exact
+    sign = np.signbit(y).astype(np.int64) << 7
+    # binade of each value (normals: exponent e in [-6, 8]); subnormals use e = -6
+    with np.errstate(divide="ignore"):
+        e = np.floor(np.log2(np.where(a > 0, a, 1.0))).astype(np.int64)
+    e = np.maximum(e, -6)
+    # the value in units of the grid spacing 2^(e - 3) of its binade, rounded half to even
+    units = np.rint(a / np.exp2(e - 3.0)).astype(np.int64)  # 8..16 for normals, 0..8 below 2^-6
+    normal = a >= 2.0 ** -6
+    carry = units == 16  # rounded up to the next binade
+    e = np.where(carry, e + 1, e)
+    units = np.where(carry, 8, units)
+    code_normal = ((e + 7) << 3) | (units - 8)
+    code_sub = units  # units of 2^-9; 8 means exactly 2^-6, code 0x08, the first normal
+    code = np.where(normal, code_normal, code_sub)
+    return (sign | code).astype(np.uint8)
+
+
+def quantize_e4m3_blocks(x, block: int = 128):
+    """FP8 block quantisation of x [..., N, d] ("each block keeps its own scale
+    factor", "FlashAttention technical analysis", jsqmd.com/news/722897,
+    section 6.3): per block of `block` rows of each head, in fp32 arithmetic,
+      amax = max |x| over the block,  scale = amax / 448 (1 when amax = 0),
+      code = e4m3(min(max(x / scale, -448), 448))
+    with the division and e4m3 both rounding to nearest even.  Returns (codes
+    uint8 [..., N, d], scales fp32 [..., ceil(N / block)])."""
+    x = np.asarray(x, dtype=np.float32)
+    n = x.shape[-2]
+    nb = (n + block - 1) // block
+    scales = np.empty(x.shape[:-2] + (nb,), dtype=np.float32)
+    codes = np.empty(x.shape, dtype=np.uint8)
+    for j in range(nb):
+        xb = x[..., j * block:(j + 1) * block, :]
+        amax = np.abs(xb).max(axis=(-1, -2))
+        sc = np.where(amax > 0, (amax / np.float32(448.0)).astype(np.float32), np.float32(1.0)).astype(np.float32)
+        scales[..., j] = sc
+        y = (xb / sc[..., None, None]).astype(np.float32)  # fp32, correctly rounded
+        codes[..., j * block:(j + 1) * block, :] = e4m3_encode(np.clip(y, np.float32(-448.0), np.float32(448.0)))
+    return codes, scales
 
 
 def attention_fp8(q8, k8, v8, q_scale, k_scale, v_scale, **kw):

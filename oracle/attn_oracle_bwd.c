@@ -21,6 +21,16 @@
  * K/V gradients of a K/V head are the sums over the query heads that read it.
  * A row with no unmasked key has P = 0: it contributes nothing and gets dQ = 0.
  *
+ * Variants (oracle_attention_bwd_mod), the same readings as the forward
+ * oracle's oracle_attention_fwd_mod: the score is
+ *   s_ij = c(x_ij) + mask_ij,  x_ij = scale * <q_i, k_j>,
+ * with c(x) = cap * tanh(x / cap) under soft-capping (else c(x) = x), an
+ * additive mask added after it, and the 2-D neighbourhood / window masks
+ * setting s_ij = -inf outside the query's grid rectangle.  The chain rule
+ * through c gives dL/dx_ij = dS_ij * c'(x_ij), c'(x) = 1 - tanh^2(x / cap);
+ * dQ and dK then follow from x as above.  The mask has no parameter to
+ * differentiate.
+ *
  * Every step is fp64; units of work are (batch, K/V head) pairs spread over
  * POSIX threads, each computed by the plain sequence below.
  */
@@ -40,7 +50,29 @@ typedef struct {
     const int32_t *key_lens;
     const int32_t *units; /* optional subset of b * Hkv + hkv */
     int n_units;
+    const double *mask;                /* additive mask or NULL */
+    int64_t mask_sb, mask_sh, mask_sq; /* its element strides */
+    double softcap;                    /* 0: off */
+    int m2_kind, m2_w, m2_size, m2_shift;
 } bwd_args;
+
+/* Whether the 2-D mask lets query i see key j (the forward oracle's rule). */
+static int bwd_allowed_2d(const bwd_args *a, int i, int j)
+{
+    if (a->m2_kind == 0) return 1;
+    const int W = a->m2_w;
+    const int ri = i / W, ci = i % W, rj = j / W, cj = j % W;
+    if (a->m2_kind == 1) {
+        const int dr = ri > rj ? ri - rj : rj - ri;
+        const int dc = ci > cj ? ci - cj : cj - ci;
+        return dr < a->m2_size && dc < a->m2_size;
+    }
+    if (a->m2_kind == 2) {
+        const int w = a->m2_size, sh = a->m2_shift;
+        return (ri + sh) / w == (rj + sh) / w && (ci + sh) / w == (cj + sh) / w;
+    }
+    return 1;
+}
 
 typedef struct {
     const bwd_args *a;
@@ -49,7 +81,7 @@ typedef struct {
 } bwd_job;
 
 /* One (batch, K/V head) pair: every query head of its group. */
-static int bwd_unit(const bwd_args *a, int b, int hk, double *P, double *dP)
+static int bwd_unit(const bwd_args *a, int b, int hk, double *P, double *dP, double *C)
 {
     const int Nq = a->Nq, Nk = a->Nk, d = a->d;
     const int group = a->Hq / a->Hkv;
@@ -65,18 +97,30 @@ static int bwd_unit(const bwd_args *a, int b, int hk, double *P, double *dP)
         const int64_t qh = ((int64_t)b * a->Hq + h) * (int64_t)Nq * d;
         const double *Q = a->q + qh, *dO = a->dout + qh;
         double *dQ = a->dq + qh;
-        /* P: scores, masks, row softmax (two passes) */
+        /* P: scores, masks, row softmax (two passes); C: the derivative c'(x) of the
+         * score variant (1 without soft-capping) */
         for (int i = 0; i < Nq; ++i) {
             double *p = P + (int64_t)i * Nk;
+            double *c = C + (int64_t)i * Nk;
+            const double *mrow = a->mask
+                ? a->mask + (int64_t)b * a->mask_sb + (int64_t)h * a->mask_sh + (int64_t)i * a->mask_sq
+                : NULL;
             double M = -INFINITY;
             for (int j = 0; j < Nk; ++j) {
-                if (j >= len || (a->is_causal && j > i)) {
+                c[j] = 1.0;
+                if (j >= len || (a->is_causal && j > i) || !bwd_allowed_2d(a, i, j)) {
                     p[j] = -INFINITY;
                     continue;
                 }
                 double dot = 0.0;
                 for (int t = 0; t < d; ++t) dot += Q[(int64_t)i * d + t] * K[(int64_t)j * d + t];
                 p[j] = a->scale * dot;
+                if (a->softcap > 0.0) {
+                    const double th = tanh(p[j] / a->softcap);
+                    p[j] = a->softcap * th;
+                    c[j] = 1.0 - th * th;
+                }
+                if (mrow) p[j] += mrow[j];
                 if (p[j] > M) M = p[j];
             }
             if (M == -INFINITY) {
@@ -102,6 +146,9 @@ static int bwd_unit(const bwd_args *a, int b, int hk, double *P, double *dP)
                 D += p[j] * s;
             }
             for (int j = 0; j < Nk; ++j) dp[j] = p[j] * (dp[j] - D);
+            /* through the score variant: dL/dx = dS * c'(x) */
+            const double *c = C + (int64_t)i * Nk;
+            for (int j = 0; j < Nk; ++j) dp[j] *= c[j];
         }
         /* dQ = scale * dS K */
         for (int i = 0; i < Nq; ++i)
@@ -131,19 +178,35 @@ static void *bwd_worker(void *p)
     const bwd_args *a = job->a;
     double *P = (double *)malloc(sizeof(double) * (size_t)a->Nq * (size_t)a->Nk);
     double *dP = (double *)malloc(sizeof(double) * (size_t)a->Nq * (size_t)a->Nk);
-    if (!P || !dP) {
-        free(P); free(dP);
+    double *C = (double *)malloc(sizeof(double) * (size_t)a->Nq * (size_t)a->Nk);
+    if (!P || !dP || !C) {
+        free(P); free(dP); free(C);
         job->status = -2;
         return NULL;
     }
     for (int u = job->first; u < job->last; ++u) {
         const int id = a->units ? a->units[u] : u;
-        bwd_unit(a, id / a->Hkv, id % a->Hkv, P, dP);
+        bwd_unit(a, id / a->Hkv, id % a->Hkv, P, dP, C);
     }
-    free(P); free(dP);
+    free(P); free(dP); free(C);
     job->status = 0;
     return NULL;
 }
+
+/*
+ * oracle_attention_bwd_mod -- oracle_attention_bwd with the score and mask
+ * variants: mask (fp64, element (b, h, i, j) at b*mask_sb + h*mask_sh +
+ * i*mask_sq + j, or NULL), softcap (0: off), m2_kind (0 none, 1 neighbourhood
+ * of radius m2_size, 2 windows of side m2_size displaced by m2_shift) on a
+ * grid of m2_w tokens per row.
+ */
+int oracle_attention_bwd_mod(const double *q, const double *k, const double *v, const double *dout,
+                             double *dq, double *dk, double *dv,
+                             int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                             double scale, int is_causal, const int32_t *key_lens,
+                             const double *mask, int64_t mask_sb, int64_t mask_sh, int64_t mask_sq,
+                             double softcap, int m2_kind, int m2_w, int m2_size, int m2_shift,
+                             const int32_t *units, int n_units, int n_threads);
 
 /*
  * oracle_attention_bwd
@@ -160,17 +223,32 @@ int oracle_attention_bwd(const double *q, const double *k, const double *v, cons
                          double scale, int is_causal, const int32_t *key_lens,
                          const int32_t *units, int n_units, int n_threads)
 {
+    return oracle_attention_bwd_mod(q, k, v, dout, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale, is_causal, key_lens,
+                                    NULL, 0, 0, 0, 0.0, 0, 1, 1, 0, units, n_units, n_threads);
+}
+
+int oracle_attention_bwd_mod(const double *q, const double *k, const double *v, const double *dout,
+                             double *dq, double *dk, double *dv,
+                             int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                             double scale, int is_causal, const int32_t *key_lens,
+                             const double *mask, int64_t mask_sb, int64_t mask_sh, int64_t mask_sq,
+                             double softcap, int m2_kind, int m2_w, int m2_size, int m2_shift,
+                             const int32_t *units, int n_units, int n_threads)
+{
     if (!q || !k || !v || !dout || !dq || !dk || !dv) return -1;
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nk <= 0 || d <= 0 || Hq % Hkv != 0) return -1;
     if (key_lens)
         for (int b = 0; b < B; ++b)
             if (key_lens[b] < 0 || key_lens[b] > Nk) return -1;
+    if (softcap < 0.0 || m2_kind < 0 || m2_kind > 2 || (m2_kind && (m2_w <= 0 || m2_size <= 0 || m2_shift < 0)))
+        return -1;
     const int total = units ? n_units : B * Hkv;
     if (units)
         for (int u = 0; u < n_units; ++u)
             if (units[u] < 0 || units[u] >= B * Hkv) return -1;
     if (total <= 0) return -1;
-    bwd_args a = {q, k, v, dout, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale, is_causal, key_lens, units, n_units};
+    bwd_args a = {q, k, v, dout, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale, is_causal, key_lens, units, n_units,
+                  mask, mask_sb, mask_sh, mask_sq, softcap, m2_kind, m2_w, m2_size, m2_shift};
     if (n_threads <= 0) n_threads = (int)sysconf(_SC_NPROCESSORS_ONLN);
     if (n_threads < 1) n_threads = 1;
     if (n_threads > total) n_threads = total;
