@@ -40,7 +40,7 @@ NOALLOC_SCRATCH_BYTES = 16 << 20  # ATTN_NOALLOC_SCRATCH_BYTES
 # Every symbol include/attn.h declares.
 EXPORTED = ("attn_fwd", "attn_fwd_mod", "attn_fwd_fp8", "attn_bwd_plan", "attn_bwd", "attn_splitkv_plan", "attn_fwd_splitkv", "attn_fwd_splitkv_noalloc",
             "attn_check_device_status", "attn_set_wait_timeout_ns", "attn_selftest_timeout",
-            "attn_selftest_exp2_poly", "attn_status_string", "attn_last_cuda_error", "attn_version")
+            "attn_selftest_exp2_poly", "attn_quantize_e4m3_blocks", "attn_bwd_ex", "attn_status_string", "attn_last_cuda_error", "attn_version")
 
 MASK2D_KINDS = {None: 0, "neighborhood": 1, "window": 2}
 
@@ -112,6 +112,11 @@ def lib() -> ctypes.CDLL:
             L.attn_selftest_timeout.argtypes = [vp]
             L.attn_selftest_exp2_poly.restype = i
             L.attn_selftest_exp2_poly.argtypes = [vp, vp, i, vp]
+            L.attn_quantize_e4m3_blocks.restype = i
+            L.attn_quantize_e4m3_blocks.argtypes = [vp, vp, vp, i, i, i, vp]
+            L.attn_bwd_ex.restype = i
+            L.attn_bwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, vp, vp, vp,
+                                      ctypes.POINTER(AttnScoreMod), vp, ctypes.c_size_t, vp]
             L.attn_status_string.restype = ctypes.c_char_p
             L.attn_status_string.argtypes = [i]
             L.attn_last_cuda_error.restype = i
@@ -228,6 +233,24 @@ def attn_set_wait_timeout_ns(ns: int) -> int:
 
 def attn_selftest_timeout(stream=None) -> int:
     return int(lib().attn_selftest_timeout(stream))
+
+
+def quantize_e4m3_blocks(x, stream=None):
+    """FP8 E4M3 block quantisation of a contiguous bf16 CUDA tensor [..., N, d]
+    on the device (attn_quantize_e4m3_blocks): returns (codes uint8 [..., N, d],
+    scales fp32 [..., ceil(N / 128)]), the inputs of attention_fp8."""
+    import torch
+    if not (x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous() and x.dim() >= 2):
+        raise TypeError("x must be a contiguous bfloat16 CUDA tensor [..., N, d]")
+    N, d = x.shape[-2], x.shape[-1]
+    heads = x.numel() // (N * d) if N * d > 0 else 0
+    codes = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    scales = torch.empty(tuple(x.shape[:-2]) + ((N + 127) // 128,), dtype=torch.float32, device=x.device)
+    st = int(lib().attn_quantize_e4m3_blocks(x.data_ptr(), codes.data_ptr(), scales.data_ptr(), int(heads), int(N),
+                                             int(d), _stream_handle(stream)))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_quantize_e4m3_blocks")
+    return codes, scales
 
 
 def exp2_poly(x, stream=None):
@@ -393,10 +416,12 @@ def attention_fp8(q8, k8, v8, q_scale, k_scale, v_scale, *, scale: float | None 
 
 
 def attention_backward(q, k, v, out, lse, dout, *, scale: float | None = None, is_causal: bool = False,
-                       key_lens=None, workspace=None, stream=None, dq=None, dk=None, dv=None):
+                       key_lens=None, workspace=None, stream=None, dq=None, dk=None, dv=None,
+                       attn_mask=None, softcap: float = 0.0, mask2d=None):
     """dQ, dK, dV of ``attention`` for the upstream gradient ``dout`` (bf16 CUDA
     tensors shaped like q / k / v); ``out`` and ``lse`` are the forward results
-    for the same inputs.  Returns (dq, dk, dv)."""
+    for the same inputs and options (attn_mask, softcap, mask2d as in
+    ``attention``).  Returns (dq, dk, dv)."""
     import torch
     for name, t, nd in (("q", q, 4), ("k", k, 4), ("v", v, 4), ("out", out, 4), ("dout", dout, 4)):
         _check_bf16_cuda(name, t, nd)
@@ -422,12 +447,34 @@ def attention_backward(q, k, v, out, lse, dout, *, scale: float | None = None, i
     if key_lens is not None:
         key_lens = key_lens.contiguous()
         kl_ptr = key_lens.data_ptr()
-    st = attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), dout.data_ptr(),
-                  dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, Nq, Nk, d,
-                  0.0 if scale is None else float(scale), is_causal, kl_ptr, workspace.data_ptr(),
-                  workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    sc = 0.0 if scale is None else float(scale)
+    if attn_mask is None and not softcap and mask2d is None:
+        st = attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), dout.data_ptr(),
+                      dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, Nq, Nk, d, sc, is_causal, kl_ptr,
+                      workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream_handle(stream))
+        if st != ATTN_OK:
+            raise AttnError(st, "attn_bwd")
+        return dq, dk, dv
+    m_ptr, ms = None, None
+    if attn_mask is not None:
+        if attn_mask.dtype != torch.float32 or attn_mask.device != q.device:
+            raise ValueError("attn_mask must be a float32 CUDA tensor")
+        m = attn_mask
+        while m.dim() < 4:
+            m = m.unsqueeze(0)
+        m = m.expand(B, Hq, Nq, Nk)
+        if m.stride(3) != 1:
+            m = m.contiguous()
+        m_ptr = m.data_ptr()
+        ms = ctypes.cast((ctypes.c_int64 * 3)(m.stride(0), m.stride(1), m.stride(2)), ctypes.c_void_p)
+    mod = score_mod(softcap, mask2d) if (softcap or mask2d is not None) else None
+    st = int(lib().attn_bwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                               dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, Nq, Nk, d,
+                               sc, int(bool(is_causal)), kl_ptr, m_ptr, ms,
+                               None if mod is None else ctypes.byref(mod), workspace.data_ptr(),
+                               workspace.numel() * workspace.element_size(), _stream_handle(stream)))
     if st != ATTN_OK:
-        raise AttnError(st, "attn_bwd")
+        raise AttnError(st, "attn_bwd_ex")
     return dq, dk, dv
 
 
@@ -441,15 +488,20 @@ def check_device_status(stream=None):
 class HostAttention:
     """End-to-end call for inputs that live in (pinned) host memory.
 
-    Each call copies Q, K, V (and key lengths) host -> device on ``stream``,
-    runs ``attn_fwd`` and copies O and LSE back into the host tensors it was
-    given; the device staging buffers (and a split-KV workspace when
-    ``split_kv`` is not None, planned for ``is_causal``) are allocated once,
-    here, and reused.
+    The batch is cut into ``chunks`` parts that flow through three streams:
+    chunk c+1 is copied host -> device while the kernel runs on chunk c and
+    chunk c-1's O and LSE are copied back, so the two copy directions and the
+    kernels overlap (each copy direction has its own engine).  The call is
+    ordered on ``stream``: it starts after the work already queued there and
+    everything it does, the last copy back included, precedes the work queued
+    there after it.  The device staging buffers (and a split-KV workspace when
+    ``split_kv`` is not None, planned for ``is_causal``), the two copy streams
+    and their events are made once, here, and reused.  With ``split_kv=0``
+    (automatic) each chunk's key ranges are planned for the chunk's batch size.
     """
 
     def __init__(self, B, Hq, Hkv, Nq, Nk, d, device="cuda:0", with_lse=True, with_key_lens=False,
-                 split_kv=None, is_causal=False):
+                 split_kv=None, is_causal=False, chunks=None):
         import torch
         dev = torch.device(device)
         bf = torch.bfloat16
@@ -467,23 +519,38 @@ class HostAttention:
             if st != ATTN_OK:
                 raise AttnError(st, "attn_splitkv_plan")
             self.workspace = torch.empty((max(nbytes, 1),), dtype=torch.uint8, device=dev)
+        n = min(B, 8) if chunks is None else max(1, min(int(chunks), B))
+        self.bounds = [(B * i // n, B * (i + 1) // n) for i in range(n)]
+        self.h2d = torch.cuda.Stream(dev)
+        self.d2h = torch.cuda.Stream(dev)
+        self.ev_in = [torch.cuda.Event() for _ in self.bounds]
+        self.ev_out = [torch.cuda.Event() for _ in self.bounds]
 
     def __call__(self, q_h, k_h, v_h, out_h, lse_h=None, key_lens_h=None, *, scale=None,
                  is_causal=False, stream=None, softcap=0.0, mask2d=None):
         import torch
         s = torch.cuda.current_stream() if stream is None else stream
-        with torch.cuda.stream(s):
-            self.q.copy_(q_h, non_blocking=True)
-            self.k.copy_(k_h, non_blocking=True)
-            self.v.copy_(v_h, non_blocking=True)
-            kl = None
-            if key_lens_h is not None:
-                self.key_lens.copy_(key_lens_h, non_blocking=True)
-                kl = self.key_lens
-            attention(self.q, self.k, self.v, scale=scale, is_causal=is_causal, key_lens=kl,
-                      out=self.out, lse=self.lse, return_lse=self.lse is not None, stream=s,
+        # the staging buffers are free once the work queued on s (earlier calls included) is done
+        self.h2d.wait_stream(s)
+        for (b0, b1), ev_in, ev_out in zip(self.bounds, self.ev_in, self.ev_out):
+            with torch.cuda.stream(self.h2d):
+                self.q[b0:b1].copy_(q_h[b0:b1], non_blocking=True)
+                self.k[b0:b1].copy_(k_h[b0:b1], non_blocking=True)
+                self.v[b0:b1].copy_(v_h[b0:b1], non_blocking=True)
+                if key_lens_h is not None:
+                    self.key_lens[b0:b1].copy_(key_lens_h[b0:b1], non_blocking=True)
+                ev_in.record(self.h2d)
+            s.wait_event(ev_in)
+            kl = None if key_lens_h is None else self.key_lens[b0:b1]
+            lse = None if self.lse is None else self.lse[b0:b1]
+            attention(self.q[b0:b1], self.k[b0:b1], self.v[b0:b1], scale=scale, is_causal=is_causal, key_lens=kl,
+                      out=self.out[b0:b1], lse=lse, return_lse=lse is not None, stream=s,
                       split_kv=self.split_kv, workspace=self.workspace, softcap=softcap, mask2d=mask2d)
-            out_h.copy_(self.out, non_blocking=True)
-            if lse_h is not None and self.lse is not None:
-                lse_h.copy_(self.lse, non_blocking=True)
+            ev_out.record(s)
+            self.d2h.wait_event(ev_out)
+            with torch.cuda.stream(self.d2h):
+                out_h[b0:b1].copy_(self.out[b0:b1], non_blocking=True)
+                if lse_h is not None and lse is not None:
+                    lse_h[b0:b1].copy_(lse, non_blocking=True)
+        s.wait_stream(self.d2h)  # the copies back complete before later work on s
         return out_h, lse_h

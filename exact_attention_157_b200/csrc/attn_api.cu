@@ -15,6 +15,8 @@
 #include "fwd_kernel_pp.cuh"
 #include "bwd_kernels.cuh"
 #include "decode_kernel.cuh"
+#include "short_kernel.cuh"
+#include "quant_kernel.cuh"
 
 using namespace attn_sm100;
 
@@ -56,6 +58,9 @@ constexpr int kSlots128 = 5, kQStages128 = 1;
 constexpr int kSlots64 = 8, kQStages64 = 2;
 // FP8 (d = 128): 16 KB tiles, so two Q buffers and 8 K/V slots
 constexpr int kSlotsF8 = 8, kQStagesF8 = 2;
+// Short-key kernel: all the shared memory a CTA may have (227 KB); the K/V
+// buffers take what the key count needs and the Q ring the rest.
+constexpr int kShortSmemMax = 232448;
 using SmemF8 = SmemPPFor<128, kSlotsF8, kQStagesF8, true>;
 
 template <int D, int NSLOT, int QS, bool M>
@@ -73,10 +78,16 @@ cudaError_t set_pp_attrs() {
 
 template <int D>
 cudaError_t set_bwd_attrs() {
-    cudaError_t e = cudaFuncSetAttribute(attn_bwd_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(attn_bwd_kernel<D, true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          SmemBwd<D>::kAlloc);
     if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(attn_bwd_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(attn_bwd_kernel<D, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SmemBwd<D>::kAlloc);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(attn_bwd_kernel<D, true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SmemBwd<D>::kAlloc);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(attn_bwd_kernel<D, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 SmemBwd<D>::kAlloc);
 }
 
@@ -132,6 +143,9 @@ attn_status_t device_setup(int* dev_out) {
     if ((e = set_decode_attrs<128>()) != cudaSuccess) return cuda_fail(e);
     if ((e = set_decode_attrs<64>()) != cudaSuccess) return cuda_fail(e);
     if ((e = set_bwd_attrs<64>()) != cudaSuccess) return cuda_fail(e);
+    if ((e = cudaFuncSetAttribute(attn_fwd_short_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  kShortSmemMax)) != cudaSuccess)
+        return cuda_fail(e);
     st.ready = true;
     st.status = ATTN_OK;
     return ATTN_OK;
@@ -139,8 +153,8 @@ attn_status_t device_setup(int* dev_out) {
 
 // 3-D map over a [heads, rows, d] bf16 tensor, box = 64 columns x 128 rows x 1,
 // 128-byte swizzle (the layout the UMMA shared-memory descriptors expect).
-attn_status_t encode_map(CUtensorMap* map, const void* base, int d, int rows, long long heads,
-                         unsigned box_rows = 128u, bool fp8 = false) {
+attn_status_t encode_map_uncached(CUtensorMap* map, const void* base, int d, int rows, long long heads,
+                                  unsigned box_rows, bool fp8) {
     const cuuint64_t eb = fp8 ? 1u : 2u;  // bytes per element; a box row is 128 bytes either way
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(heads)};
     cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * eb, static_cast<cuuint64_t>(rows) * d * eb};
@@ -153,6 +167,56 @@ attn_status_t encode_map(CUtensorMap* map, const void* base, int d, int rows, lo
         g_last_cuda_error.store(static_cast<int>(r));
         return ATTN_ERR_CUDA;
     }
+    return ATTN_OK;
+}
+
+// Encoded maps are kept per (device, base, shape, box): a call on the same
+// buffers as an earlier one (the usual case in a serving or training loop)
+// copies a 128-byte descriptor instead of asking the driver again.  A map
+// holds only the address and the layout, never data, so a stale entry is
+// harmless; the table is small and replaced round-robin.
+struct MapKey {
+    const void* base;
+    long long heads;
+    int dev, d, rows;
+    unsigned box_rows;
+    bool fp8;
+    bool operator==(const MapKey& o) const {
+        return base == o.base && heads == o.heads && dev == o.dev && d == o.d && rows == o.rows &&
+               box_rows == o.box_rows && fp8 == o.fp8;
+    }
+};
+constexpr int kMapCache = 64;
+struct MapEntry {
+    MapKey key;
+    CUtensorMap map;
+    bool used;
+};
+MapEntry g_maps[kMapCache];
+int g_map_next = 0;
+std::mutex g_map_mutex;
+
+attn_status_t encode_map(CUtensorMap* map, const void* base, int d, int rows, long long heads,
+                         unsigned box_rows = 128u, bool fp8 = false) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
+    const MapKey key{base, heads, dev, d, rows, box_rows, fp8};
+    {
+        std::lock_guard<std::mutex> lock(g_map_mutex);
+        for (int i = 0; i < kMapCache; ++i)
+            if (g_maps[i].used && g_maps[i].key == key) {
+                *map = g_maps[i].map;
+                return ATTN_OK;
+            }
+    }
+    const attn_status_t st = encode_map_uncached(map, base, d, rows, heads, box_rows, fp8);
+    if (st != ATTN_OK) return st;
+    std::lock_guard<std::mutex> lock(g_map_mutex);
+    MapEntry& e = g_maps[g_map_next];
+    g_map_next = (g_map_next + 1) % kMapCache;
+    e.key = key;
+    e.map = *map;
+    e.used = true;
     return ATTN_OK;
 }
 
@@ -271,6 +335,48 @@ SplitPlan make_plan(int B, int Hq, int Hkv, int Nq, int Nk, int d, bool causal, 
 }
 
 
+// The short-key kernel (short_kernel.cuh): tiles of 128 query rows, K/V of a
+// head resident in shared memory across its tiles.
+attn_status_t launch_short(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
+                           int Hkv, int Nq, int Nk, float scale_log2, int is_causal, const int32_t* key_lens,
+                           unsigned long long timeout_ns, unsigned int epoch, int sm_count, void* stream) {
+    ShortParams sp{};
+    sp.B = B; sp.Hq = Hq; sp.Hkv = Hkv; sp.Nq = Nq; sp.Nk = Nk;
+    sp.n_qt = (Nq + 127) / 128;
+    sp.n_pad = (Nk + 15) / 16 * 16;
+    sp.kv_bytes = sp.n_pad * 128;
+    sp.tiles = static_cast<long long>(B) * Hq * sp.n_qt;
+    if (sp.tiles > (1LL << 30)) return ATTN_ERR_INVALID_ARG;  // tile indices stay in int range
+    const SmemShort base = SmemShort::make(sp.kv_bytes, 0);
+    sp.nq_stages = (kShortSmemMax - 1024 - base.bytes) / kShortTile;
+    if (sp.nq_stages > kShortMaxQ) sp.nq_stages = kShortMaxQ;
+    sp.scale_log2 = scale_log2;
+    sp.is_causal = is_causal ? 1 : 0;
+    sp.key_lens = key_lens;
+    sp.lse = lse;
+    sp.out = out;
+    sp.timeout_ns = timeout_ns;
+    sp.epoch = epoch;
+    sp.fd_qt = make_fast_div(static_cast<uint32_t>(sp.n_qt));
+    sp.fd_hq = make_fast_div(static_cast<uint32_t>(Hq));
+    sp.fd_group = make_fast_div(static_cast<uint32_t>(Hq / Hkv));
+    CUtensorMap tq, tk, tv, to;
+    attn_status_t st;
+    if ((st = encode_map(&tq, q, 64, Nq, static_cast<long long>(B) * Hq)) != ATTN_OK) return st;
+    if ((st = encode_map(&tk, k, 64, Nk, static_cast<long long>(B) * Hkv, static_cast<unsigned>(sp.n_pad))) != ATTN_OK)
+        return st;
+    if ((st = encode_map(&tv, v, 64, Nk, static_cast<long long>(B) * Hkv, static_cast<unsigned>(sp.n_pad))) != ATTN_OK)
+        return st;
+    if ((st = encode_map(&to, out, 64, Nq, static_cast<long long>(B) * Hq)) != ATTN_OK) return st;
+    const int sms = sm_count > 0 ? sm_count : 1;
+    const unsigned grid = static_cast<unsigned>(sp.tiles < sms ? sp.tiles : sms);
+    const int smem = SmemShort::make(sp.kv_bytes, sp.nq_stages).bytes + 1024;
+    attn_fwd_short_kernel<<<grid, kShortThreads, smem, static_cast<cudaStream_t>(stream)>>>(tq, tk, tv, to, sp);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e);
+    return ATTN_OK;
+}
+
 // Host-side argument checks of the forward entry points (no CUDA call); on
 // success the element strides of the additive mask are in msb, msh, msq.
 attn_status_t validate_fwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
@@ -375,6 +481,15 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, f
     }
     p.timeout_ns = g_timeout_ns.load();
     p.epoch = next_epoch();
+
+    // Short key sequences (d = 64, at most 256 keys, no additive mask or variant,
+    // one key range): the whole score row of a tile fits one tensor-memory
+    // accumulator, so the short-key kernel runs the exact softmax without rescaling.
+    if (d == 64 && Nk <= kShortMaxKeys && additive_mask == nullptr && !use_mod &&
+        (!split_kv || make_plan(B, Hq, Hkv, Nq, Nk, d, is_causal != 0, n_splits_req,
+                                g_dev[dev].sm_count > 0 ? g_dev[dev].sm_count : 1).n_splits == 1))
+        return launch_short(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, p.scale_log2, is_causal, key_lens,
+                            p.timeout_ns, p.epoch, g_dev[dev].sm_count, stream);
 
     CUtensorMap tq, tk, tv, to;
     if ((st = encode_map(&tq, q, d, Nq, static_cast<long long>(B) * Hq)) != ATTN_OK) return st;
@@ -671,7 +786,7 @@ size_t bwd_bytes(int B, int Hq, int Nq) {
     return 2 * round_up(static_cast<size_t>(B) * Hq * nq_pad * sizeof(float), kWsAlign);
 }
 
-template <int D>
+template <int D, bool VAR>
 cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tdo,
                        const BwdParams& p, cudaStream_t s) {
     const long long rows = static_cast<long long>(p.B) * p.Hq * p.nq_pad;
@@ -679,10 +794,10 @@ cudaError_t launch_bwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const dim3 g_kv((p.Nk + kBN - 1) / kBN, p.B * p.Hkv);
-    attn_bwd_kernel<D, true><<<g_kv, kBwdThreads, SmemBwd<D>::kAlloc, s>>>(tq, tk, tv, tdo, p);
+    attn_bwd_kernel<D, true, VAR><<<g_kv, kBwdThreads, SmemBwd<D>::kAlloc, s>>>(tq, tk, tv, tdo, p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const dim3 g_q((p.Nq + kBM - 1) / kBM, p.B * p.Hq);
-    attn_bwd_kernel<D, false><<<g_q, kBwdThreads, SmemBwd<D>::kAlloc, s>>>(tq, tk, tv, tdo, p);
+    attn_bwd_kernel<D, false, VAR><<<g_q, kBwdThreads, SmemBwd<D>::kAlloc, s>>>(tq, tk, tv, tdo, p);
     return cudaGetLastError();
 }
 
@@ -694,29 +809,56 @@ extern "C" attn_status_t attn_bwd_plan(int B, int Hq, int Nq, size_t* workspace_
     return ATTN_OK;
 }
 
-extern "C" attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
-                                  const void* dout, void* dq, void* dk, void* dv,
-                                  int B, int Hq, int Hkv, int Nq, int Nk, int d,
-                                  float scale, int is_causal, const int32_t* key_lens,
-                                  void* workspace, size_t workspace_bytes, void* stream) {
+extern "C" attn_status_t attn_bwd_ex(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                                     const void* dout, void* dq, void* dk, void* dv,
+                                     int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                                     float scale, int is_causal, const int32_t* key_lens,
+                                     const float* additive_mask, const int64_t* mask_strides,
+                                     const attn_score_mod_t* mod,
+                                     void* workspace, size_t workspace_bytes, void* stream) {
     if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || lse == nullptr || dout == nullptr ||
         dq == nullptr || dk == nullptr || dv == nullptr || workspace == nullptr)
         return ATTN_ERR_INVALID_ARG;
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nk <= 0 || d <= 0 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
     if (!(std::isfinite(scale)) || scale < 0.0f) return ATTN_ERR_INVALID_ARG;
+    if (key_lens != nullptr && additive_mask != nullptr) return ATTN_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) || !aligned16(dq) ||
         !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(lse) & 3u) ||
         (key_lens != nullptr && (reinterpret_cast<uintptr_t>(key_lens) & 3u)) ||
+        (additive_mask != nullptr && (reinterpret_cast<uintptr_t>(additive_mask) & 3u)) ||
         reinterpret_cast<uintptr_t>(workspace) % kWsAlign != 0)
         return ATTN_ERR_ALIGNMENT;
     if (workspace_bytes < bwd_bytes(B, Hq, Nq)) return ATTN_ERR_INVALID_ARG;
+    long long msb = 0, msh = 0, msq = 0;
+    if (additive_mask != nullptr) {
+        if (mask_strides != nullptr) {
+            msb = mask_strides[0];
+            msh = mask_strides[1];
+            msq = mask_strides[2];
+            if (msb < 0 || msh < 0 || msq < 0) return ATTN_ERR_INVALID_ARG;
+        } else {
+            msq = Nk;
+            msh = static_cast<long long>(Nq) * Nk;
+            msb = msh * Hq;
+        }
+    }
+    const bool use_mod = mod != nullptr && (mod->softcap != 0.0f || mod->mask2d_kind != ATTN_MASK2D_NONE);
+    if (mod != nullptr) {
+        if (!std::isfinite(mod->softcap) || mod->softcap < 0.0f) return ATTN_ERR_INVALID_ARG;
+        if (mod->mask2d_kind != ATTN_MASK2D_NONE && mod->mask2d_kind != ATTN_MASK2D_NEIGHBORHOOD &&
+            mod->mask2d_kind != ATTN_MASK2D_WINDOW)
+            return ATTN_ERR_INVALID_ARG;
+        if (mod->mask2d_kind != ATTN_MASK2D_NONE && (mod->grid_w <= 0 || mod->size <= 0 || mod->shift < 0))
+            return ATTN_ERR_INVALID_ARG;
+    }
+    if (use_mod && additive_mask != nullptr) return ATTN_ERR_UNSUPPORTED;  // as attn_fwd_mod
     int dev = 0;
     attn_status_t st = device_setup(&dev);
     if (st != ATTN_OK) return st;
 
     const float scale_eff = scale == 0.0f ? static_cast<float>(1.0 / std::sqrt(static_cast<double>(d))) : scale;
-    BwdParams p;
+    BwdParams p{};
     p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Nq = Nq; p.Nk = Nk; p.group = Hq / Hkv;
     p.nq_pad = (Nq + kBwdRowPad - 1) / kBwdRowPad * kBwdRowPad;
     p.scale_log2 = static_cast<float>(static_cast<double>(scale_eff) * 1.4426950408889634);
@@ -733,6 +875,28 @@ extern "C" attn_status_t attn_bwd(const void* q, const void* k, const void* v, c
     p.dv = static_cast<uint16_t*>(dv);
     p.timeout_ns = g_timeout_ns.load();
     p.epoch = next_epoch();
+    p.mask = additive_mask;
+    p.msb = msb; p.msh = msh; p.msq = msq;
+    p.softcap_on = 0;
+    p.m2_kind = 0;
+    p.m2_w = p.m2_size = 1;
+    p.m2_shift = 0;
+    if (use_mod) {
+        if (mod->softcap > 0.0f) {
+            p.softcap_on = 1;
+            p.sc_in = static_cast<float>(2.0 * scale_eff * 1.4426950408889634 / mod->softcap);
+            p.sc_out = static_cast<float>(static_cast<double>(mod->softcap) * 1.4426950408889634);
+        }
+        if (mod->mask2d_kind != ATTN_MASK2D_NONE) {
+            p.m2_kind = mod->mask2d_kind;
+            p.m2_w = mod->grid_w;
+            p.m2_size = mod->size;
+            p.m2_shift = mod->shift;
+        }
+    }
+    p.fd_w = make_fast_div(static_cast<uint32_t>(p.m2_w));
+    p.fd_size = make_fast_div(static_cast<uint32_t>(p.m2_size));
+    const bool var = use_mod || additive_mask != nullptr;
 
     CUtensorMap tq, tk, tv, tdo;
     if ((st = encode_map(&tq, q, d, Nq, static_cast<long long>(B) * Hq)) != ATTN_OK) return st;
@@ -740,9 +904,22 @@ extern "C" attn_status_t attn_bwd(const void* q, const void* k, const void* v, c
     if ((st = encode_map(&tv, v, d, Nk, static_cast<long long>(B) * Hkv)) != ATTN_OK) return st;
     if ((st = encode_map(&tdo, dout, d, Nq, static_cast<long long>(B) * Hq)) != ATTN_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const cudaError_t e = d == 128 ? launch_bwd<128>(tq, tk, tv, tdo, p, s) : launch_bwd<64>(tq, tk, tv, tdo, p, s);
+    cudaError_t e;
+    if (d == 128)
+        e = var ? launch_bwd<128, true>(tq, tk, tv, tdo, p, s) : launch_bwd<128, false>(tq, tk, tv, tdo, p, s);
+    else
+        e = var ? launch_bwd<64, true>(tq, tk, tv, tdo, p, s) : launch_bwd<64, false>(tq, tk, tv, tdo, p, s);
     if (e != cudaSuccess) return cuda_fail(e);
     return ATTN_OK;
+}
+
+extern "C" attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                                  const void* dout, void* dq, void* dk, void* dv,
+                                  int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                                  float scale, int is_causal, const int32_t* key_lens,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+    return attn_bwd_ex(q, k, v, out, lse, dout, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale, is_causal, key_lens,
+                       nullptr, nullptr, nullptr, workspace, workspace_bytes, stream);
 }
 
 // ------------------------------------------------------------------------
@@ -801,4 +978,32 @@ extern "C" attn_status_t attn_fwd_splitkv_noalloc(const void* q, const void* k, 
     return fwd_impl(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, scale, is_causal, key_lens, additive_mask,
                     mask_strides, true, n_splits, scratch, static_cast<size_t>(ATTN_NOALLOC_SCRATCH_BYTES), nullptr,
                     stream);
+}
+
+// ------------------------------------------------------------------------
+// FP8 block quantisation (the inputs of attn_fwd_fp8 from bf16 tensors).
+extern "C" attn_status_t attn_quantize_e4m3_blocks(const void* x, void* codes, float* scales, int heads, int N, int d,
+                                                   void* stream) {
+    if (x == nullptr || codes == nullptr || scales == nullptr || heads <= 0 || N <= 0 || d <= 0)
+        return ATTN_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+    if (!aligned16(x) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(scales) & 3u)) return ATTN_ERR_ALIGNMENT;
+    const long long nb = (static_cast<long long>(N) + kQuantRows - 1) / kQuantRows;
+    if (nb * heads > 0x7fffffffLL) return ATTN_ERR_INVALID_ARG;
+    int dev = 0;
+    attn_status_t st = device_setup(&dev);
+    if (st != ATTN_OK) return st;
+    const unsigned grid = static_cast<unsigned>(nb * heads);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (d == 128)
+        attn_quantize_e4m3_kernel<128><<<grid, kQuantThreads, 0, s>>>(static_cast<const uint16_t*>(x),
+                                                                      static_cast<uint8_t*>(codes), scales, N,
+                                                                      static_cast<int>(nb));
+    else
+        attn_quantize_e4m3_kernel<64><<<grid, kQuantThreads, 0, s>>>(static_cast<const uint16_t*>(x),
+                                                                     static_cast<uint8_t*>(codes), scales, N,
+                                                                     static_cast<int>(nb));
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e);
+    return ATTN_OK;
 }

@@ -20,6 +20,14 @@
 //                                blocks; S = Q K^T, dP = dO V^T, dS to TMEM, dQ += dS K
 // Splitting dQ from dK/dV keeps every accumulator in one CTA's TMEM: no atomics.
 //
+// Score and mask variants (the VAR instantiation), the forward's readings: the
+// score is s = c(x) + mask with x = scale q.k, c(x) = cap tanh(x / cap) under
+// soft-capping (else x), and keys outside a query's 2-D neighbourhood or window
+// are masked.  P = exp(s - LSE) uses the capped, masked score; the gradient
+// with respect to x is dS c'(x), c'(x) = 1 - tanh^2(x / cap), and dQ, dK follow
+// from x as above.  The additive mask has no gradient here.  Blocks that a 2-D
+// mask hides entirely are computed (their P is 0), not skipped.
+//
 // Warps (192 threads): 0-3 elementwise (thread = TMEM lane = row), 4 TMA producer,
 // 5 TMEM owner and MMA issuer (warp-uniform, elect.sync).  Every wait is bounded.
 #pragma once
@@ -45,7 +53,30 @@ struct BwdParams {
     uint16_t* dv;
     unsigned long long timeout_ns;
     unsigned int epoch;
+    // variants (VAR instantiation): additive mask with element strides (b, h, q),
+    // soft-capping (sc_in = 2 scale log2(e) / cap, sc_out = cap log2(e)), 2-D masks
+    const float* mask;
+    long long msb, msh, msq;
+    int softcap_on;
+    float sc_in, sc_out;
+    int m2_kind, m2_w, m2_size, m2_shift;
+    FastDiv fd_w, fd_size;
 };
+
+// Grid coordinates of token n under a 2-D mask, in the form the visibility test
+// compares: (row, column) for a neighbourhood, the (row, column) window index for
+// windows.
+__device__ __forceinline__ int2 bwd_coord(const BwdParams& p, int n) {
+    const int r = fdiv(n, p.fd_w);
+    const int c = n - r * p.m2_w;
+    if (p.m2_kind == 1) return make_int2(r, c);
+    return make_int2(fdiv(r + p.m2_shift, p.fd_size), fdiv(c + p.m2_shift, p.fd_size));
+}
+
+__device__ __forceinline__ bool bwd_visible_2d(const BwdParams& p, int2 a, int2 b) {
+    if (p.m2_kind == 1) return abs(a.x - b.x) < p.m2_size && abs(a.y - b.y) < p.m2_size;
+    return a.x == b.x && a.y == b.y;
+}
 
 constexpr int kBwdThreads = 192;
 enum : unsigned int { kRoleBwdElem = 4, kRoleBwdProducer = 5, kRoleBwdMma = 6, kRoleBwdPrep = 7 };
@@ -135,7 +166,7 @@ __device__ __forceinline__ void store_row_bf16(uint32_t taddr, uint16_t* dst, fl
 // tiles are keys, the fixed operands are K and V of one 128-key block, the
 // streamed stages hold Q and dO of one query block.  DKDV = false: rows are
 // queries, fixed Q and dO, streamed K and V.
-template <int D, bool DKDV>
+template <int D, bool DKDV, bool VAR>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -329,8 +360,16 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // through a double buffer (a buffer is rewritten two iterations later, after
         // every thread has passed the barrier of the iteration between)
         __shared__ float s_l2[2][kBM], s_dd[2][kBM];
+        // VAR with a 2-D mask: grid coordinates of this iteration's columns (queries
+        // or keys), double-buffered like LSE2 and D, and of this thread's own row
+        __shared__ int2 s_xy[2][kBM];
+        const bool m2 = VAR && p.m2_kind != 0;
+        int2 my_xy = make_int2(0, 0);
+        if (m2) my_xy = bwd_coord(p, DKDV ? key_row : q_row);
         bool ok = !*abort_flag;
-        for (int it = 0; ok && it < n_iter; ++it) {
+        // Every warp runs the named barrier of every iteration, also after a failed
+        // wait (it then skips the iteration's work), so that none is left waiting.
+        for (int it = 0; it < n_iter; ++it) {
             const int ib = iter_blk(it);
             // DKDV: LSE2 and D of this iteration's 128 queries (the same addresses in every
             // lane: broadcast loads; rows are padded to 128, so 16-byte aligned)
@@ -340,10 +379,25 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const long long r = static_cast<long long>(b * p.Hq + iter_head(it)) * p.nq_pad + ib * kBM;
                 s_l2[buf][row] = __ldg(p.lse2 + r + row);
                 s_dd[buf][row] = __ldg(p.delta + r + row);
+                if (m2) s_xy[buf][row] = bwd_coord(p, ib * kBM + row);
+                named_barrier_sync(1, kBM);
+            } else if (m2) {
+                s_xy[buf][row] = bwd_coord(p, ib * kBN + row);
                 named_barrier_sync(1, kBM);
             }
+            // VAR: the additive mask row of this thread (DKDV: column = query, row = key)
+            const float* mrow = nullptr;
+            if (VAR && p.mask != nullptr) {
+                if constexpr (DKDV)
+                    mrow = p.mask + static_cast<long long>(b) * p.msb + static_cast<long long>(iter_head(it)) * p.msh +
+                           static_cast<long long>(ib) * kBM * p.msq + key_row;
+                else
+                    mrow = p.mask + static_cast<long long>(b) * p.msb + static_cast<long long>(h0) * p.msh +
+                           static_cast<long long>(q_row) * p.msq + static_cast<long long>(ib) * kBN;
+            }
+            if (!ok) continue;
             const bool got = mbar_wait(bar(L::STFULL_), it & 1, limit, abort_flag, p.epoch, kRoleBwdElem, 2);
-            if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, got)) { ok = false; continue; }
             tc_fence_after();
             #pragma unroll
             for (int c = 0; c < 4; ++c) {
@@ -371,9 +425,29 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                             dd = my_d;
                             vis = kj < kv_len && (!p.is_causal || kj <= q_row);
                         }
-                        const float pv = vis ? ex2_approx(fmaf(__uint_as_float(sv[e + u]), c2, -l2)) : 0.0f;
-                        pp[u] = pv;
-                        ds[u] = pv * (__uint_as_float(dv[e + u]) - dd);
+                        if constexpr (!VAR) {
+                            const float pv = vis ? ex2_approx(fmaf(__uint_as_float(sv[e + u]), c2, -l2)) : 0.0f;
+                            pp[u] = pv;
+                            ds[u] = pv * (__uint_as_float(dv[e + u]) - dd);
+                        } else {
+                            // base-2 logit of the capped, masked score, and c'(x)
+                            const float raw = __uint_as_float(sv[e + u]);
+                            float lg = raw * c2, g = 1.0f;
+                            if (p.softcap_on) {
+                                const float t = fmaf(rcp_approx(1.0f + ex2_approx(raw * p.sc_in)), -2.0f, 1.0f);
+                                lg = p.sc_out * t;
+                                g = fmaf(-t, t, 1.0f);
+                            }
+                            if (m2) vis = vis && bwd_visible_2d(p, my_xy, s_xy[buf][col]);
+                            // (padding query rows past Nq have no mask row: not read)
+                            if (mrow != nullptr && vis && (DKDV ? ib * kBM + col < p.Nq : q_row < p.Nq)) {
+                                const long long off = DKDV ? static_cast<long long>(col) * p.msq : col;
+                                lg = fmaf(__ldg(mrow + off), kLog2e, lg);
+                            }
+                            const float pv = vis ? ex2_approx(lg - l2) : 0.0f;
+                            pp[u] = pv;
+                            ds[u] = pv * (__uint_as_float(dv[e + u]) - dd) * g;
+                        }
                     }
                     pw[e / 2] = pack_bf16x2(pp[0], pp[1]);
                     dw[e / 2] = pack_bf16x2(ds[0], ds[1]);

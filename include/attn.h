@@ -271,6 +271,27 @@ attn_status_t attn_fwd_fp8(const void *q8, const void *k8, const void *v8,
                            float scale, int is_causal, const int32_t *key_lens, void *stream);
 
 /*
+ * attn_quantize_e4m3_blocks -- the FP8 inputs of attn_fwd_fp8 from a bf16
+ * tensor, on the device: block quantisation with one fp32 scale factor per
+ * 128-row block of every head ("FlashAttention technical analysis",
+ * jsqmd.com/news/722897, section 4.2: FP8 with block quantisation; section
+ * 6.3: each block keeps its own scale factor).  For each block, in fp32:
+ *   amax = max |x| over its rows (fewer than 128 in a head's last block),
+ *   scale = amax / 448 (1 when amax = 0), the largest finite E4M3 value 448,
+ *   code = E4M3 of min(max(x / scale, -448), 448),
+ * the division and the E4M3 conversion both rounding to nearest even.
+ *   x       device bf16 [heads, N, d], 16-byte aligned (heads = B * H)
+ *   codes   device uint8 [heads, N, d], 16-byte aligned (written)
+ *   scales  device fp32 [heads, ceil(N / 128)], 4-byte aligned (written)
+ * x must be finite.  d in {64, 128} (attn_fwd_fp8 takes d = 128).  One kernel
+ * on `stream`, reading x once.
+ * Errors: ATTN_ERR_INVALID_ARG (NULL pointer, non-positive size, more than
+ * 2^31 - 1 blocks), ATTN_ERR_UNSUPPORTED (d), ATTN_ERR_ALIGNMENT, ATTN_ERR_CUDA.
+ */
+attn_status_t attn_quantize_e4m3_blocks(const void *x, void *codes, float *scales, int heads, int N, int d,
+                                        void *stream);
+
+/*
  * attn_bwd_plan -- device workspace bytes attn_bwd needs (host-only).  The
  * workspace holds two fp32 values per query row (D = rowsum(dO * O) and the
  * base-2 LSE), rows padded to a multiple of 128 per head.
@@ -293,8 +314,8 @@ attn_status_t attn_bwd_plan(int B, int Hq, int Nq, size_t *workspace_bytes);
  *   q, out, dout, dq   bf16 [B, Hq, Nq, d]     (dq written)
  *   k, v, dk, dv       bf16 [B, Hkv, Nk, d]    (dk, dv written)
  *   lse                fp32 [B, Hq, Nq], as written by attn_fwd for the same inputs
- * scale, is_causal, key_lens: as attn_fwd (additive masks are not supported
- * here).  Rows of dq with no visible key and keys no query sees get 0.
+ * scale, is_causal, key_lens: as attn_fwd (additive masks and the score
+ * variants: attn_bwd_ex).  Rows of dq with no visible key and keys no query sees get 0.
  * workspace: device, 256-byte aligned, >= attn_bwd_plan bytes; scratch whose
  * contents need not be initialised; calls in flight at once must not share it.
  * Three kernels run on `stream` (row statistics, dK/dV, dQ).
@@ -305,6 +326,31 @@ attn_status_t attn_bwd(const void *q, const void *k, const void *v, const void *
                        int B, int Hq, int Hkv, int Nq, int Nk, int d,
                        float scale, int is_causal, const int32_t *key_lens,
                        void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * attn_bwd_ex -- attn_bwd for the forward's score and mask variants: the
+ * gradients of attn_fwd with an additive mask, or of attn_fwd_mod with
+ * soft-capping and / or a 2-D neighbourhood or window mask (`out` and `lse`
+ * must come from that forward call with the same options).  With the score
+ * s = c(x) + mask, x = scale * q.k, c(x) = softcap * tanh(x / softcap) (else
+ * c(x) = x): P = exp(s - LSE), dS = P o (dP - D) as in attn_bwd, and the
+ * gradient with respect to x is dS * c'(x), c'(x) = 1 - tanh^2(x / softcap),
+ * from which dQ = scale dX K and dK = scale dX^T Q; keys a 2-D mask hides get
+ * P = 0 (their blocks are computed, not skipped).  The additive mask gets no
+ * gradient.  With all variants off it computes exactly what attn_bwd computes.
+ *   additive_mask, mask_strides: as attn_fwd (fp32 device, NULL = none);
+ *   mod: host pointer or NULL, as attn_fwd_mod.
+ * An additive mask does not combine with key_lens or with `mod`
+ * (ATTN_ERR_INVALID_ARG / ATTN_ERR_UNSUPPORTED, as in the forward).
+ * Errors: as attn_bwd, plus those of attn_fwd_mod's `mod` checks.
+ */
+attn_status_t attn_bwd_ex(const void *q, const void *k, const void *v, const void *out, const float *lse,
+                          const void *dout, void *dq, void *dk, void *dv,
+                          int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                          float scale, int is_causal, const int32_t *key_lens,
+                          const float *additive_mask, const int64_t *mask_strides,
+                          const attn_score_mod_t *mod,
+                          void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * attn_check_device_status -- synchronise `stream`, then read and clear the

@@ -88,3 +88,64 @@ def test_bwd_deterministic():
     a = run_bwd(q, k, v, do, is_causal=True)
     b = run_bwd(q, k, v, do, is_causal=True)
     assert all(torch.equal(x, y) for x, y in zip(a, b))
+
+
+# ----------------------------------------------- score and mask variants
+def check_variant(B, Hq, Hkv, Nq, Nk, d, seed, causal=False, mask=None, softcap=0.0, mask2d=None):
+    """attn_bwd_ex against the backward oracle with the same variant; the GPU
+    forward (attn_fwd with the mask, or attn_fwd_mod) provides O and LSE."""
+    q, k, v = make_qkv(B, Hq, Hkv, Nq, Nk, d, seed=seed)
+    do, _, _ = make_qkv(B, Hq, Hkv, Nq, Nk, d, seed=seed + 1)
+    kw = dict(is_causal=causal, softcap=softcap, mask2d=mask2d)
+    if mask is not None:
+        kw["attn_mask"] = mask
+    dq, dk, dv = run_bwd(q, k, v, do, **kw)
+    rq, rk, rv = oracle.attention_bwd(q, k, v, do, is_causal=causal, softcap=softcap, mask2d=mask2d,
+                                      mask=None if mask is None else mask.double().numpy())
+    assert_grad_close("dq", dq, rq)
+    assert_grad_close("dk", dk, rk)
+    assert_grad_close("dv", dv, rv)
+    return dq, dk, dv
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_softcap(d, causal):
+    """A cap of 1 on scores of standard deviation 1: tanh bends most of them."""
+    check_variant(2, 4, 2, 300, 260, d, seed=41 + d + causal, causal=causal, softcap=1.0)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_bwd_additive_mask(d):
+    g = torch.Generator().manual_seed(7)
+    mask = torch.randn(2, 2, 200, 260, generator=g) * 2.0
+    mask[0, 1, :, 100:] = -float("inf")   # padding-like stripe
+    mask[1, 0, 7, :] = -float("inf")      # a query row with no key
+    dq, dk, dv = check_variant(2, 2, 2, 200, 260, d, seed=51 + d, mask=mask)
+    assert torch.all(dq[1, 0, 7] == 0)
+
+
+def test_bwd_additive_mask_broadcast_causal():
+    g = torch.Generator().manual_seed(8)
+    mask = torch.randn(1, 1, 257, 257, generator=g)
+    check_variant(2, 4, 4, 257, 257, 128, seed=61, causal=True, mask=mask)
+
+
+@pytest.mark.parametrize("mask2d", [("neighborhood", 20, 3), ("window", 16, 4), ("window", 16, 4, 2)])
+@pytest.mark.parametrize("d", [64, 128])
+def test_bwd_mask2d(mask2d, d):
+    check_variant(2, 2, 1, 400, 400, d, seed=71 + d, mask2d=mask2d)
+
+
+def test_bwd_neighbourhood_softcap_causal():
+    """The 56-wide grid of the ViT workload, radius 5, with the cap of 30."""
+    check_variant(1, 2, 2, 56 * 6, 56 * 6, 64, seed=81, causal=True, softcap=30.0, mask2d=("neighborhood", 56, 5))
+
+
+def test_bwd_variants_off_equal_plain():
+    """attn_bwd_ex with every variant off and attn_bwd give the same bits."""
+    q, k, v = make_qkv(1, 2, 2, 300, 300, 64, seed=91)
+    do, _, _ = make_qkv(1, 2, 2, 300, 300, 64, seed=92)
+    a = run_bwd(q, k, v, do)
+    b = run_bwd(q, k, v, do, softcap=0.0, mask2d=None)
+    assert all(torch.equal(x, y) for x, y in zip(a, b))
