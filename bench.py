@@ -42,15 +42,19 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 _CSRC = "exact_attention_157_b200/csrc/"
 _COMMON = [_CSRC + "fwd_common.cuh", _CSRC + "sm100_ptx.cuh"]
 KERNEL_SOURCES = {"tile": [_CSRC + "fwd_kernel_pp.cuh"] + _COMMON,
+                  "short": [_CSRC + "short_kernel.cuh"] + _COMMON,
                   "decode": [_CSRC + "decode_kernel.cuh"] + _COMMON,
                   "bwd": [_CSRC + "bwd_kernels.cuh"] + _COMMON}
 
 
 def kernel_family(w) -> str:
+    """Which kernel a workload's forward runs on (the dispatch of attn_api.cu)."""
     if w.backward:
         return "bwd"
     if w.split_kv and w.Hq // w.Hkv * w.Nq <= 16 and not w.is_causal:
         return "decode"
+    if w.d == 64 and w.Nk <= 256 and not w.fp8 and not w.softcap and w.mask2d is None and not w.split_kv:
+        return "short"
     return "tile"
 
 

@@ -514,13 +514,18 @@ class HostAttention:
         self.key_lens = torch.empty((B,), dtype=torch.int32, device=dev) if with_key_lens else None
         self.split_kv = split_kv
         self.workspace = None
-        if split_kv is not None:
-            st, _, nbytes = attn_splitkv_plan(B, Hq, Nq, Nk, d, int(split_kv), 0, Hkv=Hkv, is_causal=is_causal)
-            if st != ATTN_OK:
-                raise AttnError(st, "attn_splitkv_plan")
-            self.workspace = torch.empty((max(nbytes, 1),), dtype=torch.uint8, device=dev)
         n = min(B, 8) if chunks is None else max(1, min(int(chunks), B))
         self.bounds = [(B * i // n, B * (i + 1) // n) for i in range(n)]
+        if split_kv is not None:
+            # each chunk is planned for its own batch size (a smaller batch may take
+            # more key ranges): the workspace holds the largest of those plans
+            nbytes = 0
+            for cb in sorted({b1 - b0 for b0, b1 in self.bounds}):
+                st, _, nb = attn_splitkv_plan(cb, Hq, Nq, Nk, d, int(split_kv), 0, Hkv=Hkv, is_causal=is_causal)
+                if st != ATTN_OK:
+                    raise AttnError(st, "attn_splitkv_plan")
+                nbytes = max(nbytes, nb)
+            self.workspace = torch.empty((max(nbytes, 1),), dtype=torch.uint8, device=dev)
         self.h2d = torch.cuda.Stream(dev)
         self.d2h = torch.cuda.Stream(dev)
         self.ev_in = [torch.cuda.Event() for _ in self.bounds]

@@ -129,8 +129,9 @@ struct SmemBwd {
     static constexpr int kStages = 2 * kTile;
     static constexpr int kBars = kStages + 2 * kStage;
     // barriers
-    static constexpr int FIXFULL = 0, STFULL_ = 1, PFULL = 2, DONE = 3, RFULL = 4, REMPTY = 6;
-    static constexpr int kNumBars = 8;
+    // PFULL: the first 64 columns of P / dS stored; PFULL1: the last 64
+    static constexpr int FIXFULL = 0, STFULL_ = 1, PFULL = 2, DONE = 3, RFULL = 4, REMPTY = 6, PFULL1 = 8;
+    static constexpr int kNumBars = 9;
     static constexpr int kMisc = kBars + 8 * kNumBars;
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;
@@ -224,6 +225,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mbar_init(bar(L::FIXFULL), 1);
         mbar_init(bar(L::STFULL_), 1);
         mbar_init(bar(L::PFULL), 128);
+        mbar_init(bar(L::PFULL1), 128);
         mbar_init(bar(L::DONE), 1);
         for (int s = 0; s < 2; ++s) {
             mbar_init(bar(L::RFULL + s), 1);
@@ -319,24 +321,32 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                             kIdescS, kk > 0 ? 1u : 0u);
             }
             mma_commit_warp(bar(L::STFULL_));
-            if (!mbar_wait_warp(bar(L::PFULL), it & 1, limit, abort_flag, p.epoch, kRoleBwdMma, 3)) { ok = false; break; }
-            tc_fence_after();
             // bf16 operands in TMEM (A) times a streamed tile as B (MN-major, 16 rows per step):
             // DKDV: dV += P^T dO (P^T in kColA), dK += dS^T Q (dS^T in kColB).
             // dQ:   dQ += dS K (dS in kColA).
-            #pragma unroll
-            for (int kk = 0; kk < kBN / 16; ++kk) {
-                const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
-                if constexpr (DKDV) {
-                    mma_ts_warp(tmem + L::kColAcc0, tmem + L::kColA + kk * 8,
-                                smem_desc_sw128(st1 + kk * 2048, L::kChunkBytes, 1024), kIdescAcc, acc);
-                    mma_ts_warp(tmem + L::kColAcc1, tmem + L::kColB + kk * 8,
-                                smem_desc_sw128(st0 + kk * 2048, L::kChunkBytes, 1024), kIdescAcc, acc);
-                } else {
-                    mma_ts_warp(tmem + L::kColAcc0, tmem + L::kColA + kk * 8,
-                                smem_desc_sw128(st0 + kk * 2048, L::kChunkBytes, 1024), kIdescAcc, acc);
+            // The first 64 columns (steps 0-3) start as soon as the elementwise warps have
+            // stored them (PFULL), while the last 64 are computed (PFULL1).
+            for (int half = 0; half < 2 && ok; ++half) {
+                if (!mbar_wait_warp(bar(half == 0 ? L::PFULL : L::PFULL1), it & 1, limit, abort_flag, p.epoch,
+                                    kRoleBwdMma, 3 + 4 * half))
+                    { ok = false; break; }
+                tc_fence_after();
+                #pragma unroll
+                for (int k4 = 0; k4 < kBN / 32; ++k4) {
+                    const int kk = half * (kBN / 32) + k4;
+                    const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
+                    if constexpr (DKDV) {
+                        mma_ts_warp(tmem + L::kColAcc0, tmem + L::kColA + kk * 8,
+                                    smem_desc_sw128(st1 + kk * 2048, L::kChunkBytes, 1024), kIdescAcc, acc);
+                        mma_ts_warp(tmem + L::kColAcc1, tmem + L::kColB + kk * 8,
+                                    smem_desc_sw128(st0 + kk * 2048, L::kChunkBytes, 1024), kIdescAcc, acc);
+                    } else {
+                        mma_ts_warp(tmem + L::kColAcc0, tmem + L::kColA + kk * 8,
+                                    smem_desc_sw128(st0 + kk * 2048, L::kChunkBytes, 1024), kIdescAcc, acc);
+                    }
                 }
             }
+            if (!ok) break;
             mma_commit_warp(bar(L::REMPTY + s));  // the stage may be refilled once these complete
         }
         mma_commit_warp(bar(L::DONE));
@@ -458,10 +468,13 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 } else {
                     tmem_st16(lane_tmem + L::kColA + c * 16, dw);  // dS over S columns already read
                 }
+                if (c == 1 || c == 3) {
+                    // columns 0-63 (then 64-127) stored: their products may start
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(bar(c == 1 ? L::PFULL : L::PFULL1));
+                }
             }
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(bar(L::PFULL));
         }
         // ------------------------------------------------------------- epilogue
         bool have = n_iter > 0 && ok;

@@ -443,21 +443,28 @@ attn_fwd_short_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                             #pragma unroll
                             for (int c = 0; c < 64; ++c) sc[c] = (j0 + c < lim) ? sc[c] : -INFINITY;
                         }
+                        // four independent chains of 3-input maxima (a shorter dependency chain)
                         float x0 = fmax3(sc[0], sc[1], sc[2]), x1 = fmax3(sc[3], sc[4], sc[5]);
+                        float x2 = fmax3(sc[6], sc[7], sc[8]), x3 = fmax3(sc[9], sc[10], sc[11]);
                         #pragma unroll
-                        for (int c = 6; c < 30; c += 4) {
+                        for (int c = 12; c < 28; c += 8) {
                             x0 = fmax3(x0, sc[c], sc[c + 1]);
                             x1 = fmax3(x1, sc[c + 2], sc[c + 3]);
+                            x2 = fmax3(x2, sc[c + 4], sc[c + 5]);
+                            x3 = fmax3(x3, sc[c + 6], sc[c + 7]);
                         }
-                        x0 = fmax3(x0, sc[30], sc[31]);
+                        x0 = fmax3(x0, sc[28], sc[29]);
+                        x1 = fmax3(x1, sc[30], sc[31]);
                         if (two) {
                             #pragma unroll
-                            for (int c = 32; c < 64; c += 4) {
+                            for (int c = 32; c < 64; c += 8) {
                                 x0 = fmax3(x0, sc[c], sc[c + 1]);
                                 x1 = fmax3(x1, sc[c + 2], sc[c + 3]);
+                                x2 = fmax3(x2, sc[c + 4], sc[c + 5]);
+                                x3 = fmax3(x3, sc[c + 6], sc[c + 7]);
                             }
                         }
-                        const float cmax = fmaxf(x0, x1) * c_log2;
+                        const float cmax = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3)) * c_log2;
                         if (g == 0) {
                             m = cmax == -INFINITY ? 0.0f : cmax;
                         } else if (__any_sync(0xffffffffu, cmax > m + kLazyTau)) {

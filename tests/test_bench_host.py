@@ -12,7 +12,8 @@ from workloads import WORKLOADS
 
 
 @pytest.mark.parametrize("name,family", [
-    ("long", "tile"), ("vit", "tile"), ("long_fp8", "tile"), ("vit3136_neighborhood", "tile"),
+    ("long", "tile"), ("vit", "short"), ("unet_cross", "short"), ("tiny", "short"), ("unet_self", "tile"),
+    ("long_fp8", "tile"), ("vit3136_neighborhood", "tile"),
     ("decode_gqa", "decode"), ("decode_gqa_small", "decode"),
     ("long_bwd", "bwd"), ("prefill_gqa_bwd", "bwd"),
 ])
@@ -57,8 +58,8 @@ def test_committed_traffic_records_are_well_formed():
 
 
 def test_kernel_source_hash_depends_on_family_sources():
-    hashes = {f: bench.kernel_source_hash(f) for f in ("tile", "decode", "bwd")}
-    assert len(set(hashes.values())) == 3 and all(len(h) == 16 for h in hashes.values())
+    hashes = {f: bench.kernel_source_hash(f) for f in ("tile", "short", "decode", "bwd")}
+    assert len(set(hashes.values())) == 4 and all(len(h) == 16 for h in hashes.values())
 
 
 def test_flops_dense_causal_backward_and_fp8():

@@ -45,3 +45,21 @@ def test_short_keys_and_split_kv():
         torch.cuda.current_stream().synchronize()
         ea.check_device_status()
         assert torch.equal(oh, ref_o.cpu()) and torch.equal(lseh, ref_l.cpu())
+
+
+def test_automatic_split_kv_chunks_plan_their_own_ranges():
+    """split_kv=0 (automatic) on a decoding shape: a chunk of one batch entry
+    takes more key ranges than the whole batch, so the workspace must hold the
+    largest chunk plan; the result equals the device call within the parity
+    tolerances (the ranges, and so the merge order, differ)."""
+    B, Hq, Hkv, Nq, Nk, d = 8, 32, 8, 1, 16384, 128
+    q, k, v = make_qkv(B, Hq, Hkv, Nq, Nk, d, seed=5)
+    ref_o, ref_l = ea.attention(q.to(DEV), k.to(DEV), v.to(DEV), split_kv=0)
+    runner = ea.HostAttention(B, Hq, Hkv, Nq, Nk, d, device=DEV, split_kv=0)
+    oh = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+    lseh = torch.empty((B, Hq, Nq), dtype=torch.float32).pin_memory()
+    runner(q.pin_memory(), k.pin_memory(), v.pin_memory(), oh, lseh)
+    torch.cuda.current_stream().synchronize()
+    ea.check_device_status()
+    assert (oh.float() - ref_o.cpu().float()).abs().max().item() <= 1e-2
+    assert (lseh - ref_l.cpu()).abs().max().item() <= 1e-3
