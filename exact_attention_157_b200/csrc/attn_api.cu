@@ -470,6 +470,10 @@ attn_status_t fwd_impl(const void* q, const void* k, const void* v, void* out, f
             p.softcap_on = 1;
             p.sc_in = static_cast<float>(2.0 * scale_eff * 1.4426950408889634 / mod->softcap);
             p.sc_out = static_cast<float>(static_cast<double>(mod->softcap) * 1.4426950408889634);
+            p.sc_a = static_cast<float>(static_cast<double>(scale_eff) / mod->softcap);
+            p.sc_lim = static_cast<float>(kTanhPolyRange * static_cast<double>(mod->softcap) / scale_eff);
+            for (int i = 0; i < kTanhPolyTerms; ++i)
+                p.sc_poly[i] = static_cast<float>(scale_eff * 1.4426950408889634 * kTanhPoly[i]);
             p.scale_log2 = 1.0f;
         }
         p.m2_kind = mod->mask2d_kind;

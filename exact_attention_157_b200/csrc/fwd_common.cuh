@@ -11,6 +11,16 @@ constexpr int kBM = 128;          // query rows per tile (= TMEM lanes)
 constexpr int kBN = 128;          // keys per block
 constexpr int kTmemCols = 512;
 constexpr float kLazyTau = 8.0f;  // rescale only when the max grows by > 2^8
+
+// tanh(t) = t * P(t^2) for |t| <= kTanhPolyRange: P of degree 5 in t^2, fitted by
+// weighted least squares on 4000 Chebyshev nodes of [0, kTanhPolyRange^2], the
+// weights driven towards least maximum relative error (2.9e-8 for the fit; 1.6e-7
+// with float32 coefficients and Horner evaluation, against tanh in fp64).  The
+// soft-capped score cap * tanh(scale * x / cap) then costs FMA-pipe work only.
+constexpr int kTanhPolyTerms = 6;
+constexpr float kTanhPolyRange = 0.75f;
+constexpr float kTanhPoly[kTanhPolyTerms] = {1.000000000e+00f, -3.333295882e-01f, 1.332540661e-01f,
+                                             -5.334442854e-02f, 1.958290674e-02f, -4.716256633e-03f};
 // FP8 probabilities: a tighter threshold (stale-max factor at most 2^2) frees six
 // binades of the E4M3 range, used to store P * 2^6; the largest stored value is
 // then 2^8 <= 448 and normal E4M3 values reach down to 2^-12 of the row max.
@@ -69,6 +79,9 @@ struct FwdParams {
     int softcap_on;
     float sc_in;   // 2 * scale * log2(e) / cap: base-2 exponent of e^(2x / cap) per raw score
     float sc_out;  // cap * log2(e)
+    float sc_a;    // scale / cap: the argument of tanh per raw score
+    float sc_lim;  // kTanhPolyRange / sc_a: raw scores up to this magnitude take the polynomial
+    float sc_poly[kTanhPolyTerms];  // scale * log2(e) * the polynomial's coefficients
     int m2_kind, m2_w, m2_size, m2_shift;
     // FP8 instantiation: per-128-row block scales of Q [B*Hq][nqb] and K, V [B*Hkv][nkb]
     const float* q_scale;

@@ -658,10 +658,41 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 if (p.is_causal && q_idx - j0 + 1 < lim) lim = q_idx - j0 + 1;
                 if constexpr (MOD) {
                     if (p.softcap_on) {
-                        // base-2 logit cap * log2(e) * tanh(x / cap), with tanh(u) = 1 - 2 / (1 + e^(2u))
+                        // base-2 logit cap * log2(e) * tanh(x / cap).  When every raw score
+                        // of the warp's block has |scale * s / cap| <= kTanhPolyRange, tanh is
+                        // the odd polynomial (FMA pipe only); otherwise tanh(u) =
+                        // 1 - 2 / (1 + e^(2u)) on the special-function unit.
+                        float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
                         #pragma unroll
-                        for (int c = 0; c < kBN; ++c)
-                            s[c] = fmaf(rcp_approx(1.0f + ex2_approx(s[c] * p.sc_in)), -2.0f * p.sc_out, p.sc_out);
+                        for (int c = 0; c < kBN; c += 8) {
+                            a0 = fmax3(a0, fabsf(s[c]), fabsf(s[c + 1]));
+                            a1 = fmax3(a1, fabsf(s[c + 2]), fabsf(s[c + 3]));
+                            a2 = fmax3(a2, fabsf(s[c + 4]), fabsf(s[c + 5]));
+                            a3 = fmax3(a3, fabsf(s[c + 6]), fabsf(s[c + 7]));
+                        }
+                        const bool in_range = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3)) <= p.sc_lim;
+                        if (__all_sync(0xffffffffu, in_range)) {
+                            const uint64_t ca = pack_f32x2(p.sc_a, p.sc_a);
+                            #pragma unroll
+                            for (int c = 0; c < kBN / 2; ++c) {
+                                const uint64_t sv = pack_f32x2(s[2 * c], s[2 * c + 1]);
+                                const uint64_t t = ffma2(sv, ca, 0ull);
+                                const uint64_t w = ffma2(t, t, 0ull);
+                                uint64_t h = ffma2(w, pack_f32x2(p.sc_poly[5], p.sc_poly[5]),
+                                                   pack_f32x2(p.sc_poly[4], p.sc_poly[4]));
+                                h = ffma2(w, h, pack_f32x2(p.sc_poly[3], p.sc_poly[3]));
+                                h = ffma2(w, h, pack_f32x2(p.sc_poly[2], p.sc_poly[2]));
+                                h = ffma2(w, h, pack_f32x2(p.sc_poly[1], p.sc_poly[1]));
+                                h = ffma2(w, h, pack_f32x2(p.sc_poly[0], p.sc_poly[0]));
+                                const uint64_t r = ffma2(sv, h, 0ull);
+                                s[2 * c] = lo_f32(r);
+                                s[2 * c + 1] = hi_f32(r);
+                            }
+                        } else {
+                            #pragma unroll
+                            for (int c = 0; c < kBN; ++c)
+                                s[c] = fmaf(rcp_approx(1.0f + ex2_approx(s[c] * p.sc_in)), -2.0f * p.sc_out, p.sc_out);
+                        }
                     }
                     if (p.m2_kind != 0) {
                         // keys of this block inside the row's grid rectangle, as a 128-bit set:

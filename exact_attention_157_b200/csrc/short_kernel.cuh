@@ -5,8 +5,7 @@
 // With at most 256 keys a whole score row fits in one tensor-memory
 // accumulator, so the softmax needs no running rescale: S = Q K^T is computed
 // in one product (N = the tile's key count rounded up to 16), the softmax reads
-// the row twice from tensor memory (maximum, then exponentials), and P V is one
-// product.  This is the three steps of the definition per 128-row tile ("Flash
+// the row once from tensor memory, 64 keys per step, and P V is one product.  This is the three steps of the definition per 128-row tile ("Flash
 // Attention in a production Stable-Diffusion service", xxmr.cn/news/81028,
 // section 2.3), tiled over queries as "FlashAttention technical analysis"
 // (jsqmd.com/news/722897) section 2.2 tiles Q; the key block is the whole
@@ -25,7 +24,6 @@
 //               is stored, for the even tiles
 //   warp 10     MMA issuer of slot 1 (odd tiles)
 //   warp 11     idle (completes the third warpgroup)
-//   warps 10-11 idle (complete the third warpgroup)
 //
 // Tensor memory, slot s = columns [256 s, 256 s + 256): S in [0, N), P (bf16
 // pairs) in [0, N / 2) written over the scores already read, O (64 fp32
@@ -35,7 +33,9 @@
 //
 // Each slot's MMA warp issues S(n), PV(n), S(n + 2), PV(n + 2), ... for its
 // tiles: S(n + 2) once the epilogue of tile n has read O out of the slot
-// (OEMPTY).  Commits release the Q stage (after S) and, with one arrival from
+// (OEMPTY).  With kShortEarlyS, an S whose columns stay below O (N <= 128) is
+// issued right after PV(n) and only PV(n + 2) waits for that read; on B200 this
+// measured slower (unet_cross 15.4 against 14.9 us), so it is off.  Commits release the Q stage (after S) and, with one arrival from
 // each MMA warp, the K/V buffer (after the warp's last P V of the run; a warp
 // with no tile in a run arrives once the run's K/V have landed, so that its
 // arrival counts towards that use of the buffer).
@@ -55,6 +55,9 @@ namespace attn_sm100 {
 constexpr int kShortThreads = 384;
 constexpr bool kShortTurns = true;        // softmax warpgroups take turns (token)
 constexpr bool kShortDirectStore = true;  // O rows stored from registers (else staged, TMA store)
+constexpr bool kShortWarpStaged = true;   // direct stores: rows regrouped per warp through shared memory
+constexpr bool kShortEarlyS = false;      // S(n + 2) before the epilogue of n when it fits below O (measured slower)
+constexpr uint32_t kShortOCol = 128;      // first tensor-memory column of O within a slot
 constexpr int kShortMaxKeys = 256;
 constexpr int kShortMaxQ = 8;          // Q stages at most
 constexpr int kShortTile = 128 * 128;  // one 128-row tile of 64 bf16 columns (16 KB)
@@ -345,20 +348,27 @@ attn_fwd_short_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         bool ok = true;
         Ent cur = next_own();
         if (cur.valid) ok = release_idle_runs(cur.run) && issue_s(cur);
+        bool o_held = false;  // O of this slot's previous tile not yet read out by its epilogue
         for (int i = 0; ok && cur.valid; ++i) {
+            const Ent nxt = next_own();  // off the path from P to P V
             if (!mbar_wait_warp(bar(L::PFULL + w), i & 1, limit, abort_flag, p.epoch, kRoleMma, 48))
                 { ok = false; break; }
+            // P V overwrites O: the previous tile's epilogue must have read it
+            if (o_held && !mbar_wait_warp(bar(L::OEMPTY + w), (i - 1) & 1, limit, abort_flag, p.epoch, kRoleMma, 49))
+                { ok = false; break; }
             tc_fence_after();
-            const Ent nxt = next_own();
             const bool last_of_run = !nxt.valid || nxt.run != cur.run;
-            short_issue_pv(tmem + 256u * w + 128u, tmem + 256u * w,
+            short_issue_pv(tmem + 256u * w + kShortOCol, tmem + 256u * w,
                            sbase + ((cur.run & 1) ? lay.kv1 : lay.kv0) + p.kv_bytes, cur.x.ncols, bar(L::OFULL + w),
                            last_of_run ? bar(L::KVEMPTY + (cur.run & 1)) : 0u);
             if (last_of_run) to_release = cur.run + 1;
             if (!nxt.valid) break;
             if (!release_idle_runs(nxt.run)) { ok = false; break; }
-            // the slot is free once the epilogue of this tile has read O out of it
-            if (!mbar_wait_warp(bar(L::OEMPTY + w), i & 1, limit, abort_flag, p.epoch, kRoleMma, 49))
+            // S(n + 2) goes into the slot at once when its columns stay clear of O
+            // (products of one thread run in order, so P V has read P before S
+            // overwrites it); a longer S waits until the epilogue has read O out
+            o_held = kShortEarlyS && nxt.x.ncols <= static_cast<int>(kShortOCol);
+            if (!o_held && !mbar_wait_warp(bar(L::OEMPTY + w), i & 1, limit, abort_flag, p.epoch, kRoleMma, 49))
                 { ok = false; break; }
             if (!issue_s(nxt)) { ok = false; break; }
             cur = nxt;
@@ -529,18 +539,47 @@ attn_fwd_short_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             ok = tile_ok;
             const float inv_l = l_sum > 0.0f ? 1.0f / l_sum : 0.0f;
             if constexpr (kShortDirectStore) {
-                // each thread writes its own 128-byte row of O from registers
                 if (tile_ok) {
                     tc_fence_after();
                     uint32_t o[64];
-                    tmem_ld32(lane_tmem + 128, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
-                    tmem_ld32(lane_tmem + 160, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
+                    tmem_ld32(lane_tmem + kShortOCol, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
+                    tmem_ld32(lane_tmem + kShortOCol + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
                     tmem_wait_ld();
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(bar(L::OEMPTY + s));  // the MMA warp may put the next S here
-                    if (q < p.Nq && !*abort_flag) {
-                        const long long r = static_cast<long long>(x.bh) * p.Nq + q;
+                    if (lane == 0) mbar_arrive(bar(L::OEMPTY + s));  // O may be overwritten now
+                    const long long r = static_cast<long long>(x.bh) * p.Nq + q;
+                    if constexpr (kShortWarpStaged) {
+                        // the warp's 32 rows (4 KB) pass through shared memory (16-byte
+                        // units swizzled by row, no bank conflicts), then each store
+                        // instruction writes four whole consecutive rows (512 bytes)
+                        uint8_t* ws = stage + (warp & 3) * 4096;
+                        #pragma unroll
+                        for (int v = 0; v < 8; ++v)
+                            *reinterpret_cast<uint4*>(ws + lane * 128 + ((v ^ (lane & 7)) << 4)) = make_uint4(
+                                pack_bf16x2(__uint_as_float(o[8 * v]) * inv_l, __uint_as_float(o[8 * v + 1]) * inv_l),
+                                pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv_l, __uint_as_float(o[8 * v + 3]) * inv_l),
+                                pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv_l, __uint_as_float(o[8 * v + 5]) * inv_l),
+                                pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv_l, __uint_as_float(o[8 * v + 7]) * inv_l));
+                        __syncwarp();
+                        const int q_warp = x.q0 + (warp & 3) * 32;  // the warp's first row
+                        const int cu = lane & 7;                     // 16-byte unit of the row
+                        if (!*abort_flag) {
+                            #pragma unroll
+                            for (int j = 0; j < 8; ++j) {
+                                const int rr = 4 * j + (lane >> 3);  // row within the warp
+                                const uint4 val = *reinterpret_cast<const uint4*>(ws + rr * 128 + ((cu ^ (rr & 7)) << 4));
+                                if (q_warp + rr < p.Nq) {
+                                    const long long g = static_cast<long long>(x.bh) * p.Nq + q_warp + rr;
+                                    reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + g * 64)[cu] = val;
+                                }
+                            }
+                        }
+                        __syncwarp();  // the buffer is written again only after every lane has read it
+                        if (q < p.Nq && !*abort_flag && p.lse != nullptr)
+                            p.lse[r] = l_sum > 0.0f ? (m + __log2f(l_sum)) * kLn2 : -INFINITY;
+                    } else if (q < p.Nq && !*abort_flag) {
+                        // each thread writes its own 128-byte row of O from registers
                         uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + r * 64);
                         #pragma unroll
                         for (int v = 0; v < 8; ++v)
@@ -556,12 +595,12 @@ attn_fwd_short_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 uint32_t o[64];
                 if (tile_ok) {
                     tc_fence_after();
-                    tmem_ld32(lane_tmem + 128, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
-                    tmem_ld32(lane_tmem + 160, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
+                    tmem_ld32(lane_tmem + kShortOCol, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
+                    tmem_ld32(lane_tmem + kShortOCol + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
                     tmem_wait_ld();
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(bar(L::OEMPTY + s));  // the MMA warp may put the next S here
+                    if (lane == 0) mbar_arrive(bar(L::OEMPTY + s));  // O may be overwritten now
                 }
                 // the previous tile's TMA store must have read the staging buffer
                 if ((threadIdx.x & 127) == 0) bulk_wait_group_read0();

@@ -89,15 +89,18 @@ def test_large_scores():
 
 
 @pytest.mark.parametrize("causal", [False, True])
-def test_later_keys_dominate(causal):
-    """Later key chunks exceed the first chunk's maximum by far more than the
+@pytest.mark.parametrize("q_gain", [4.0, 10.0])
+def test_later_keys_dominate(causal, q_gain):
+    """Later 64-key steps exceed the first step's maximum by far more than the
     rescale threshold (2^8): the stored probabilities and the row sum are
-    rescaled by powers of two, several times per row."""
+    rescaled by powers of two, several times per row.  Rescales over the 960
+    rows, counted on these inputs in fp64: gain 4, 2376 with 930 rows rescaling
+    at least twice (causal 951, 296); gain 10, 2537 (causal 1058, 346)."""
     B, H, N = 2, 2, 240
     q, k, v = make_qkv(B, H, H, N, N, 64, seed=17 + causal)
     ramp = torch.linspace(0.05, 8.0, N).view(1, 1, N, 1)
     k = (k.float() * ramp).to(torch.bfloat16)
-    q = (q.float() * 4.0).to(torch.bfloat16)
+    q = (q.float() * q_gain).to(torch.bfloat16)
     out, lse = run_gpu(q, k, v, is_causal=causal)
     ro, rl, ra = reference(q, k, v, is_causal=causal)
     assert_close(out, lse, ro, rl, rabs=ra)

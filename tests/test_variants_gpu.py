@@ -2,6 +2,8 @@
 masks) against the fp64 oracle, with the tolerances of the plain path:
 |O - O_ref| <= 1e-2 beyond the bf16 half-ulp, |LSE - LSE_ref| <= 1e-3, masked
 keys and rows without keys exact."""
+import math
+
 import pytest
 import torch
 
@@ -96,3 +98,25 @@ def test_masked_keys_bit_exact_under_mask2d():
     o2, l2 = run_gpu(q, k2, v2, mask2d=("neighborhood", W, R))
     rows = slice(0, 3 * W)
     assert torch.equal(o1[:, :, rows], o2[:, :, rows]) and torch.equal(l1[:, :, rows], l2[:, :, rows])
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_softcap_polynomial_and_special_function_blocks(d, causal):
+    """Query rows scaled from 0.3 to 30 under cap 30: the warps of the first rows
+    keep every raw score of their key blocks within the polynomial's range
+    (|scale * s / cap| <= 0.75) and take the FMA-pipe tanh, the last ones do not
+    and take 1 - 2 / (1 + e^(2u)); both in one call, against the oracle."""
+    B, H, N, cap = 1, 2, 700, 30.0
+    q, k, v = make_qkv(B, H, H, N, N, d, seed=90 + d + causal)
+    ramp = torch.logspace(math.log10(0.3), math.log10(30.0), N).view(1, 1, N, 1)
+    q = (q.float() * ramp).to(torch.bfloat16)
+    # the premise, per warp of 32 rows: the largest |scale * s / cap| over its keys
+    u = (q.double() @ k.double().transpose(-1, -2)).abs() / math.sqrt(d) / cap
+    if causal:
+        u = u * torch.ones(N, N, dtype=torch.bool).tril()
+    per_warp = torch.stack([u[..., r:r + 32, :].amax(dim=(-1, -2)) for r in range(0, N, 32)], dim=-1)
+    assert (per_warp <= 0.7).any() and (per_warp > 0.8).any()
+    out, lse = run_gpu(q, k, v, is_causal=causal, softcap=cap)
+    ro, rl, ra = reference(q, k, v, is_causal=causal, softcap=cap)
+    assert_close(out, lse, ro, rl, rabs=ra)
