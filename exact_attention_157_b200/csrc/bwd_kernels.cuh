@@ -19,6 +19,10 @@
 //   attn_bwd_kernel<D, false>    dQ: one CTA per 128-row query block, looping over key
 //                                blocks; S = Q K^T, dP = dO V^T, dS to TMEM, dQ += dS K
 // Splitting dQ from dK/dV keeps every accumulator in one CTA's TMEM: no atomics.
+// Each iteration's 128 columns pass in two halves of 64 through two TMEM buffers,
+// so that the elementwise step of one half overlaps the tensor work of its
+// neighbours (the accumulating products of the previous half, S and dP of the
+// next).
 //
 // Score and mask variants (the VAR instantiation), the forward's readings: the
 // score is s = c(x) + mask with x = scale q.k, c(x) = cap tanh(x / cap) under
@@ -128,14 +132,19 @@ struct SmemBwd {
     static constexpr int kStage = 2 * kTile;
     static constexpr int kStages = 2 * kTile;
     static constexpr int kBars = kStages + 2 * kStage;
-    // barriers
-    // PFULL: the first 64 columns of P / dS stored; PFULL1: the last 64
-    static constexpr int FIXFULL = 0, STFULL_ = 1, PFULL = 2, DONE = 3, RFULL = 4, REMPTY = 6, PFULL1 = 8;
-    static constexpr int kNumBars = 9;
+    // barriers, per TMEM buffer b: STFULL + b (S and dP of a half block computed),
+    // PFULL + b (P and dS of it stored); per stage s: RFULL + s, REMPTY + s
+    static constexpr int FIXFULL = 0, DONE = 1, STFULL = 2, PFULL = 4, RFULL = 6, REMPTY = 8;
+    static constexpr int kNumBars = 10;
     static constexpr int kMisc = kBars + 8 * kNumBars;
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;
-    static constexpr int kColA = 0, kColB = 128, kColAcc0 = 256, kColAcc1 = 256 + D;
+    // Two TMEM buffers of one half block (64 columns of the iteration's 128) each:
+    // buffer b holds S (or S^T) in [128 b, 128 b + 64) and dP (dP^T) in
+    // [128 b + 64, 128 b + 128); P and dS (bf16 pairs) overwrite the first 32
+    // columns of each.  The accumulators follow.
+    static constexpr int kHalf = 64;
+    static constexpr int kColBuf = 128, kColDP = 64, kColAcc0 = 256, kColAcc1 = 256 + D;
     static_assert(kColAcc1 + D <= kTmemCols, "TMEM budget");
     static_assert(kAlloc <= 232448, "shared memory budget");
 };
@@ -223,11 +232,10 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     if (threadIdx.x == 0) {
         mbar_init(bar(L::FIXFULL), 1);
-        mbar_init(bar(L::STFULL_), 1);
-        mbar_init(bar(L::PFULL), 128);
-        mbar_init(bar(L::PFULL1), 128);
         mbar_init(bar(L::DONE), 1);
         for (int s = 0; s < 2; ++s) {
+            mbar_init(bar(L::STFULL + s), 1);
+            mbar_init(bar(L::PFULL + s), 128);
             mbar_init(bar(L::RFULL + s), 1);
             mbar_init(bar(L::REMPTY + s), 1);
         }
@@ -295,59 +303,70 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
     } else if (warp == 5) {
         // ================================ MMA issuer ================================
-        constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, false);
+        // The iteration's 128 columns (queries for dK/dV, keys for dQ) go through the
+        // tensor cores in two halves of 64, g = 2 it + hh, alternating between the two
+        // TMEM buffers: while the elementwise warps turn S and dP of half g into P and
+        // dS, the tensor cores run the accumulating products of half g - 1 and S, dP of
+        // half g + 1.  Products of one thread run in order, so S of half g + 2 may
+        // overwrite the buffer whose P and dS the products of half g read.
+        constexpr uint32_t kIdescS = idesc_bf16_f32(128, L::kHalf, false);
         constexpr uint32_t kIdescAcc = idesc_bf16_f32(128, D, true);
         bool ok = n_iter > 0 && !*abort_flag;
         if (ok) ok = mbar_wait_warp(bar(L::FIXFULL), 0, limit, abort_flag, p.epoch, kRoleBwdMma, 1);
         const uint32_t f0 = sbase + L::kFixed0, f1 = sbase + L::kFixed1;
-        for (int it = 0; ok && it < n_iter; ++it) {
-            const int s = it & 1;
-            const uint32_t st0 = sbase + L::kStages + s * L::kStage, st1 = st0 + L::kTile;
-            if (!mbar_wait_warp(bar(L::RFULL + s), (it >> 1) & 1, limit, abort_flag, p.epoch, kRoleBwdMma, 2))
+        const int n_half = 2 * n_iter;
+        // DKDV: S^T = K Q^T, dP^T = V dO^T.  dQ: S = Q K^T, dP = dO V^T.  A = fixed
+        // (f0 / f1), B = the half's 64 rows of the streamed tiles (st0 / st1), K-major
+        // over d; 64 rows are 8 KB into each 128-row, 128-byte swizzled chunk.
+        auto issue_s = [&](int g) -> bool {
+            const int it = g >> 1, hh = g & 1, s = it & 1, buf = g & 1;
+            if (hh == 0 &&
+                !mbar_wait_warp(bar(L::RFULL + s), (it >> 1) & 1, limit, abort_flag, p.epoch, kRoleBwdMma, 2))
+                return false;
+            tc_fence_after();
+            const uint32_t st0 = sbase + L::kStages + s * L::kStage + hh * (L::kHalf * 128), st1 = st0 + L::kTile;
+            const uint32_t cb = tmem + buf * L::kColBuf;
+            #pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
+                mma_ss_warp(cb, smem_desc_sw128(f0 + off, 16, 1024), smem_desc_sw128(st0 + off, 16, 1024), kIdescS,
+                            kk > 0 ? 1u : 0u);
+            }
+            #pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
+                mma_ss_warp(cb + L::kColDP, smem_desc_sw128(f1 + off, 16, 1024), smem_desc_sw128(st1 + off, 16, 1024),
+                            kIdescS, kk > 0 ? 1u : 0u);
+            }
+            mma_commit_warp(bar(L::STFULL + buf));
+            return true;
+        };
+        for (int g = 0; ok && g < 2 && g < n_half; ++g) ok = issue_s(g);
+        for (int g = 0; ok && g < n_half; ++g) {
+            const int it = g >> 1, hh = g & 1, s = it & 1, buf = g & 1;
+            if (!mbar_wait_warp(bar(L::PFULL + buf), (g >> 1) & 1, limit, abort_flag, p.epoch, kRoleBwdMma, 3))
                 { ok = false; break; }
             tc_fence_after();
-            // DKDV: S^T = K Q^T, dP^T = V dO^T.  dQ: S = Q K^T, dP = dO V^T.
-            // A = fixed (f0 / f1), B = streamed (st0 / st1), both K-major over d.
+            // bf16 operands in TMEM (A) times the half's 64 streamed rows as B (MN-major,
+            // 16 rows per step): DKDV: dV += P^T dO, dK += dS^T Q.  dQ: dQ += dS K.
+            const uint32_t st0 = sbase + L::kStages + s * L::kStage, st1 = st0 + L::kTile;
+            const uint32_t cb = tmem + buf * L::kColBuf;
             #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t off = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
-                mma_ss_warp(tmem + L::kColA, smem_desc_sw128(f0 + off, 16, 1024), smem_desc_sw128(st0 + off, 16, 1024),
-                            kIdescS, kk > 0 ? 1u : 0u);
-            }
-            #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t off = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
-                mma_ss_warp(tmem + L::kColB, smem_desc_sw128(f1 + off, 16, 1024), smem_desc_sw128(st1 + off, 16, 1024),
-                            kIdescS, kk > 0 ? 1u : 0u);
-            }
-            mma_commit_warp(bar(L::STFULL_));
-            // bf16 operands in TMEM (A) times a streamed tile as B (MN-major, 16 rows per step):
-            // DKDV: dV += P^T dO (P^T in kColA), dK += dS^T Q (dS^T in kColB).
-            // dQ:   dQ += dS K (dS in kColA).
-            // The first 64 columns (steps 0-3) start as soon as the elementwise warps have
-            // stored them (PFULL), while the last 64 are computed (PFULL1).
-            for (int half = 0; half < 2 && ok; ++half) {
-                if (!mbar_wait_warp(bar(half == 0 ? L::PFULL : L::PFULL1), it & 1, limit, abort_flag, p.epoch,
-                                    kRoleBwdMma, 3 + 4 * half))
-                    { ok = false; break; }
-                tc_fence_after();
-                #pragma unroll
-                for (int k4 = 0; k4 < kBN / 32; ++k4) {
-                    const int kk = half * (kBN / 32) + k4;
-                    const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
-                    if constexpr (DKDV) {
-                        mma_ts_warp(tmem + L::kColAcc0, tmem + L::kColA + kk * 8,
-                                    smem_desc_sw128(st1 + kk * 2048, L::kChunkBytes, 1024), kIdescAcc, acc);
-                        mma_ts_warp(tmem + L::kColAcc1, tmem + L::kColB + kk * 8,
-                                    smem_desc_sw128(st0 + kk * 2048, L::kChunkBytes, 1024), kIdescAcc, acc);
-                    } else {
-                        mma_ts_warp(tmem + L::kColAcc0, tmem + L::kColA + kk * 8,
-                                    smem_desc_sw128(st0 + kk * 2048, L::kChunkBytes, 1024), kIdescAcc, acc);
-                    }
+            for (int k4 = 0; k4 < L::kHalf / 16; ++k4) {
+                const int kk = hh * (L::kHalf / 16) + k4;  // 16-row step within the 128 streamed rows
+                const uint32_t acc = (g > 0 || k4 > 0) ? 1u : 0u;
+                if constexpr (DKDV) {
+                    mma_ts_warp(tmem + L::kColAcc0, cb + k4 * 8, smem_desc_sw128(st1 + kk * 2048, L::kChunkBytes, 1024),
+                                kIdescAcc, acc);
+                    mma_ts_warp(tmem + L::kColAcc1, cb + L::kColDP + k4 * 8,
+                                smem_desc_sw128(st0 + kk * 2048, L::kChunkBytes, 1024), kIdescAcc, acc);
+                } else {
+                    mma_ts_warp(tmem + L::kColAcc0, cb + L::kColDP + k4 * 8,
+                                smem_desc_sw128(st0 + kk * 2048, L::kChunkBytes, 1024), kIdescAcc, acc);
                 }
             }
-            if (!ok) break;
-            mma_commit_warp(bar(L::REMPTY + s));  // the stage may be refilled once these complete
+            if (hh == 1) mma_commit_warp(bar(L::REMPTY + s));  // the stage may be refilled once these complete
+            if (g + 2 < n_half && !issue_s(g + 2)) { ok = false; break; }
         }
         mma_commit_warp(bar(L::DONE));
         mbar_drain(bar(L::DONE), 0, kRoleBwdMma, 4);
@@ -406,74 +425,75 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                            static_cast<long long>(q_row) * p.msq + static_cast<long long>(ib) * kBN;
             }
             if (!ok) continue;
-            const bool got = mbar_wait(bar(L::STFULL_), it & 1, limit, abort_flag, p.epoch, kRoleBwdElem, 2);
-            if (!__all_sync(0xffffffffu, got)) { ok = false; continue; }
-            tc_fence_after();
-            #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t sv[32], dv[32];
-                tmem_ld32(lane_tmem + L::kColA + c * 32, sv);
-                tmem_ld32(lane_tmem + L::kColB + c * 32, dv);
-                tmem_wait_ld();
-                uint32_t pw[16], dw[16];
+            for (int hh = 0; hh < 2 && ok; ++hh) {
+                const int g = 2 * it + hh, hb = g & 1;
+                const bool got = mbar_wait(bar(L::STFULL + hb), (g >> 1) & 1, limit, abort_flag, p.epoch,
+                                           kRoleBwdElem, 2);
+                if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t cb = lane_tmem + hb * L::kColBuf;
                 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    float pp[2], ds[2];
+                for (int c = 0; c < L::kHalf / 32; ++c) {
+                    uint32_t sv[32], dv[32];
+                    tmem_ld32(cb + c * 32, sv);
+                    tmem_ld32(cb + L::kColDP + c * 32, dv);
+                    tmem_wait_ld();
+                    uint32_t pw[16], dw[16];
                     #pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int col = c * 32 + e + u;  // query (DKDV) or key (dQ) within the block
-                        float l2, dd;
-                        bool vis;
-                        if constexpr (DKDV) {
-                            const int qi = ib * kBM + col;
-                            l2 = s_l2[buf][col];  // the same address in every lane: a broadcast
-                            dd = s_dd[buf][col];
-                            vis = key_row < kv_len && (!p.is_causal || key_row <= qi);
-                        } else {
-                            const int kj = ib * kBN + col;
-                            l2 = my_lse2;
-                            dd = my_d;
-                            vis = kj < kv_len && (!p.is_causal || kj <= q_row);
-                        }
-                        if constexpr (!VAR) {
-                            const float pv = vis ? ex2_approx(fmaf(__uint_as_float(sv[e + u]), c2, -l2)) : 0.0f;
-                            pp[u] = pv;
-                            ds[u] = pv * (__uint_as_float(dv[e + u]) - dd);
-                        } else {
-                            // base-2 logit of the capped, masked score, and c'(x)
-                            const float raw = __uint_as_float(sv[e + u]);
-                            float lg = raw * c2, g = 1.0f;
-                            if (p.softcap_on) {
-                                const float t = fmaf(rcp_approx(1.0f + ex2_approx(raw * p.sc_in)), -2.0f, 1.0f);
-                                lg = p.sc_out * t;
-                                g = fmaf(-t, t, 1.0f);
+                    for (int e = 0; e < 32; e += 2) {
+                        float pp[2], ds[2];
+                        #pragma unroll
+                        for (int u = 0; u < 2; ++u) {
+                            // query (DKDV) or key (dQ) within the iteration's 128
+                            const int col = hh * L::kHalf + c * 32 + e + u;
+                            float l2, dd;
+                            bool vis;
+                            if constexpr (DKDV) {
+                                const int qi = ib * kBM + col;
+                                l2 = s_l2[buf][col];  // the same address in every lane: a broadcast
+                                dd = s_dd[buf][col];
+                                vis = key_row < kv_len && (!p.is_causal || key_row <= qi);
+                            } else {
+                                const int kj = ib * kBN + col;
+                                l2 = my_lse2;
+                                dd = my_d;
+                                vis = kj < kv_len && (!p.is_causal || kj <= q_row);
                             }
-                            if (m2) vis = vis && bwd_visible_2d(p, my_xy, s_xy[buf][col]);
-                            // (padding query rows past Nq have no mask row: not read)
-                            if (mrow != nullptr && vis && (DKDV ? ib * kBM + col < p.Nq : q_row < p.Nq)) {
-                                const long long off = DKDV ? static_cast<long long>(col) * p.msq : col;
-                                lg = fmaf(__ldg(mrow + off), kLog2e, lg);
+                            if constexpr (!VAR) {
+                                const float pv = vis ? ex2_approx(fmaf(__uint_as_float(sv[e + u]), c2, -l2)) : 0.0f;
+                                pp[u] = pv;
+                                ds[u] = pv * (__uint_as_float(dv[e + u]) - dd);
+                            } else {
+                                // base-2 logit of the capped, masked score, and c'(x)
+                                const float raw = __uint_as_float(sv[e + u]);
+                                float lg = raw * c2, gd = 1.0f;
+                                if (p.softcap_on) {
+                                    const float t = fmaf(rcp_approx(1.0f + ex2_approx(raw * p.sc_in)), -2.0f, 1.0f);
+                                    lg = p.sc_out * t;
+                                    gd = fmaf(-t, t, 1.0f);
+                                }
+                                if (m2) vis = vis && bwd_visible_2d(p, my_xy, s_xy[buf][col]);
+                                // (padding query rows past Nq have no mask row: not read)
+                                if (mrow != nullptr && vis && (DKDV ? ib * kBM + col < p.Nq : q_row < p.Nq)) {
+                                    const long long off = DKDV ? static_cast<long long>(col) * p.msq : col;
+                                    lg = fmaf(__ldg(mrow + off), kLog2e, lg);
+                                }
+                                const float pv = vis ? ex2_approx(lg - l2) : 0.0f;
+                                pp[u] = pv;
+                                ds[u] = pv * (__uint_as_float(dv[e + u]) - dd) * gd;
                             }
-                            const float pv = vis ? ex2_approx(lg - l2) : 0.0f;
-                            pp[u] = pv;
-                            ds[u] = pv * (__uint_as_float(dv[e + u]) - dd) * g;
                         }
+                        pw[e / 2] = pack_bf16x2(pp[0], pp[1]);
+                        dw[e / 2] = pack_bf16x2(ds[0], ds[1]);
                     }
-                    pw[e / 2] = pack_bf16x2(pp[0], pp[1]);
-                    dw[e / 2] = pack_bf16x2(ds[0], ds[1]);
+                    // P (DKDV only) over the S columns already read, dS over the dP columns
+                    if constexpr (DKDV) tmem_st16(cb + c * 16, pw);
+                    tmem_st16(cb + L::kColDP + c * 16, dw);
                 }
-                if constexpr (DKDV) {
-                    tmem_st16(lane_tmem + L::kColA + c * 16, pw);  // P^T over S^T columns already read
-                    tmem_st16(lane_tmem + L::kColB + c * 16, dw);  // dS^T over dP^T columns already read
-                } else {
-                    tmem_st16(lane_tmem + L::kColA + c * 16, dw);  // dS over S columns already read
-                }
-                if (c == 1 || c == 3) {
-                    // columns 0-63 (then 64-127) stored: their products may start
-                    tmem_wait_st();
-                    tc_fence_before();
-                    mbar_arrive(bar(c == 1 ? L::PFULL : L::PFULL1));
-                }
+                // the half's P and dS stored: its products may start
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar(L::PFULL + hb));
             }
         }
         // ------------------------------------------------------------- epilogue
