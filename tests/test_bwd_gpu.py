@@ -149,3 +149,12 @@ def test_bwd_variants_off_equal_plain():
     a = run_bwd(q, k, v, do)
     b = run_bwd(q, k, v, do, softcap=0.0, mask2d=None)
     assert all(torch.equal(x, y) for x, y in zip(a, b))
+
+
+@pytest.mark.parametrize("N,causal", [(4096, False), (2048, True)])
+def test_bwd_long_head_against_the_oracle(N, causal):
+    """One head of the long workload's shape (d = 128, N = 4096: each dK/dV CTA
+    loops over 32 query blocks, each dQ CTA over 32 key blocks, 64 half blocks
+    through the two TMEM buffers, as in the benchmark's launch; the causal case at
+    N = 2048), every element of dQ, dK and dV against the oracle."""
+    check(1, 1, 1, N, N, 128, seed=1100 + N + causal, causal=causal)
