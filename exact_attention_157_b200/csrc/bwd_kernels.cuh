@@ -135,7 +135,8 @@ struct SmemBwd {
     // barriers, per TMEM buffer b: STFULL + b (S and dP of a half block computed),
     // PFULL + b (P and dS of it stored); per stage s: RFULL + s, REMPTY + s
     static constexpr int FIXFULL = 0, DONE = 1, STFULL = 2, PFULL = 4, RFULL = 6, REMPTY = 8;
-    static constexpr int kNumBars = 10;
+    static constexpr int FIXTM = 10;  // dQ kernel: Q and dO copied into TMEM (128 arrivals)
+    static constexpr int kNumBars = 11;
     static constexpr int kMisc = kBars + 8 * kNumBars;
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;
@@ -145,6 +146,10 @@ struct SmemBwd {
     // columns of each.  The accumulators follow.
     static constexpr int kHalf = 64;
     static constexpr int kColBuf = 128, kColDP = 64, kColAcc0 = 256, kColAcc1 = 256 + D;
+    // dQ kernel: the fixed Q and dO as bf16 pairs (D / 2 columns each), the A
+    // operands of S and dP, so that only the streamed K and V come from shared memory
+    static constexpr int kColFixT = 384;
+    static_assert(kColFixT + D <= kTmemCols && kColAcc0 + D <= kColFixT, "TMEM budget of the dQ kernel");
     static_assert(kColAcc1 + D <= kTmemCols, "TMEM budget");
     static_assert(kAlloc <= 232448, "shared memory budget");
 };
@@ -233,6 +238,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (threadIdx.x == 0) {
         mbar_init(bar(L::FIXFULL), 1);
         mbar_init(bar(L::DONE), 1);
+        mbar_init(bar(L::FIXTM), 128);
         for (int s = 0; s < 2; ++s) {
             mbar_init(bar(L::STFULL + s), 1);
             mbar_init(bar(L::PFULL + s), 128);
@@ -313,6 +319,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         constexpr uint32_t kIdescAcc = idesc_bf16_f32(128, D, true);
         bool ok = n_iter > 0 && !*abort_flag;
         if (ok) ok = mbar_wait_warp(bar(L::FIXFULL), 0, limit, abort_flag, p.epoch, kRoleBwdMma, 1);
+        if (!DKDV && ok) ok = mbar_wait_warp(bar(L::FIXTM), 0, limit, abort_flag, p.epoch, kRoleBwdMma, 5);
         const uint32_t f0 = sbase + L::kFixed0, f1 = sbase + L::kFixed1;
         const int n_half = 2 * n_iter;
         // DKDV: S^T = K Q^T, dP^T = V dO^T.  dQ: S = Q K^T, dP = dO V^T.  A = fixed
@@ -329,14 +336,22 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t off = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
-                mma_ss_warp(cb, smem_desc_sw128(f0 + off, 16, 1024), smem_desc_sw128(st0 + off, 16, 1024), kIdescS,
-                            kk > 0 ? 1u : 0u);
+                if constexpr (DKDV)
+                    mma_ss_warp(cb, smem_desc_sw128(f0 + off, 16, 1024), smem_desc_sw128(st0 + off, 16, 1024), kIdescS,
+                                kk > 0 ? 1u : 0u);
+                else  // A = Q from TMEM, 16 columns of d (8 TMEM columns) per step
+                    mma_ts_warp(cb, tmem + L::kColFixT + kk * 8, smem_desc_sw128(st0 + off, 16, 1024), kIdescS,
+                                kk > 0 ? 1u : 0u);
             }
             #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t off = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
-                mma_ss_warp(cb + L::kColDP, smem_desc_sw128(f1 + off, 16, 1024), smem_desc_sw128(st1 + off, 16, 1024),
-                            kIdescS, kk > 0 ? 1u : 0u);
+                if constexpr (DKDV)
+                    mma_ss_warp(cb + L::kColDP, smem_desc_sw128(f1 + off, 16, 1024),
+                                smem_desc_sw128(st1 + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+                else
+                    mma_ts_warp(cb + L::kColDP, tmem + L::kColFixT + D / 2 + kk * 8,
+                                smem_desc_sw128(st1 + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
             }
             mma_commit_warp(bar(L::STFULL + buf));
             return true;
@@ -396,6 +411,36 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         int2 my_xy = make_int2(0, 0);
         if (m2) my_xy = bwd_coord(p, DKDV ? key_row : q_row);
         bool ok = !*abort_flag;
+        if constexpr (!DKDV) {
+            // Q and dO of this CTA's 128 rows into TMEM (this thread's row: lane = row,
+            // bf16 pairs along d), read from their 128-byte swizzled shared-memory tiles
+            if (n_iter > 0) {
+                if (ok) {
+                    const bool got = mbar_wait(bar(L::FIXFULL), 0, limit, abort_flag, p.epoch, kRoleBwdElem, 4);
+                    ok = __all_sync(0xffffffffu, got);
+                }
+                if (ok) {
+                    #pragma unroll
+                    for (int f = 0; f < 2; ++f) {
+                        const uint8_t* tile = smem + (f == 0 ? L::kFixed0 : L::kFixed1);
+                        #pragma unroll
+                        for (int c = 0; c < L::kChunks; ++c) {
+                            uint32_t w[32];
+                            #pragma unroll
+                            for (int u = 0; u < 8; ++u) {
+                                const uint4 v = *reinterpret_cast<const uint4*>(
+                                    tile + c * L::kChunkBytes + row * 128 + ((u ^ (row & 7)) << 4));
+                                w[4 * u] = v.x; w[4 * u + 1] = v.y; w[4 * u + 2] = v.z; w[4 * u + 3] = v.w;
+                            }
+                            tmem_st32(lane_tmem + L::kColFixT + f * (D / 2) + c * 32, w);
+                        }
+                    }
+                    tmem_wait_st();
+                }
+                tc_fence_before();
+                mbar_arrive(bar(L::FIXTM));  // also after a failed wait: the MMA warp then finds the abort
+            }
+        }
         // Every warp runs the named barrier of every iteration, also after a failed
         // wait (it then skips the iteration's work), so that none is left waiting.
         for (int it = 0; it < n_iter; ++it) {
