@@ -403,7 +403,8 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // before the wait for S^T and dP^T (the loads overlap those products) and shared
         // through a double buffer (a buffer is rewritten two iterations later, after
         // every thread has passed the barrier of the iteration between)
-        __shared__ float s_l2[2][kBM], s_dd[2][kBM];
+        __shared__ __align__(16) float s_l2[2][kBM];
+        __shared__ __align__(16) float s_dd[2][kBM];
         // VAR with a 2-D mask: grid coordinates of this iteration's columns (queries
         // or keys), double-buffered like LSE2 and D, and of this thread's own row
         __shared__ int2 s_xy[2][kBM];
@@ -477,6 +478,54 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t cb = lane_tmem + hb * L::kColBuf;
+                // Every score of the half visible for every row of the warp (no key past
+                // the key length, no pair across the causal diagonal): no per-element test.
+                bool all_vis;
+                if constexpr (DKDV) {
+                    const int q_first = ib * kBM + hh * L::kHalf;
+                    all_vis = key_row < kv_len && (!p.is_causal || key_row <= q_first);
+                } else {
+                    const int k_last = ib * kBN + hh * L::kHalf + L::kHalf - 1;
+                    all_vis = k_last < kv_len && (!p.is_causal || k_last <= q_row);
+                }
+                all_vis = __all_sync(0xffffffffu, all_vis);
+                if (!VAR && all_vis) {
+                    #pragma unroll
+                    for (int c = 0; c < L::kHalf / 32; ++c) {
+                        uint32_t sv[32], dv[32];
+                        tmem_ld32(cb + c * 32, sv);
+                        tmem_ld32(cb + L::kColDP + c * 32, dv);
+                        tmem_wait_ld();
+                        uint32_t pw[16], dw[16];
+                        #pragma unroll
+                        for (int e = 0; e < 32; e += 4) {
+                            float l2[4], dd[4];
+                            if constexpr (DKDV) {
+                                // the same 16 bytes in every lane: broadcast loads
+                                const int col = hh * L::kHalf + c * 32 + e;
+                                const float4 a = *reinterpret_cast<const float4*>(&s_l2[buf][col]);
+                                const float4 b4 = *reinterpret_cast<const float4*>(&s_dd[buf][col]);
+                                l2[0] = a.x; l2[1] = a.y; l2[2] = a.z; l2[3] = a.w;
+                                dd[0] = b4.x; dd[1] = b4.y; dd[2] = b4.z; dd[3] = b4.w;
+                            } else {
+                                #pragma unroll
+                                for (int u = 0; u < 4; ++u) { l2[u] = my_lse2; dd[u] = my_d; }
+                            }
+                            float pv[4], ds[4];
+                            #pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                pv[u] = ex2_approx(fmaf(__uint_as_float(sv[e + u]), c2, -l2[u]));
+                                ds[u] = pv[u] * (__uint_as_float(dv[e + u]) - dd[u]);
+                            }
+                            pw[e / 2] = pack_bf16x2(pv[0], pv[1]);
+                            pw[e / 2 + 1] = pack_bf16x2(pv[2], pv[3]);
+                            dw[e / 2] = pack_bf16x2(ds[0], ds[1]);
+                            dw[e / 2 + 1] = pack_bf16x2(ds[2], ds[3]);
+                        }
+                        if constexpr (DKDV) tmem_st16(cb + c * 16, pw);
+                        tmem_st16(cb + L::kColDP + c * 16, dw);
+                    }
+                } else {
                 #pragma unroll
                 for (int c = 0; c < L::kHalf / 32; ++c) {
                     uint32_t sv[32], dv[32];
@@ -534,6 +583,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     // P (DKDV only) over the S columns already read, dS over the dP columns
                     if constexpr (DKDV) tmem_st16(cb + c * 16, pw);
                     tmem_st16(cb + L::kColDP + c * 16, dw);
+                }
                 }
                 // the half's P and dS stored: its products may start
                 tmem_wait_st();
