@@ -32,8 +32,9 @@
 // from x as above.  The additive mask has no gradient here.  Blocks that a 2-D
 // mask hides entirely are computed (their P is 0), not skipped.
 //
-// Warps (192 threads): 0-3 elementwise (thread = TMEM lane = row), 4 TMA producer,
-// 5 TMEM owner and MMA issuer (warp-uniform, elect.sync).  Every wait is bounded.
+// Warps (320 threads): 0-7 elementwise (thread = TMEM lane = row; warps w and w + 4
+// share a lane quarter and split each half block's columns), 8 TMA producer, 9 TMEM
+// owner and MMA issuer (warp-uniform, elect.sync).  Every wait is bounded.
 #pragma once
 
 #include "fwd_common.cuh"
@@ -82,7 +83,13 @@ __device__ __forceinline__ bool bwd_visible_2d(const BwdParams& p, int2 a, int2 
     return a.x == b.x && a.y == b.y;
 }
 
-constexpr int kBwdThreads = 192;
+// Elementwise warps: kBwdSplit per TMEM lane quarter, each taking 1 / kBwdSplit of
+// every half block's columns; then the TMA producer warp and the MMA warp.
+constexpr int kBwdElemWarps = 8;
+constexpr int kBwdSplit = kBwdElemWarps / 4;
+constexpr int kBwdElemThreads = 32 * kBwdElemWarps;
+constexpr int kBwdProducerWarp = kBwdElemWarps, kBwdMmaWarp = kBwdElemWarps + 1;
+constexpr int kBwdThreads = 32 * (kBwdElemWarps + 2);
 enum : unsigned int { kRoleBwdElem = 4, kRoleBwdProducer = 5, kRoleBwdMma = 6, kRoleBwdPrep = 7 };
 
 // D_i = sum_t dO_it O_it and LSE2_i, one warp per (head, padded row).
@@ -142,8 +149,8 @@ struct SmemBwd {
     static constexpr int kAlloc = kBytes + 1024;
     // Two TMEM buffers of one half block (64 columns of the iteration's 128) each:
     // buffer b holds S (or S^T) in [128 b, 128 b + 64) and dP (dP^T) in
-    // [128 b + 64, 128 b + 128); P and dS (bf16 pairs) overwrite the first 32
-    // columns of each.  The accumulators follow.
+    // [128 b + 64, 128 b + 128); P and dS (bf16 pairs) of each 32-column chunk
+    // overwrite the first 16 columns of that chunk.  The accumulators follow.
     static constexpr int kHalf = 64;
     static constexpr int kColBuf = 128, kColDP = 64, kColAcc0 = 256, kColAcc1 = 256 + D;
     // dQ kernel: the fixed Q and dO as bf16 pairs (D / 2 columns each), the A
@@ -157,9 +164,12 @@ struct SmemBwd {
 // Writes one row of `D` fp32 TMEM columns, times `mul`, as bf16 to global `dst`
 // (or zeros when `zero`), 32 columns per TMEM load.
 template <int D>
-__device__ __forceinline__ void store_row_bf16(uint32_t taddr, uint16_t* dst, float mul, bool zero, bool write) {
+__device__ __forceinline__ void store_row_bf16(uint32_t taddr, uint16_t* dst, float mul, bool zero, bool write,
+                                               int c0 = 0, int nc = D / 32) {
     #pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
+    for (int ci = 0; ci < D / 32; ++ci) {
+        if (ci >= nc) break;
+        const int c = c0 + ci;
         uint32_t v[32];
         if (!zero) {
             tmem_ld32(taddr + c * 32, v);
@@ -238,21 +248,21 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (threadIdx.x == 0) {
         mbar_init(bar(L::FIXFULL), 1);
         mbar_init(bar(L::DONE), 1);
-        mbar_init(bar(L::FIXTM), 128);
+        mbar_init(bar(L::FIXTM), kBwdElemThreads);
         for (int s = 0; s < 2; ++s) {
             mbar_init(bar(L::STFULL + s), 1);
-            mbar_init(bar(L::PFULL + s), 128);
+            mbar_init(bar(L::PFULL + s), kBwdElemThreads);
             mbar_init(bar(L::RFULL + s), 1);
             mbar_init(bar(L::REMPTY + s), 1);
         }
         *abort_flag = launch_aborted(p.epoch) ? 1 : 0;
         fence_mbar_init();
     }
-    if (warp == 5) {
+    if (warp == kBwdMmaWarp) {
         tmem_alloc(smem_u32(tmem_slot), kTmemCols);
         tmem_relinquish();
     }
-    if (warp == 4 && lane == 0) {
+    if (warp == kBwdProducerWarp && lane == 0) {
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
         prefetch_tmap(&tm_v);
@@ -263,7 +273,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 4) {
+    if (warp == kBwdProducerWarp) {
         // =============================== TMA producer ===============================
         if (lane == 0 && n_iter > 0 && !*abort_flag) {
             bool ok = true;
@@ -307,7 +317,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             for (int s = 0; s < 2; ++s)
                 if (loads[s] > 0) mbar_drain(bar(L::RFULL + s), (loads[s] - 1) & 1, kRoleBwdProducer, 3);
         }
-    } else if (warp == 5) {
+    } else if (warp == kBwdMmaWarp) {
         // ================================ MMA issuer ================================
         // The iteration's 128 columns (queries for dK/dV, keys for dQ) go through the
         // tensor cores in two halves of 64, g = 2 it + hh, alternating between the two
@@ -369,14 +379,16 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             #pragma unroll
             for (int k4 = 0; k4 < L::kHalf / 16; ++k4) {
                 const int kk = hh * (L::kHalf / 16) + k4;  // 16-row step within the 128 streamed rows
+                // P and dS of 32-column chunk c sit in the first 16 columns of that chunk
+                const uint32_t pc = (k4 >> 1) * 32 + (k4 & 1) * 8;
                 const uint32_t acc = (g > 0 || k4 > 0) ? 1u : 0u;
                 if constexpr (DKDV) {
-                    mma_ts_warp(tmem + L::kColAcc0, cb + k4 * 8, smem_desc_sw128(st1 + kk * 2048, L::kChunkBytes, 1024),
+                    mma_ts_warp(tmem + L::kColAcc0, cb + pc, smem_desc_sw128(st1 + kk * 2048, L::kChunkBytes, 1024),
                                 kIdescAcc, acc);
-                    mma_ts_warp(tmem + L::kColAcc1, cb + L::kColDP + k4 * 8,
+                    mma_ts_warp(tmem + L::kColAcc1, cb + L::kColDP + pc,
                                 smem_desc_sw128(st0 + kk * 2048, L::kChunkBytes, 1024), kIdescAcc, acc);
                 } else {
-                    mma_ts_warp(tmem + L::kColAcc0, cb + L::kColDP + k4 * 8,
+                    mma_ts_warp(tmem + L::kColAcc0, cb + L::kColDP + pc,
                                 smem_desc_sw128(st0 + kk * 2048, L::kChunkBytes, 1024), kIdescAcc, acc);
                 }
             }
@@ -387,8 +399,9 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mbar_drain(bar(L::DONE), 0, kRoleBwdMma, 4);
     } else {
         // ============================ elementwise warps =============================
-        const int row = warp * 32 + lane;  // TMEM lane
-        const uint32_t lane_tmem = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+        const int quarter = warp & 3, sub = warp >> 2;  // TMEM lane quarter, column share
+        const int row = quarter * 32 + lane;            // TMEM lane
+        const uint32_t lane_tmem = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
         const float c2 = p.scale_log2;
         // per-row constants of the dQ kernel (rows are queries)
         const int q_row = DKDV ? 0 : blk * kBM + row;
@@ -423,6 +436,7 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 if (ok) {
                     #pragma unroll
                     for (int f = 0; f < 2; ++f) {
+                        if (kBwdSplit == 2 && f != sub) continue;  // Q by one warp of the quarter, dO by the other
                         const uint8_t* tile = smem + (f == 0 ? L::kFixed0 : L::kFixed1);
                         #pragma unroll
                         for (int c = 0; c < L::kChunks; ++c) {
@@ -452,13 +466,15 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if constexpr (DKDV) {
                 // rows are padded to a multiple of 128 per head: row < 128 stays in bounds
                 const long long r = static_cast<long long>(b * p.Hq + iter_head(it)) * p.nq_pad + ib * kBM;
-                s_l2[buf][row] = __ldg(p.lse2 + r + row);
-                s_dd[buf][row] = __ldg(p.delta + r + row);
-                if (m2) s_xy[buf][row] = bwd_coord(p, ib * kBM + row);
-                named_barrier_sync(1, kBM);
+                if (sub == 0) {
+                    s_l2[buf][row] = __ldg(p.lse2 + r + row);
+                    s_dd[buf][row] = __ldg(p.delta + r + row);
+                    if (m2) s_xy[buf][row] = bwd_coord(p, ib * kBM + row);
+                }
+                named_barrier_sync(1, kBwdElemThreads);
             } else if (m2) {
-                s_xy[buf][row] = bwd_coord(p, ib * kBN + row);
-                named_barrier_sync(1, kBM);
+                if (sub == 0) s_xy[buf][row] = bwd_coord(p, ib * kBN + row);
+                named_barrier_sync(1, kBwdElemThreads);
             }
             // VAR: the additive mask row of this thread (DKDV: column = query, row = key)
             const float* mrow = nullptr;
@@ -489,9 +505,11 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     all_vis = k_last < kv_len && (!p.is_causal || k_last <= q_row);
                 }
                 all_vis = __all_sync(0xffffffffu, all_vis);
+                constexpr int kMyChunks = L::kHalf / 32 / kBwdSplit;  // 32-column chunks of this warp
                 if (!VAR && all_vis) {
                     #pragma unroll
-                    for (int c = 0; c < L::kHalf / 32; ++c) {
+                    for (int ci = 0; ci < kMyChunks; ++ci) {
+                        const int c = sub * kMyChunks + ci;
                         uint32_t sv[32], dv[32];
                         tmem_ld32(cb + c * 32, sv);
                         tmem_ld32(cb + L::kColDP + c * 32, dv);
@@ -522,12 +540,13 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                             dw[e / 2] = pack_bf16x2(ds[0], ds[1]);
                             dw[e / 2 + 1] = pack_bf16x2(ds[2], ds[3]);
                         }
-                        if constexpr (DKDV) tmem_st16(cb + c * 16, pw);
-                        tmem_st16(cb + L::kColDP + c * 16, dw);
+                        if constexpr (DKDV) tmem_st16(cb + c * 32, pw);
+                        tmem_st16(cb + L::kColDP + c * 32, dw);
                     }
                 } else {
                 #pragma unroll
-                for (int c = 0; c < L::kHalf / 32; ++c) {
+                for (int ci = 0; ci < kMyChunks; ++ci) {
+                    const int c = sub * kMyChunks + ci;
                     uint32_t sv[32], dv[32];
                     tmem_ld32(cb + c * 32, sv);
                     tmem_ld32(cb + L::kColDP + c * 32, dv);
@@ -580,9 +599,11 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         pw[e / 2] = pack_bf16x2(pp[0], pp[1]);
                         dw[e / 2] = pack_bf16x2(ds[0], ds[1]);
                     }
-                    // P (DKDV only) over the S columns already read, dS over the dP columns
-                    if constexpr (DKDV) tmem_st16(cb + c * 16, pw);
-                    tmem_st16(cb + L::kColDP + c * 16, dw);
+                    // P (DKDV only) over this chunk's S columns, already read by this
+                    // thread, dS over its dP columns (a warp sharing the lane quarter
+                    // reads the other chunk: no store may land there)
+                    if constexpr (DKDV) tmem_st16(cb + c * 32, pw);
+                    tmem_st16(cb + L::kColDP + c * 32, dw);
                 }
                 }
                 // the half's P and dS stored: its products may start
@@ -603,19 +624,23 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if constexpr (DKDV) {
                 const bool write = key_row < p.Nk;
                 const long long base = (static_cast<long long>(b * p.Hkv + hk) * p.Nk + key_row) * D;
-                store_row_bf16<D>(lane_tmem + L::kColAcc0, p.dv + base, 1.0f, n_iter == 0, write);
-                store_row_bf16<D>(lane_tmem + L::kColAcc1, p.dk + base, p.scale, n_iter == 0, write);
+                if (kBwdSplit == 1 || sub == 0)
+                    store_row_bf16<D>(lane_tmem + L::kColAcc0, p.dv + base, 1.0f, n_iter == 0, write);
+                if (kBwdSplit == 1 || sub == 1)
+                    store_row_bf16<D>(lane_tmem + L::kColAcc1, p.dk + base, p.scale, n_iter == 0, write);
             } else {
                 const bool write = q_row < p.Nq;
                 const long long base = (static_cast<long long>(blockIdx.y) * p.Nq + q_row) * D;
-                store_row_bf16<D>(lane_tmem + L::kColAcc0, p.dq + base, p.scale, n_iter == 0, write);
+                constexpr int kMine = D / 32 / kBwdSplit;  // 32-column chunks of dQ this warp writes
+                store_row_bf16<D>(lane_tmem + L::kColAcc0, p.dq + base, p.scale, n_iter == 0, write, sub * kMine,
+                                  kMine);
             }
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == kBwdMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
