@@ -456,22 +456,33 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 mbar_arrive(bar(L::FIXTM));  // also after a failed wait: the MMA warp then finds the abort
             }
         }
+        // DKDV: LSE2 and D of query `row` of an iteration's block, loaded one iteration
+        // ahead into registers so that their latency overlaps the previous iteration
+        // (rows are padded to a multiple of 128 per head: row < 128 stays in bounds)
+        float pre_l2 = 0.0f, pre_dd = 0.0f;
+        auto prefetch_rows = [&](int it2) {
+            if (DKDV && sub == 0 && it2 < n_iter) {
+                const long long r = static_cast<long long>(b * p.Hq + iter_head(it2)) * p.nq_pad + iter_blk(it2) * kBM;
+                pre_l2 = __ldg(p.lse2 + r + row);
+                pre_dd = __ldg(p.delta + r + row);
+            }
+        };
+        prefetch_rows(0);
         // Every warp runs the named barrier of every iteration, also after a failed
         // wait (it then skips the iteration's work), so that none is left waiting.
         for (int it = 0; it < n_iter; ++it) {
             const int ib = iter_blk(it);
-            // DKDV: LSE2 and D of this iteration's 128 queries (the same addresses in every
-            // lane: broadcast loads; rows are padded to 128, so 16-byte aligned)
+            // DKDV: LSE2 and D of this iteration's 128 queries in shared memory, read by
+            // every lane at the same address (broadcast loads)
             const int buf = it & 1;
             if constexpr (DKDV) {
-                // rows are padded to a multiple of 128 per head: row < 128 stays in bounds
-                const long long r = static_cast<long long>(b * p.Hq + iter_head(it)) * p.nq_pad + ib * kBM;
                 if (sub == 0) {
-                    s_l2[buf][row] = __ldg(p.lse2 + r + row);
-                    s_dd[buf][row] = __ldg(p.delta + r + row);
+                    s_l2[buf][row] = pre_l2;
+                    s_dd[buf][row] = pre_dd;
                     if (m2) s_xy[buf][row] = bwd_coord(p, ib * kBM + row);
                 }
                 named_barrier_sync(1, kBwdElemThreads);
+                prefetch_rows(it + 1);
             } else if (m2) {
                 if (sub == 0) s_xy[buf][row] = bwd_coord(p, ib * kBN + row);
                 named_barrier_sync(1, kBwdElemThreads);
