@@ -226,6 +226,16 @@ cudaError_t launch_pp(const CUtensorMap& tq, const CUtensorMap& tk, const CUtens
     constexpr int kSmem = SmemPPFor<D, NSLOT, QS, false>::kAlloc;
     FwdParams p = p_in;
     set_fast_divs(p);
+    // A last round of two-tile units that would fill at most half the CTAs runs as
+    // single-tile units, two per unit (d = 64, plain and additive-mask launches
+    // without a causal mask; causal ones pair heavy and light units instead).
+    const int n_units = p.B * p.Hq * p.n_qtiles * p.n_splits;
+    const int tail = static_cast<int>(n_units % static_cast<int>(grid));
+    const bool split_tail = D == 64 && p.n_splits == 1 && !p.is_causal && p.unit_run == 1 && !p.softcap_on &&
+                            p.m2_kind == 0 && n_units > static_cast<int>(grid) && tail > 0 &&
+                            2 * tail <= static_cast<int>(grid);
+    p.n_full_units = split_tail ? n_units - tail : n_units;
+    p.n_units_total = split_tail ? n_units + tail : n_units;
     if (p.n_splits > 1)
         attn_fwd_pp_kernel<D, NSLOT, QS, M, true, false, false><<<grid, kPPThreads, kSmem, stream>>>(tq, tk, tv, to, p);
     else if (!M && (p.softcap_on || p.m2_kind != 0))
@@ -772,6 +782,7 @@ extern "C" attn_status_t attn_fwd_fp8(const void* q8, const void* k8, const void
     const long long want = (n_units + p.unit_run - 1) / p.unit_run;
     const unsigned g = static_cast<unsigned>(want < sms ? want : sms);
     set_fast_divs(p);
+    p.n_full_units = p.n_units_total = static_cast<int>(n_units);
     attn_fwd_pp_kernel<128, kSlotsF8, kQStagesF8, false, false, false, true>
         <<<g, kPPThreads, SmemF8::kAlloc, static_cast<cudaStream_t>(stream)>>>(tq, tk, tv, tq, p);
     const cudaError_t e = cudaGetLastError();

@@ -65,6 +65,10 @@ struct FwdParams {
     float* lse;
     void* out;     // O base (bf16), for rows written without the TMA store
     int unit_run;  // persistent kernel: consecutive units per CTA turn (1 or 2)
+    // Units [0, n_full_units) hold two 128-row tiles; the units after them, up to
+    // n_units_total, are the single tiles of the remaining two-tile units (a last
+    // round that would leave SMs idle is run as twice as many half-size units).
+    int n_full_units, n_units_total;
     // split-KV mode: every unit covers one range of split_keys keys (a multiple of
     // 128); partial results go to the workspace, [n_splits][B*Hq][Nq][d] for O
     // (fp32, normalised by the partial row sum) and [n_splits][B*Hq][Nq] for LSE

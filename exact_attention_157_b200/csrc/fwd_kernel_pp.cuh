@@ -192,9 +192,20 @@ __device__ __forceinline__ int unit_seq(int c, int k, int G, int P) {
 // FAST: the unit decode divides by multiplication (FastDiv).  Measured on B200: it
 // pays where units are short and many per CTA (d = 64: vit -4 %, unet_cross -8 %
 // time), and costs 2-3 % at d = 128, whose units run 32 key blocks each.
+// The two-tile unit that sequence position s belongs to (s itself below
+// n_full_units; a single tile of unit n_full_units + (s - n_full_units) / 2 after).
+// Single-tile units exist only in the d = 64 instantiations (SINGLE); at d = 128 a
+// unit runs 32 key blocks per tile and a last round costs little.
+template <bool SINGLE>
+__device__ __forceinline__ int unit_base(const FwdParams& p, int s) {
+    if constexpr (!SINGLE) return s;
+    return s < p.n_full_units ? s : p.n_full_units + ((s - p.n_full_units) >> 1);
+}
+
 template <bool FAST>
 __device__ __forceinline__ int unit_key_len(const FwdParams& p, int s, int n_units) {
     if (p.key_lens == nullptr || s >= n_units) return p.Nk;
+    s = unit_base<FAST>(p, s);
     if constexpr (FAST) return __ldg(p.key_lens + fdiv(fdiv(s, p.fd_per_head), p.fd_hq));
     return __ldg(p.key_lens + (s / (p.n_qtiles * p.n_splits)) / p.Hq);
 }
@@ -205,6 +216,9 @@ template <bool SPLIT, bool MOD, bool FAST>
 __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int s, int kv_len, bool report) {
     Unit x;
     int pos;
+    // a single-tile unit: 1 = the first 128 rows of its unit, 2 = the second
+    const int single = !FAST || s < p.n_full_units ? 0 : 1 + ((s - p.n_full_units) & 1);
+    s = unit_base<FAST>(p, s);
     if constexpr (SPLIT) {
         const int per_head = p.n_qtiles * p.n_splits;
         x.bh = FAST ? fdiv(s, p.fd_per_head) : s / per_head;
@@ -249,6 +263,16 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int s, int kv_le
         x.n_t[t] = end > k_lo ? (end - k_lo + kBN - 1) / kBN : 0;
     }
     if (!x.tile_b_valid) x.n_t[1] = 0;
+    if (single != 0) {
+        // (only without causal masks and 2-D masks: both tiles of the unit see the
+        // same key blocks, so tile B's count serves the single tile)
+        if (single == 2) {
+            x.q0 += kBM;
+            x.n_t[0] = x.tile_b_valid ? x.n_t[1] : 0;
+        }
+        x.tile_b_valid = false;
+        x.n_t[1] = 0;
+    }
     return x;
 }
 
@@ -281,7 +305,7 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     // p.n_qtiles counts 256-row units per head; p.n_splits key ranges per head
-    const int n_units = p.B * p.Hq * p.n_qtiles * p.n_splits;
+    const int n_units = p.n_units_total;
 
     auto bar = [&](int i) -> uint32_t { return sbase + L::kBars + 8u * i; };
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
@@ -890,7 +914,7 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 // directly (this unit loaded nothing and owns no Q buffer).
                 tc_fence_before();
                 mbar_arrive(bar(L::OEMPTY + t));
-                if (q_idx < p.Nq && ok && !*abort_flag) {
+                if (q_idx < p.Nq && (t == 0 || x.tile_b_valid) && ok && !*abort_flag) {
                     const long long r = static_cast<long long>(x.bh) * p.Nq + q_idx;
                     if constexpr (SPLIT) {
                         const long long rs = static_cast<long long>(x.split) * p.B * p.Hq * p.Nq + r;
@@ -919,7 +943,10 @@ attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             if constexpr (SPLIT || FP8 || kOStage) {
                 if ((threadIdx.x & 127) == 0) release_q(qb);
             }
-            const bool do_epilogue = __all_sync(0xffffffffu, ok && !*abort_flag) && q0_t < p.Nq;
+            // (tile B of a single-tile unit writes nothing: its rows belong to the unit's
+            // other half, whose own unit computes them)
+            const bool do_epilogue = __all_sync(0xffffffffu, ok && !*abort_flag) && q0_t < p.Nq &&
+                                     (t == 0 || x.tile_b_valid);
             const float inv_l = l_sum > 0.0f ? 1.0f / l_sum : 0.0f;
             if constexpr (SPLIT) {
                 // Split-KV: this key range's O (normalised by its own row sum) and LSE go

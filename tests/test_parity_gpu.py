@@ -59,6 +59,27 @@ def test_many_units_per_cta_with_idle_tile(Nq, Nk, d, causal):
 
 
 @pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("masked", [False, True])
+def test_single_tile_last_round(d, masked):
+    """154 two-tile units on 148 SMs: the last round's 6 units run as 12
+    single-tile units (both halves of each; the second half of a head's last unit
+    holds rows 2688..2799 of 2800), with key lengths, or with an additive mask
+    broadcast over batch and heads; 400 keys keep the oracle quick."""
+    B, H, N, Nk = 2, 7, 2800, 400
+    q, k, v = make_qkv(B, H, H, N, Nk, d, seed=41 + d + masked)
+    if masked:
+        g = torch.Generator().manual_seed(43)
+        mask = torch.randn(1, 1, N, Nk, generator=g)
+        out, lse = run_gpu(q, k, v, attn_mask=mask)
+        ro, rl, ra = reference(q, k, v, mask=mask.double().numpy())
+    else:
+        lens = torch.tensor([400, 150], dtype=torch.int32)
+        out, lse = run_gpu(q, k, v, key_lens=lens)
+        ro, rl, ra = reference(q, k, v, key_lens=lens.tolist())
+    assert_close(out, lse, ro, rl, rabs=ra)
+
+
+@pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("causal", [False, True])
 def test_key_lens_vs_oracle(d, causal):
     B, H, N = 5, 2, 300
