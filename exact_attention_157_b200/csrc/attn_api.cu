@@ -227,13 +227,13 @@ cudaError_t launch_pp(const CUtensorMap& tq, const CUtensorMap& tk, const CUtens
     FwdParams p = p_in;
     set_fast_divs(p);
     // A last round of two-tile units that would fill at most half the CTAs runs as
-    // single-tile units, two per unit (d = 64, plain and additive-mask launches
-    // without a causal mask; causal ones pair heavy and light units instead).
+    // single-tile units, two per unit (d = 64 without causal or 2-D masks: causal
+    // launches pair heavy and light units instead, and a single tile under a 2-D
+    // mask would still visit the key blocks of both tiles' rectangles).
     const int n_units = p.B * p.Hq * p.n_qtiles * p.n_splits;
     const int tail = static_cast<int>(n_units % static_cast<int>(grid));
-    const bool split_tail = D == 64 && p.n_splits == 1 && !p.is_causal && p.unit_run == 1 && !p.softcap_on &&
-                            p.m2_kind == 0 && n_units > static_cast<int>(grid) && tail > 0 &&
-                            2 * tail <= static_cast<int>(grid);
+    const bool split_tail = D == 64 && p.n_splits == 1 && !p.is_causal && p.unit_run == 1 && p.m2_kind == 0 &&
+                            n_units > static_cast<int>(grid) && tail > 0 && 2 * tail <= static_cast<int>(grid);
     p.n_full_units = split_tail ? n_units - tail : n_units;
     p.n_units_total = split_tail ? n_units + tail : n_units;
     if (p.n_splits > 1)

@@ -264,8 +264,8 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int s, int kv_le
     }
     if (!x.tile_b_valid) x.n_t[1] = 0;
     if (single != 0) {
-        // (only without causal masks and 2-D masks: both tiles of the unit see the
-        // same key blocks, so tile B's count serves the single tile)
+        // (only without causal masks: both tiles of the unit see the same key blocks,
+        // so tile B's count serves the single tile)
         if (single == 2) {
             x.q0 += kBM;
             x.n_t[0] = x.tile_b_valid ? x.n_t[1] : 0;
