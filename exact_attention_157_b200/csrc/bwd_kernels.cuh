@@ -343,27 +343,25 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tc_fence_after();
             const uint32_t st0 = sbase + L::kStages + s * L::kStage + hh * (L::kHalf * 128), st1 = st0 + L::kTile;
             const uint32_t cb = tmem + buf * L::kColBuf;
+            // four K steps of 16 (32 bytes: +2 in descriptor units) per 64-column chunk,
+            // issued by one elected lane per batch; the STFULL commit after the last
             #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t off = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
-                if constexpr (DKDV)
-                    mma_ss_warp(cb, smem_desc_sw128(f0 + off, 16, 1024), smem_desc_sw128(st0 + off, 16, 1024), kIdescS,
-                                kk > 0 ? 1u : 0u);
-                else  // A = Q from TMEM, 16 columns of d (8 TMEM columns) per step
-                    mma_ts_warp(cb, tmem + L::kColFixT + kk * 8, smem_desc_sw128(st0 + off, 16, 1024), kIdescS,
-                                kk > 0 ? 1u : 0u);
+            for (int f = 0; f < 2; ++f) {
+                const uint32_t dst = cb + f * L::kColDP;
+                const uint32_t bs = f == 0 ? st0 : st1;
+                #pragma unroll
+                for (int cc = 0; cc < L::kChunks; ++cc) {
+                    const uint32_t commit = (f == 1 && cc == L::kChunks - 1) ? bar(L::STFULL + buf) : 0u;
+                    const uint64_t bd = smem_desc_sw128(bs + cc * L::kChunkBytes, 16, 1024);
+                    if constexpr (DKDV)
+                        mma_ss_batch_warp<false, 4, 2, 2>(
+                            dst, smem_desc_sw128((f == 0 ? f0 : f1) + cc * L::kChunkBytes, 16, 1024), bd, kIdescS,
+                            cc > 0 ? 1u : 0u, commit);
+                    else  // A = Q (or dO) from TMEM: 16 columns of d = 8 TMEM columns per step
+                        mma_ts4_batch_warp<8, 2>(dst, tmem + L::kColFixT + f * (D / 2) + cc * 32, bd, kIdescS,
+                                                 cc > 0 ? 1u : 0u, commit);
+                }
             }
-            #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t off = (kk >> 2) * L::kChunkBytes + (kk & 3) * 32;
-                if constexpr (DKDV)
-                    mma_ss_warp(cb + L::kColDP, smem_desc_sw128(f1 + off, 16, 1024),
-                                smem_desc_sw128(st1 + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
-                else
-                    mma_ts_warp(cb + L::kColDP, tmem + L::kColFixT + D / 2 + kk * 8,
-                                smem_desc_sw128(st1 + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
-            }
-            mma_commit_warp(bar(L::STFULL + buf));
             return true;
         };
         for (int g = 0; ok && g < 2 && g < n_half; ++g) ok = issue_s(g);
