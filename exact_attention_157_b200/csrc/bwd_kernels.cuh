@@ -410,10 +410,11 @@ attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             my_d = p.delta[r];
         }
         const int key_row = DKDV ? blk * kBN + row : 0;
-        // DKDV: LSE2 and D of each iteration's 128 queries, one value per thread, loaded
-        // before the wait for S^T and dP^T (the loads overlap those products) and shared
-        // through a double buffer (a buffer is rewritten two iterations later, after
-        // every thread has passed the barrier of the iteration between)
+        // DKDV: LSE2 and D of each iteration's 128 queries, one value per thread of the
+        // first warp of each lane quarter, stored at the start of the iteration from
+        // registers loaded one iteration earlier, and shared through a double buffer (a
+        // buffer is rewritten two iterations later, after every thread has passed the
+        // barrier of the iteration between)
         __shared__ __align__(16) float s_l2[2][kBM];
         __shared__ __align__(16) float s_dd[2][kBM];
         // VAR with a 2-D mask: grid coordinates of this iteration's columns (queries
